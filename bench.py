@@ -1,0 +1,374 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input: copy-on-write block
+copies (when the workload has shared blocks), slot mapping, KV append, then paged attention over
+the mixed batch (CUDA-core split-K kernel, tcgen05 prefill tiles when present, log-sum-exp merge).
+The default workload is the LLaMA-13B-shaped fp16 decode batch (64 rows, 40/40 heads, head_dim
+128, context U[128,2048], one appended token per row). Its KV pool is ~1.4 GB, larger than the
+126 MB L2, so no explicit L2 flush is used between steps.
+
+Metric: KV bytes the step must read (every (request, KV head, context token) once as K and once as
+V) divided by the step time, in GB/s; also decode sequence-tokens per second (sum of decode rows'
+context lengths / time). Multi-GPU (torchrun): every rank runs its own replica with its own seed
+(requests are independent: no data-path collective), and the whole-job value divides all ranks'
+bytes by the slowest rank's time.
+
+--impl reference times the CPU oracle (test infrastructure) on a bounded sample of the same
+workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged-attn KV-read GB/s (% of B200 HBM peak) and decode seqs·tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU work of the oracle sample")
+    ap.add_argument("--split-blocks", type=int, default=0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_desc(wl):
+    ctx = np.asarray(wl.prior_lens, np.int64) + np.asarray(list(wl.batch.values()), np.int64)
+    return ctx
+
+
+def kv_bytes(wl) -> int:
+    ctx = workload_desc(wl)
+    eb = 4 if wl.dtype == "f32" else 2
+    return int(ctx[np.asarray(list(wl.batch.values())) > 0].sum()) * wl.num_kv_heads * 2 * wl.head_dim * eb
+
+
+def decode_seq_tokens(wl) -> int:
+    ctx = workload_desc(wl)
+    n = np.asarray(list(wl.batch.values()))
+    return int(ctx[n == 1].sum())
+
+
+def decode_kernel_bytes(wl) -> int:
+    """Algorithmic bytes of the CUDA-core kernel per launch: K+V of every decode row's (request, KV
+    head) context, plus its q rows read and output rows written."""
+    ctx = workload_desc(wl)
+    n = np.asarray(list(wl.batch.values()))
+    eb = 4 if wl.dtype == "f32" else 2
+    dec = n == 1
+    kv = int(ctx[dec].sum()) * wl.num_kv_heads * 2 * wl.head_dim * eb
+    qo = int(dec.sum()) * wl.num_q_heads * wl.head_dim * eb * 2
+    return kv + qo
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = bus_id
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(", ") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        if self.bus_id:
+            mine = [r for r in rows if len(r) > 1 and r[1].strip().lower().endswith(self.bus_id.lower()[-12:])]
+            rows = mine or rows
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[2]))
+                mx.append(float(r[3]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, r[6:10]):
+                if val.strip().lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def bus_id_of(dev) -> str | None:
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+def run_oracle_sample(wl, h, target_seconds: float):
+    """The oracle, as it stands, on the first m requests (all heads, all rows) of the step, with the
+    step's own KV append applied first. Returns dict(value_gbs, seconds, requests, cores, bytes)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    qsl, ctx = oracle.flatten_batch(wl.batch, wl.prior_lens)
+    counts = np.asarray(list(wl.batch.values()), np.int64)
+    if wl.write_batch:
+        wcounts = np.asarray([wl.write_batch.get(r, 0) for r in wl.batch.keys()], np.int64)
+        wqsl, wctx = oracle.flatten_batch(dict(zip(wl.batch.keys(), wcounts)), ctx.astype(np.int64) - wcounts)
+        if len(wl.copy_pairs):
+            oracle.copy_blocks([h["k_pool"]], [h["v_pool"]], wl.copy_pairs)
+        slots = oracle.slot_mapping(wl.block_tables, wqsl, wctx)
+        oracle.kv_cache_write(h["k_new"], h["v_new"], h["k_pool"], h["v_pool"], slots)
+    eb = 4 if wl.dtype == "f32" else 2
+    per_req = ctx.astype(np.int64) * wl.num_kv_heads * 2 * wl.head_dim * eb
+    order = [r for r in range(len(ctx)) if counts[r] > 0]
+
+    def run(m):
+        rows = np.concatenate([np.arange(qsl[r], qsl[r + 1]) for r in order[:m]]).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.paged_attention(h["q"], h["k_pool"], h["v_pool"], wl.block_tables, ctx, qsl, wl.scale, wl.dtype,
+                               rows=rows, nthreads=cores)
+        return time.perf_counter() - t0, int(per_req[order[:m]].sum())
+
+    m = 1
+    dt, by = run(m)
+    while dt < target_seconds * 0.3 and m < len(order):
+        m = min(len(order), max(m + 1, int(m * min(8.0, target_seconds / max(dt, 1e-3)))))
+        dt, by = run(m)
+    return {"value_gbs": by / dt / 1e9, "seconds": dt, "requests": m, "of": len(order), "cores": cores, "bytes": by}
+
+
+def storage(t):
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float32:
+        return t.numpy().copy()
+    return t.view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    from paged_kv_cache_446_b200 import workloads as W
+    wl = W.make(args.config, device="cpu")
+    h = {k: storage(getattr(wl, k)) for k in ("q", "k_pool", "v_pool", "k_new", "v_new")}
+    per_step = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    samples = []
+    for i in range(args.warmup + args.steps):
+        hh = {k: v.copy() for k, v in h.items()} if (wl.write_batch or len(wl.copy_pairs)) else h
+        r = run_oracle_sample(wl, hh, per_step)
+        if i >= args.warmup:
+            samples.append(r)
+    secs = sum(s["seconds"] for s in samples)
+    by = sum(s["bytes"] for s in samples)
+    value = by / secs / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(samples),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) q/k/v; seeded block placement)",
+            "config": {"workload": wl.name, "requests_per_step_sample": samples[-1]["requests"],
+                       "requests": samples[-1]["of"]},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": samples[-1]["cores"], "kind": "oracle",
+                             "sample": f"first {samples[-1]['requests']} of {samples[-1]['of']} requests of "
+                                       f"{wl.name} per step (all heads and rows, after the step's KV append)"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from paged_kv_cache_446_b200 import pkv
+    from paged_kv_cache_446_b200 import workloads as W
+    from paged_kv_cache_446_b200.step import PagedAttentionStep
+
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    seed = 1000 + int(args.config[1]) + 100 * rank
+    wl = W.make(args.config, device=dev, seed=seed)
+    dt = W.TORCH_DTYPES[wl.dtype]
+    opts = {"split_blocks": args.split_blocks} if args.split_blocks else {}
+    step = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,
+                              wl.num_kv_heads, wl.head_dim, dt, dev, write_batch=wl.write_batch or None,
+                              copy_pairs=wl.copy_pairs, **opts)
+    out = torch.empty_like(wl.q)
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        h = {k: storage(getattr(wl, k)) for k in ("q", "k_pool", "v_pool", "k_new", "v_new")}
+        r = run_oracle_sample(wl, h, args.cpu_seconds)
+        del h
+        cpu_baseline = {"value": r["value_gbs"], "unit": "GB/s", "cores": r["cores"], "kind": "oracle",
+                        "sample": f"first {r['requests']} of {r['of']} requests of {wl.name} (all heads and rows, "
+                                  f"after the step's KV append), {r['seconds']:.1f} s"}
+
+    def run_step():
+        step.run(wl.q, wl.k_pool, wl.v_pool, wl.scale, wl.k_new, wl.v_new, out=out)
+
+    for _ in range(args.warmup):
+        run_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler(bus_id_of(dev)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pkv.profile_start(capacity=16 * args.steps + 16)
+    ev0.record()
+    for _ in range(args.steps):
+        run_step()
+    ev1.record()
+    torch.cuda.synchronize()
+    prof = pkv.profile_stop()
+    ms_total = ev0.elapsed_time(ev1)
+    clocks = sampler.stop() if sampler else None
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_per_step = float(t.item()) / args.steps
+    code, detail = pkv.device_error()
+    assert code == 0, f"device error {code} at {detail}"
+
+    # ---- end to end through the public API: pinned host inputs in, output back to the host ----
+    e2e = None
+    if not args.no_e2e:
+        hq = wl.q.cpu().pin_memory()
+        hkn = wl.k_new.cpu().pin_memory()
+        hvn = wl.v_new.cpu().pin_memory()
+        hbt = torch.from_numpy(wl.block_tables).pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dq, dkn, dvn = torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new)
+        ws = step.plan.workspace
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dkn.copy_(hkn, non_blocking=True)
+            dvn.copy_(hvn, non_blocking=True)
+            step.block_tables.copy_(hbt, non_blocking=True)
+            step.plan = pkv.AttentionPlan(wl.batch, wl.prior_lens, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, dt,
+                                          dev, workspace=ws, **opts)
+            step.run(dq, wl.k_pool, wl.v_pool, wl.scale, dkn, dvn, out=out)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item()) / args.steps
+        h2d = (hq.numel() * hq.element_size() + hkn.numel() * hkn.element_size() + hvn.numel() * hvn.element_size()
+               + hbt.numel() * 4 + int(step.plan.plan.meta_bytes) + 2 * 4 * (len(wl.batch) + 1))
+        d2h = hout.numel() * hout.element_size()
+        e2e = {"value": world * kv_bytes(wl) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak, peak_kind = peaks()
+    value = world * kv_bytes(wl) / (ms_per_step * 1e-3) / 1e9
+    dec_ms, dec_n = prof["decode"]
+    roof = None
+    if dec_n:
+        dec_avg_ms = dec_ms / dec_n
+        achieved = decode_kernel_bytes(wl) / (dec_avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None, "kernel": "decode_kernel (CUDA-core split-K)", "kernel_ms": dec_avg_ms,
+                "peak_source": f"{peak_kind} hbm_gbs (burst copy)"}
+    launches = sum(v[1] for k, v in prof.items() if k != "dropped")
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) q/k/v drawn on the device; seeded random block placement)",
+        "config": {"workload": wl.name, "requests": len(wl.batch), "num_q_heads": wl.num_q_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
+                   "num_blocks": wl.num_blocks, "kv_bytes_per_step_per_gpu": kv_bytes(wl),
+                   "l2": "inputs larger than L2 (KV pool read per step >> 126 MB); no flush",
+                   "parallelism": f"replicas x{world} (independent requests per GPU)"},
+        "frac_of_hbm_peak": value / world / peak,
+        "decode_seq_tokens_per_s": world * decode_seq_tokens(wl) / (ms_per_step * 1e-3),
+        "decode_steps_per_s": 1e3 / ms_per_step,
+        "kernel_ms_per_step": {k: v[0] / max(1, args.steps) for k, v in prof.items() if k != "dropped"},
+        "roofline": roof,
+        "cpu_baseline": cpu_baseline,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

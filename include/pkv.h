@@ -1,0 +1,245 @@
+/*
+ * pkv.h -- C ABI of a B200 (sm_100a) PagedAttention library.
+ *
+ * The KV cache lives in one pool of fixed 16-token blocks; each request owns an ordered table of
+ * physical block ids; attention reads K and V block by block through that table and returns what
+ * contiguous storage would (blog.mckayzhao.com/?p=56, "PagedAttention：操作系统课本里翻出来的灵感";
+ * 一文搞懂vLLM：为啥它能让一张GPU扛住几十倍用户？, "PagedAttention：核心思路").
+ *
+ * Conventions for every call:
+ *   - Device pointers are caller-owned (typically torch tensors); the library allocates no device
+ *     memory. Host pointers are read during the call only.
+ *   - Kernels run asynchronously on the caller's stream `stream` (0 = legacy default stream).
+ *   - Argument errors are detected on the host before any launch and returned as a pkv_status;
+ *     no call traps on the device. Kernels that find an out-of-range block id or slot at run time
+ *     skip that access and record the first such event in a device error word read by
+ *     pkv_device_error(). Bounded waits that expire record PKV_ERR_DEVICE_TIMEOUT there.
+ *   - The element type (pkv_dtype) is the same for q, k, v, new K/V and the output.
+ *
+ * Layouts (row-major, element counts):
+ *   q, out          [T, Hq, D]                 T = query rows of the batch
+ *   k_pool, v_pool  [num_blocks, Hkv, 16, D]   one (block, kv head) is a contiguous 16*D run
+ *   k_new, v_new    [T_new, Hkv, D]
+ *   block_tables    int32 [R, max_blocks_per_seq]; entries past ceil(context/16) are ignored
+ *   context_lens    int32 [R]   tokens in the cache after this step's tokens are appended
+ *   query_start_loc int32 [R+1] prefix sum of the step's {request_id: num_tokens} counts
+ *   slot_mapping    int64 [T_new] physical slot = block_id * 16 + offset; negative = skip
+ * Query head h reads KV head h / (Hq / Hkv). Row j of a request with n rows and context ctx sits
+ * at position ctx - n + j and attends keys 0 .. ctx - n + j.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* pkv_stream_t; /* same handle as cudaStream_t */
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,          /* a null pointer, a negative size, an inconsistent batch */
+    PKV_ERR_UNSUPPORTED = 2,          /* a shape or type this build does not handle */
+    PKV_ERR_CUDA = 3,                 /* a CUDA runtime call failed; see pkv_last_error() */
+    PKV_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below what the plan needs */
+    PKV_ERR_DEVICE_TIMEOUT = 5,       /* a kernel's bounded wait expired (device error word only) */
+    PKV_ERR_DEVICE_RANGE = 6          /* a kernel met an out-of-range id (device error word only) */
+} pkv_status;
+
+typedef enum pkv_dtype { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+
+#define PKV_BLOCK_SIZE 16
+#define PKV_PLAN_MAGIC 0x706b7631u /* "pkv1" */
+
+/* Human-readable name of a status (static storage). */
+const char* pkv_status_string(pkv_status s);
+/* Message of the last failing call on this host thread (static thread-local storage). */
+const char* pkv_last_error(void);
+/* Library version string. */
+const char* pkv_version(void);
+
+/*
+ * pkv_slot_mapping -- physical slot of every token this step appends.
+ * Source: 一文搞懂vLLM, "快速回顾 prefill、decode 和 KV cache" (every processed token adds one K/V entry)
+ * and "PagedAttention：核心思路" (a new block is used once the previous one is full, tracked in the
+ * request's block table); blog.mckayzhao.com/?p=56, "PagedAttention" section (table = logical ->
+ * physical map). Row j of request r lands at position p = ctx_r - n_r + j and
+ *   slot = block_tables[r][p / 16] * 16 + p % 16.
+ * Device inputs: block_tables [R, max_blocks_per_seq], query_start_loc [R+1], context_lens [R].
+ * Device output: slot_mapping [num_tokens] (num_tokens = query_start_loc[R], given by the caller).
+ * A table entry outside [0, num_blocks) yields slot -1 and sets the device error word.
+ * Errors: INVALID_ARG for null pointers (with num_tokens > 0) or negative sizes.
+ */
+pkv_status pkv_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq, const int32_t* query_start_loc,
+                            const int32_t* context_lens, int num_reqs, int num_blocks, int64_t* slot_mapping,
+                            int num_tokens, pkv_stream_t stream);
+
+/*
+ * pkv_kv_cache_write -- append new K/V rows into their slots:
+ *   k_pool[slot / 16][h][slot % 16][:] = k_new[t][h][:]   (same for V), for every slot >= 0.
+ * Source: 一文搞懂vLLM, "快速回顾 prefill、decode 和 KV cache" (the cache grows by one entry per token).
+ * Slots must be distinct within one call (else which row lands is unspecified); slots at or
+ * beyond num_blocks * 16 are skipped and set the device error word. Bit-exact copy.
+ * Errors: INVALID_ARG (null pointer with num_tokens > 0, negative sizes), UNSUPPORTED
+ * (block_size != 16, head_dim * element size not a multiple of 16 bytes or above 1024 bytes).
+ */
+pkv_status pkv_kv_cache_write(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                              const int64_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads,
+                              int head_dim, int block_size, pkv_dtype dtype, pkv_stream_t stream);
+
+/*
+ * pkv_copy_blocks -- copy-on-write block copy: for every layer l and every (src, dst) pair,
+ * block dst of k_pools[l] and of v_pools[l] (all KV heads) becomes a copy of block src.
+ * Source: blog.mckayzhao.com/?p=56, "还不止是分页：Copy-on-Write 和内存共享" (copy the shared block,
+ * modify the copy, leave the original unchanged); 一文搞懂vLLM, "PagedAttention 是怎么共享内存的".
+ * k_pools, v_pools: HOST arrays of num_layers device pointers, each [num_blocks, Hkv, 16, D].
+ * block_mapping: DEVICE int32 [num_pairs][2] = (src, dst). Preconditions: no dst repeats and no
+ * dst is also a src in the same call; src == dst is a no-op; ids outside [0, num_blocks) are
+ * skipped and set the device error word. Bit-exact.
+ * Errors: INVALID_ARG (null pointers, negative sizes), UNSUPPORTED (block_size != 16).
+ */
+pkv_status pkv_copy_blocks(void* const* k_pools, void* const* v_pools, int num_layers,
+                           const int32_t* block_mapping, int num_pairs, int num_blocks, int num_kv_heads,
+                           int head_dim, int block_size, pkv_dtype dtype, pkv_stream_t stream);
+
+/* Planner knobs (all zero = defaults). */
+typedef struct pkv_plan_options {
+    int32_t split_blocks;      /* >0: decode/support rows are cut into chunks of this many blocks;
+                                  0: chosen from the batch size and the SM count */
+    int32_t no_split;          /* 1: every row is one chunk (no log-sum-exp merge) */
+    int32_t cuda_core_only;    /* 1: multi-row requests also go to the CUDA-core path (no tcgen05) */
+    int32_t num_sms;           /* SM count the chunking targets; 0 = query the current device
+                                  (pkv_attention_plan) or 148 (pkv_attention_plan_host) */
+} pkv_plan_options;
+
+/*
+ * Host description of a planned batch (caller-owned memory, filled by the planner). The work
+ * lists themselves live in the caller's device workspace at the byte offsets below.
+ */
+typedef struct pkv_plan {
+    uint32_t magic;              /* PKV_PLAN_MAGIC once filled */
+    int32_t num_reqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim, dtype;
+    int32_t num_decode_rows;     /* rows served by the CUDA-core split-K kernel */
+    int32_t num_prefill_rows;    /* rows served by the tcgen05 tile kernel */
+    int32_t num_items;           /* CUDA-core work items (row, kv head, block chunk) */
+    int32_t num_tiles;           /* tcgen05 tiles (request, kv head, 128 packed rows) */
+    int32_t num_merge_rows;      /* (row, kv head) pairs merged from several chunks */
+    int32_t num_partials;        /* chunk partial results in the workspace */
+    int32_t split_blocks;        /* chunk length in blocks used for this batch */
+    int32_t max_blocks;          /* longest context in blocks */
+    int64_t off_items, off_tiles, off_merge, off_part_o, off_part_ml; /* byte offsets into workspace */
+    int64_t meta_bytes;          /* bytes uploaded by pkv_attention_plan (work lists) */
+    int64_t ws_bytes;            /* total workspace bytes this plan needs */
+    int64_t kv_bytes;            /* algorithmic K+V bytes read: sum over rows' attended keys of
+                                    2*D*elem per (kv head, key), counted once per (request, kv head)
+                                    for decode rows and once per request for prefill rows */
+    int64_t attn_flops;          /* 4*D per (query row, query head, attended key) */
+} pkv_plan;
+
+/*
+ * pkv_attention_workspace_size -- bytes of device workspace pkv_attention_plan will need for this
+ * batch (same host inputs as the planner). Host-only; does not touch the GPU unless
+ * opts->num_sms == 0, in which case it reads the current device's SM count.
+ */
+pkv_status pkv_attention_workspace_size(const int32_t* h_query_start_loc, const int32_t* h_context_lens,
+                                        int num_reqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                        pkv_dtype dtype, const pkv_plan_options* opts, size_t* bytes);
+
+/*
+ * pkv_attention_plan_host -- split the batch into work lists on the host, without any CUDA call.
+ * Source for the batch: blog.mckayzhao.com/?p=56, "V1 架构：推倒重来的勇气" (one step = a dict
+ * {request_id: num_tokens}; decode rows and chunked-prefill rows share the batch) and "进阶特性"
+ * (chunked prefill). Rows with num_tokens == 1 become decode work; requests with more rows go to
+ * the tcgen05 tile kernel when dtype is f16/bf16, head_dim is 128 and Hq/Hkv divides 128 (otherwise
+ * to the CUDA-core kernel, one row at a time with its causal limit). Long rows are cut into
+ * chunks whose partial results a log-sum-exp merge combines.
+ * h_meta (host, meta_capacity bytes) receives the image that pkv_attention_plan uploads to the
+ * start of the workspace; pass NULL to only fill *plan.
+ * Errors: INVALID_ARG (query_start_loc not starting at 0 or decreasing, context < num_tokens,
+ * num_tokens > 0 with context 0, Hq % Hkv != 0), UNSUPPORTED (head_dim not 64/128, Hq/Hkv > 16),
+ * WORKSPACE_TOO_SMALL (meta_capacity below plan->meta_bytes).
+ */
+pkv_status pkv_attention_plan_host(const int32_t* h_query_start_loc, const int32_t* h_context_lens, int num_reqs,
+                                   int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
+                                   const pkv_plan_options* opts, void* h_meta, size_t meta_capacity,
+                                   pkv_plan* plan);
+
+/*
+ * pkv_attention_plan -- pkv_attention_plan_host, then one cudaMemcpyAsync of the work lists into
+ * d_workspace on `stream`. A plan stays valid for any number of pkv_paged_attention calls on the
+ * same batch shape (e.g. every layer of a model step) while the workspace is not reused.
+ * Errors: as pkv_attention_plan_host, plus WORKSPACE_TOO_SMALL (ws_bytes < plan->ws_bytes) and CUDA.
+ */
+pkv_status pkv_attention_plan(const int32_t* h_query_start_loc, const int32_t* h_context_lens, int num_reqs,
+                              int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
+                              const pkv_plan_options* opts, void* d_workspace, size_t ws_bytes, pkv_plan* plan,
+                              pkv_stream_t stream);
+
+/*
+ * pkv_paged_attention -- attention for every row of a planned mixed batch.
+ * Source: blog.mckayzhao.com/?p=56, "PagedAttention：操作系统课本里翻出来的灵感" (find each block
+ * through the table, read K and V block by block; same result as contiguous storage) and
+ * "V1 架构：推倒重来的勇气" (decode and chunked-prefill rows in one batch).
+ *   out[row][h][:] = sum_t softmax_t(scale * q[row][h] . K_r[t]) V_r[t],  t = 0 .. ctx_r - n_r + j
+ * with K_r[t] = k_pool[block_tables[r][t/16]][h / (Hq/Hkv)][t%16]. Softmax and accumulation in fp32;
+ * the output is rounded to the element type. Launches, on `stream`: the tcgen05 prefill tile
+ * kernel (if the plan has tiles), the CUDA-core split-K kernel (if it has items) and the
+ * log-sum-exp merge kernel (if it has merge rows). The plan and workspace must come from
+ * pkv_attention_plan with the same batch; q/out shapes must match it.
+ * Errors: INVALID_ARG (null pointers, plan magic/shape mismatch), WORKSPACE_TOO_SMALL, CUDA.
+ */
+pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                               const int32_t* query_start_loc, int num_blocks, float scale, const pkv_plan* plan,
+                               void* d_workspace, size_t ws_bytes, pkv_stream_t stream);
+
+/*
+ * Host-side validators (no CUDA calls). They check the preconditions the kernels rely on and
+ * return INVALID_ARG with a message in pkv_last_error() on the first violation.
+ *   pkv_validate_tables: for every request, entries [0, ceil(ctx/16)) lie in [0, num_blocks) and
+ *     ceil(ctx/16) <= max_blocks_per_seq.
+ *   pkv_validate_slots: every slot >= 0 is below num_blocks*16 and no slot repeats.
+ *   pkv_validate_copy_pairs: ids in range, no dst repeats, no dst is also a src.
+ */
+pkv_status pkv_validate_tables(const int32_t* h_block_tables, const int32_t* h_context_lens, int num_reqs,
+                               int max_blocks_per_seq, int num_blocks);
+pkv_status pkv_validate_slots(const int64_t* h_slot_mapping, int num_tokens, int num_blocks);
+pkv_status pkv_validate_copy_pairs(const int32_t* h_pairs, int num_pairs, int num_blocks);
+
+/*
+ * pkv_device_error -- read and clear the device error word of the current device (synchronises
+ * `stream`). *code receives PKV_OK or the first PKV_ERR_DEVICE_* recorded since the last read;
+ * *detail receives the offending index (or -1).
+ */
+pkv_status pkv_device_error(int* code, int64_t* detail, pkv_stream_t stream);
+
+/*
+ * Kernel timing (no counterpart on the pages; a measurement aid). Between pkv_profile_start and
+ * pkv_profile_stop, every kernel the library launches on the calling host thread is bracketed by
+ * a pair of CUDA events recorded on the launch stream. pkv_profile_stop synchronises those events,
+ * writes per-kind totals (milliseconds) and launch counts into arrays of PKV_KERNEL_KINDS entries,
+ * and stops recording. At most `capacity` launches are timed; later ones are counted but not
+ * timed (*dropped receives how many). Events are created on the current device at start.
+ * Errors: INVALID_ARG (capacity < 1, null outputs, stop without start), CUDA.
+ */
+typedef enum pkv_kernel_kind {
+    PKV_KERNEL_SLOT_MAPPING = 0,
+    PKV_KERNEL_KV_WRITE = 1,
+    PKV_KERNEL_COPY_BLOCKS = 2,
+    PKV_KERNEL_DECODE = 3,
+    PKV_KERNEL_MERGE = 4,
+    PKV_KERNEL_PREFILL_TC = 5,
+    PKV_KERNEL_KINDS = 6
+} pkv_kernel_kind;
+
+pkv_status pkv_profile_start(int capacity);
+pkv_status pkv_profile_stop(double* total_ms, int* launches, int* dropped);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

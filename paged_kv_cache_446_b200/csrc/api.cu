@@ -1,0 +1,558 @@
+// C ABI entry points (include/pkv.h): argument checks, the host planner and kernel launches.
+#include <algorithm>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+#include "pkv.h"
+
+namespace pkv {
+
+__device__ DeviceError g_device_error;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+pkv_status fail(pkv_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+pkv_status fail(pkv_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return s;
+}
+
+pkv_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(PKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int elem_bytes(pkv_dtype dt) { return dt == PKV_F32 ? 4 : 2; }
+bool dtype_ok(int dt) { return dt == PKV_F32 || dt == PKV_F16 || dt == PKV_BF16; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t align256(int64_t x) { return (x + 255) / 256 * 256; }
+
+int current_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+// Work lists of one batch, before they are written into the metadata image.
+struct PlanLists {
+    std::vector<DecodeItem> items;
+    std::vector<PrefillTile> tiles;
+    std::vector<MergeRow> merges;
+    int num_partials = 0;
+};
+
+// Query rows per tcgen05 tile: the 128 MMA rows hold (128 / G) consecutive query rows x G heads.
+int tile_tokens(int group) { return 128 / group; }
+
+pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int Hkv, int D, pkv_dtype dt,
+                      const pkv_plan_options* opts, int num_sms, PlanLists* L, pkv_plan* plan) {
+    if (!qsl || (R > 0 && !ctx) || !plan) return fail(PKV_ERR_INVALID_ARG, "null planner argument");
+    if (R < 0) return fail(PKV_ERR_INVALID_ARG, "num_reqs < 0");
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)", Hq, Hkv);
+    if (D != 64 && D != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", D);
+    if (!dtype_ok(dt)) return fail(PKV_ERR_INVALID_ARG, "bad dtype %d", (int)dt);
+    const int G = Hq / Hkv;
+    if (qsl[0] != 0) return fail(PKV_ERR_INVALID_ARG, "query_start_loc[0] = %d, expected 0", qsl[0]);
+    for (int r = 0; r < R; ++r) {
+        const int n = qsl[r + 1] - qsl[r];
+        if (n < 0) return fail(PKV_ERR_INVALID_ARG, "query_start_loc decreases at request %d", r);
+        if (ctx[r] < n) return fail(PKV_ERR_INVALID_ARG, "request %d: context_len %d < num_tokens %d", r, ctx[r], n);
+        if (n > 0 && ctx[r] < 1) return fail(PKV_ERR_INVALID_ARG, "request %d: empty context with query rows", r);
+    }
+    pkv_plan_options o{};
+    if (opts) o = *opts;
+    const bool tc_ok = !o.cuda_core_only && prefill_tc_supported((int)dt, D, G);
+    const int eb = elem_bytes(dt);
+
+    struct CoreRow { int row, req, limit; };
+    std::vector<CoreRow> core_rows;
+    int64_t kv_bytes = 0, flops = 0;
+    int decode_rows = 0, prefill_rows = 0, max_blocks = 0;
+    for (int r = 0; r < R; ++r) {
+        const int n = qsl[r + 1] - qsl[r];
+        if (n == 0) continue;
+        const int P = ctx[r] - n;
+        max_blocks = std::max<int>(max_blocks, (int)ceil_div(ctx[r], kBlockSize));
+        kv_bytes += (int64_t)ctx[r] * Hkv * 2 * D * eb;
+        // keys attended: sum_j (P + j + 1)
+        flops += 4LL * D * Hq * ((int64_t)n * P + (int64_t)n * (n + 1) / 2);
+        if (n > 1 && tc_ok) {
+            prefill_rows += n;
+            const int tt = tile_tokens(G);
+            for (int h = 0; h < Hkv; ++h)
+                for (int t0 = 0; t0 < n; t0 += tt) {
+                    const int last = std::min(n, t0 + tt);
+                    const int keys = P + last;  // keys visible to the tile's last row
+                    L->tiles.push_back(PrefillTile{r, h, t0, (int)ceil_div(keys, 128)});
+                }
+        } else {
+            if (n == 1) ++decode_rows;
+            for (int j = 0; j < n; ++j) core_rows.push_back(CoreRow{qsl[r] + j, r, P + j + 1});
+        }
+    }
+    // Chunk length: enough items for ~4 per resident warp, but never below 8 blocks.
+    const int groups = (int)ceil_div(G, kMaxGroupPerItem);
+    int64_t total_blocks = 0;
+    for (const CoreRow& c : core_rows) total_blocks += ceil_div(c.limit, kBlockSize) * Hkv * groups;
+    int chunk;
+    if (o.no_split) chunk = 1 << 30;
+    else if (o.split_blocks > 0) chunk = o.split_blocks;
+    else {
+        const int64_t workers = (int64_t)std::max(num_sms, 1) * 8;
+        chunk = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(total_blocks, workers * 4), 8), 1 << 20);
+    }
+    for (const CoreRow& c : core_rows) {
+        const int nb = (int)ceil_div(c.limit, kBlockSize);
+        const int pieces = (int)ceil_div(nb, chunk);
+        for (int h = 0; h < Hkv; ++h)
+            for (int g0 = 0; g0 < G; g0 += kMaxGroupPerItem) {
+                int first = -1;
+                if (pieces > 1) {
+                    first = L->num_partials;
+                    L->num_partials += pieces;
+                    L->merges.push_back(MergeRow{c.row, h * G + g0, std::min(kMaxGroupPerItem, G - g0), first, pieces, {0, 0, 0}});
+                }
+                for (int p = 0; p < pieces; ++p) {
+                    const int b0 = p * chunk, b1 = std::min(nb, b0 + chunk);
+                    L->items.push_back(DecodeItem{c.row, c.req, h, g0, b0, b1, c.limit, pieces > 1 ? first + p : -1});
+                }
+            }
+    }
+    // Longest work first: balances the static round-robin over persistent warps / CTAs.
+    std::stable_sort(L->items.begin(), L->items.end(), [](const DecodeItem& a, const DecodeItem& b) {
+        return (a.blk_end - a.blk_begin) > (b.blk_end - b.blk_begin);
+    });
+    std::stable_sort(L->tiles.begin(), L->tiles.end(),
+                     [](const PrefillTile& a, const PrefillTile& b) { return a.key_tiles > b.key_tiles; });
+
+    std::memset(plan, 0, sizeof *plan);
+    plan->magic = PKV_PLAN_MAGIC;
+    plan->num_reqs = R;
+    plan->num_q_tokens = R > 0 ? qsl[R] : 0;
+    plan->num_q_heads = Hq;
+    plan->num_kv_heads = Hkv;
+    plan->head_dim = D;
+    plan->dtype = (int32_t)dt;
+    plan->num_decode_rows = decode_rows;
+    plan->num_prefill_rows = prefill_rows;
+    plan->num_items = (int32_t)L->items.size();
+    plan->num_tiles = (int32_t)L->tiles.size();
+    plan->num_merge_rows = (int32_t)L->merges.size();
+    plan->num_partials = L->num_partials;
+    plan->split_blocks = chunk;
+    plan->max_blocks = max_blocks;
+    int64_t off = 256;  // first 256 bytes reserved
+    plan->off_items = off;
+    off = align256(off + (int64_t)L->items.size() * sizeof(DecodeItem));
+    plan->off_tiles = off;
+    off = align256(off + (int64_t)L->tiles.size() * sizeof(PrefillTile));
+    plan->off_merge = off;
+    off = align256(off + (int64_t)L->merges.size() * sizeof(MergeRow));
+    plan->meta_bytes = off;
+    plan->off_part_o = off;
+    off = align256(off + (int64_t)L->num_partials * kMaxGroupPerItem * D * 4);
+    plan->off_part_ml = off;
+    off = align256(off + (int64_t)L->num_partials * kMaxGroupPerItem * 2 * 4);
+    plan->ws_bytes = off;
+    plan->kv_bytes = kv_bytes;
+    plan->attn_flops = flops;
+    return PKV_OK;
+}
+
+void write_meta(const PlanLists& L, const pkv_plan& plan, unsigned char* meta) {
+    std::memset(meta, 0, (size_t)plan.meta_bytes);
+    if (!L.items.empty()) std::memcpy(meta + plan.off_items, L.items.data(), L.items.size() * sizeof(DecodeItem));
+    if (!L.tiles.empty()) std::memcpy(meta + plan.off_tiles, L.tiles.data(), L.tiles.size() * sizeof(PrefillTile));
+    if (!L.merges.empty()) std::memcpy(meta + plan.off_merge, L.merges.data(), L.merges.size() * sizeof(MergeRow));
+}
+
+// Per-thread kernel timing state (pkv_profile_start / pkv_profile_stop).
+struct Profiler {
+    bool on = false;
+    std::vector<cudaEvent_t> ev;  // 2 per record
+    std::vector<int> kind;
+    int used = 0;
+    int launches[PKV_KERNEL_KINDS] = {0};
+    int dropped = 0;
+};
+thread_local Profiler t_prof;
+
+// Brackets one launch with events when profiling is on.
+struct ProfileScope {
+    int slot = -1;
+    cudaStream_t s;
+    ProfileScope(int k, cudaStream_t stream) : s(stream) {
+        if (!t_prof.on) return;
+        t_prof.launches[k]++;
+        if (t_prof.used * 2 + 1 >= (int)t_prof.ev.size()) {
+            t_prof.dropped++;
+            return;
+        }
+        slot = t_prof.used++;
+        t_prof.kind[slot] = k;
+        cudaEventRecord(t_prof.ev[2 * slot], s);
+    }
+    ~ProfileScope() {
+        if (slot >= 0) cudaEventRecord(t_prof.ev[2 * slot + 1], s);
+    }
+};
+
+}  // namespace
+
+DeviceError* device_error_word() {
+    static std::mutex mu;
+    static DeviceError* addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<DeviceError*>(p);
+    }
+    return addr[dev];
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+const char* pkv_status_string(pkv_status s) {
+    switch (s) {
+        case PKV_OK: return "ok";
+        case PKV_ERR_INVALID_ARG: return "invalid argument";
+        case PKV_ERR_UNSUPPORTED: return "unsupported";
+        case PKV_ERR_CUDA: return "CUDA error";
+        case PKV_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case PKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case PKV_ERR_DEVICE_RANGE: return "device index out of range";
+    }
+    return "unknown status";
+}
+
+const char* pkv_last_error(void) { return t_last_error.c_str(); }
+
+const char* pkv_version(void) { return "pkv 0.1 sm_100a"; }
+
+pkv_status pkv_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq, const int32_t* query_start_loc,
+                            const int32_t* context_lens, int num_reqs, int num_blocks, int64_t* slot_mapping,
+                            int num_tokens, pkv_stream_t stream) {
+    if (num_reqs < 0 || num_tokens < 0 || max_blocks_per_seq < 0 || num_blocks < 0)
+        return fail(PKV_ERR_INVALID_ARG, "negative size");
+    if (num_tokens == 0 || num_reqs == 0) return PKV_OK;
+    if (!block_tables || !query_start_loc || !context_lens || !slot_mapping)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    DeviceError* err = device_error_word();
+    if (!err) return fail(PKV_ERR_CUDA, "device error word unavailable");
+    ProfileScope prof(PKV_KERNEL_SLOT_MAPPING, (cudaStream_t)stream);
+    cudaError_t e = launch_slot_mapping(block_tables, max_blocks_per_seq, query_start_loc, context_lens, num_reqs,
+                                        num_blocks, slot_mapping, num_tokens, err, (cudaStream_t)stream);
+    return e == cudaSuccess ? PKV_OK : cuda_fail(e, "slot_mapping launch");
+}
+
+pkv_status pkv_kv_cache_write(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                              const int64_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads,
+                              int head_dim, int block_size, pkv_dtype dtype, pkv_stream_t stream) {
+    if (num_tokens < 0 || num_blocks < 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return fail(PKV_ERR_INVALID_ARG, "bad size");
+    if (!dtype_ok(dtype)) return fail(PKV_ERR_INVALID_ARG, "bad dtype");
+    if (block_size != kBlockSize) return fail(PKV_ERR_UNSUPPORTED, "block_size %d (only 16)", block_size);
+    const int row = head_dim * elem_bytes(dtype);
+    if (row % 16 != 0 || row > 1024) return fail(PKV_ERR_UNSUPPORTED, "row of %d bytes", row);
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_new || !v_new || !k_pool || !v_pool || !slot_mapping) return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    if (((uintptr_t)k_new | (uintptr_t)v_new | (uintptr_t)k_pool | (uintptr_t)v_pool) & 15)
+        return fail(PKV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    DeviceError* err = device_error_word();
+    if (!err) return fail(PKV_ERR_CUDA, "device error word unavailable");
+    ProfileScope prof(PKV_KERNEL_KV_WRITE, (cudaStream_t)stream);
+    cudaError_t e = launch_kv_write(k_new, v_new, k_pool, v_pool, slot_mapping, num_tokens, num_blocks, num_kv_heads,
+                                    row, err, (cudaStream_t)stream);
+    return e == cudaSuccess ? PKV_OK : cuda_fail(e, "kv_cache_write launch");
+}
+
+pkv_status pkv_copy_blocks(void* const* k_pools, void* const* v_pools, int num_layers, const int32_t* block_mapping,
+                           int num_pairs, int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                           pkv_dtype dtype, pkv_stream_t stream) {
+    if (num_layers < 0 || num_pairs < 0 || num_blocks < 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return fail(PKV_ERR_INVALID_ARG, "bad size");
+    if (!dtype_ok(dtype)) return fail(PKV_ERR_INVALID_ARG, "bad dtype");
+    if (block_size != kBlockSize) return fail(PKV_ERR_UNSUPPORTED, "block_size %d (only 16)", block_size);
+    const long long bb = (long long)num_kv_heads * kBlockSize * head_dim * elem_bytes(dtype);
+    if (bb % 16 != 0) return fail(PKV_ERR_UNSUPPORTED, "block of %lld bytes", bb);
+    if (num_pairs == 0 || num_layers == 0) return PKV_OK;
+    if (!k_pools || !v_pools || !block_mapping) return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    for (int l = 0; l < num_layers; ++l) {
+        if (!k_pools[l] || !v_pools[l]) return fail(PKV_ERR_INVALID_ARG, "null pool pointer for layer %d", l);
+        if (((uintptr_t)k_pools[l] | (uintptr_t)v_pools[l]) & 15)
+            return fail(PKV_ERR_INVALID_ARG, "pools must be 16-byte aligned");
+    }
+    DeviceError* err = device_error_word();
+    if (!err) return fail(PKV_ERR_CUDA, "device error word unavailable");
+    ProfileScope prof(PKV_KERNEL_COPY_BLOCKS, (cudaStream_t)stream);
+    cudaError_t e = launch_copy_blocks(k_pools, v_pools, num_layers, block_mapping, num_pairs, num_blocks, bb, err,
+                                       (cudaStream_t)stream);
+    return e == cudaSuccess ? PKV_OK : cuda_fail(e, "copy_blocks launch");
+}
+
+pkv_status pkv_attention_workspace_size(const int32_t* h_query_start_loc, const int32_t* h_context_lens,
+                                        int num_reqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                        pkv_dtype dtype, const pkv_plan_options* opts, size_t* bytes) {
+    if (!bytes) return fail(PKV_ERR_INVALID_ARG, "null bytes");
+    PlanLists L;
+    pkv_plan plan;
+    const int sms = (opts && opts->num_sms > 0) ? opts->num_sms : current_sm_count();
+    pkv_status s = plan_lists(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim,
+                              dtype, opts, sms, &L, &plan);
+    if (s != PKV_OK) return s;
+    *bytes = (size_t)plan.ws_bytes;
+    return PKV_OK;
+}
+
+pkv_status pkv_attention_plan_host(const int32_t* h_query_start_loc, const int32_t* h_context_lens, int num_reqs,
+                                   int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
+                                   const pkv_plan_options* opts, void* h_meta, size_t meta_capacity,
+                                   pkv_plan* plan) {
+    PlanLists L;
+    const int sms = (opts && opts->num_sms > 0) ? opts->num_sms : 148;
+    pkv_status s = plan_lists(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim,
+                              dtype, opts, sms, &L, plan);
+    if (s != PKV_OK) return s;
+    if (h_meta) {
+        if (meta_capacity < (size_t)plan->meta_bytes)
+            return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "metadata needs %lld bytes", (long long)plan->meta_bytes);
+        write_meta(L, *plan, static_cast<unsigned char*>(h_meta));
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_attention_plan(const int32_t* h_query_start_loc, const int32_t* h_context_lens, int num_reqs,
+                              int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
+                              const pkv_plan_options* opts, void* d_workspace, size_t ws_bytes, pkv_plan* plan,
+                              pkv_stream_t stream) {
+    PlanLists L;
+    const int sms = (opts && opts->num_sms > 0) ? opts->num_sms : current_sm_count();
+    pkv_status s = plan_lists(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim,
+                              dtype, opts, sms, &L, plan);
+    if (s != PKV_OK) return s;
+    if (!d_workspace) return fail(PKV_ERR_INVALID_ARG, "null workspace");
+    if (ws_bytes < (size_t)plan->ws_bytes) {
+        plan->magic = 0;
+        return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes, plan needs %lld", ws_bytes,
+                    (long long)plan->ws_bytes);
+    }
+    static thread_local std::vector<unsigned char> meta;
+    meta.resize((size_t)plan->meta_bytes);
+    write_meta(L, *plan, meta.data());
+    // Pageable source: the call returns once the bytes are staged, so `meta` may be reused.
+    cudaError_t e = cudaMemcpyAsync(d_workspace, meta.data(), meta.size(), cudaMemcpyHostToDevice, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        plan->magic = 0;
+        return cuda_fail(e, "plan upload");
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                               const int32_t* query_start_loc, int num_blocks, float scale, const pkv_plan* plan,
+                               void* d_workspace, size_t ws_bytes, pkv_stream_t stream) {
+    if (!plan || plan->magic != PKV_PLAN_MAGIC) return fail(PKV_ERR_INVALID_ARG, "plan missing or not filled");
+    if (plan->num_q_tokens == 0) return PKV_OK;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start_loc || !d_workspace)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    if (ws_bytes < (size_t)plan->ws_bytes)
+        return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes, plan needs %lld", ws_bytes, (long long)plan->ws_bytes);
+    if (num_blocks <= 0 || max_blocks_per_seq < plan->max_blocks)
+        return fail(PKV_ERR_INVALID_ARG, "num_blocks %d / max_blocks_per_seq %d too small for the plan (%d)", num_blocks,
+                    max_blocks_per_seq, plan->max_blocks);
+    if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_pool | (uintptr_t)v_pool | (uintptr_t)d_workspace) & 15)
+        return fail(PKV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "scale is not finite");
+    DeviceError* err = device_error_word();
+    if (!err) return fail(PKV_ERR_CUDA, "device error word unavailable");
+    const int sms = current_sm_count();
+    unsigned char* ws = static_cast<unsigned char*>(d_workspace);
+    const float scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int G = plan->num_q_heads / plan->num_kv_heads;
+    if (plan->num_tiles > 0) {
+        PrefillArgs a{};
+        a.q = q; a.out = out; a.k_pool = k_pool; a.v_pool = v_pool; a.block_tables = block_tables;
+        a.context_lens = context_lens; a.query_start_loc = query_start_loc;
+        a.tiles = reinterpret_cast<const PrefillTile*>(ws + plan->off_tiles);
+        a.err = err; a.num_tiles = plan->num_tiles; a.max_blocks_per_seq = max_blocks_per_seq;
+        a.num_blocks = num_blocks; a.num_q_heads = plan->num_q_heads; a.num_kv_heads = plan->num_kv_heads;
+        a.group = G; a.num_q_tokens = plan->num_q_tokens; a.scale_log2 = scale_log2;
+        ProfileScope prof(PKV_KERNEL_PREFILL_TC, s);
+        cudaError_t e = launch_prefill_tc(plan->dtype, a, sms, s);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill tile launch");
+    }
+    if (plan->num_items > 0) {
+        DecodeArgs a{};
+        a.q = q; a.out = out; a.k_pool = k_pool; a.v_pool = v_pool; a.block_tables = block_tables;
+        a.items = reinterpret_cast<const DecodeItem*>(ws + plan->off_items);
+        a.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
+        a.part_ml = reinterpret_cast<float*>(ws + plan->off_part_ml);
+        a.err = err; a.num_items = plan->num_items; a.max_blocks_per_seq = max_blocks_per_seq;
+        a.num_blocks = num_blocks; a.num_q_heads = plan->num_q_heads; a.num_kv_heads = plan->num_kv_heads;
+        a.group = G; a.scale_log2 = scale_log2;
+        ProfileScope prof(PKV_KERNEL_DECODE, s);
+        cudaError_t e = launch_decode(plan->dtype, plan->head_dim, a, sms, s);
+        if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    }
+    if (plan->num_merge_rows > 0) {
+        MergeArgs m{};
+        m.out = out;
+        m.rows = reinterpret_cast<const MergeRow*>(ws + plan->off_merge);
+        m.part_o = reinterpret_cast<const float*>(ws + plan->off_part_o);
+        m.part_ml = reinterpret_cast<const float*>(ws + plan->off_part_ml);
+        m.num_rows = plan->num_merge_rows;
+        m.num_q_heads = plan->num_q_heads;
+        ProfileScope prof(PKV_KERNEL_MERGE, s);
+        cudaError_t e = launch_merge(plan->dtype, plan->head_dim, m, s);
+        if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_validate_tables(const int32_t* h_block_tables, const int32_t* h_context_lens, int num_reqs,
+                               int max_blocks_per_seq, int num_blocks) {
+    if (num_reqs < 0 || max_blocks_per_seq < 0 || num_blocks < 0) return fail(PKV_ERR_INVALID_ARG, "negative size");
+    if (num_reqs > 0 && (!h_block_tables || !h_context_lens)) return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    for (int r = 0; r < num_reqs; ++r) {
+        if (h_context_lens[r] < 0) return fail(PKV_ERR_INVALID_ARG, "request %d: negative context", r);
+        const int64_t nb = ceil_div(h_context_lens[r], kBlockSize);
+        if (nb > max_blocks_per_seq)
+            return fail(PKV_ERR_INVALID_ARG, "request %d: needs %lld blocks, table holds %d", r, (long long)nb,
+                        max_blocks_per_seq);
+        for (int64_t i = 0; i < nb; ++i) {
+            const int32_t b = h_block_tables[(int64_t)r * max_blocks_per_seq + i];
+            if (b < 0 || b >= num_blocks)
+                return fail(PKV_ERR_INVALID_ARG, "request %d: table entry %lld = %d outside [0, %d)", r, (long long)i, b,
+                            num_blocks);
+        }
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_validate_slots(const int64_t* h_slot_mapping, int num_tokens, int num_blocks) {
+    if (num_tokens < 0 || num_blocks < 0) return fail(PKV_ERR_INVALID_ARG, "negative size");
+    if (num_tokens > 0 && !h_slot_mapping) return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    std::vector<int64_t> s;
+    s.reserve(num_tokens);
+    const int64_t limit = (int64_t)num_blocks * kBlockSize;
+    for (int t = 0; t < num_tokens; ++t) {
+        const int64_t v = h_slot_mapping[t];
+        if (v < 0) continue;
+        if (v >= limit) return fail(PKV_ERR_INVALID_ARG, "token %d: slot %lld beyond the pool", t, (long long)v);
+        s.push_back(v);
+    }
+    std::sort(s.begin(), s.end());
+    for (size_t i = 1; i < s.size(); ++i)
+        if (s[i] == s[i - 1]) return fail(PKV_ERR_INVALID_ARG, "slot %lld used twice", (long long)s[i]);
+    return PKV_OK;
+}
+
+pkv_status pkv_validate_copy_pairs(const int32_t* h_pairs, int num_pairs, int num_blocks) {
+    if (num_pairs < 0 || num_blocks < 0) return fail(PKV_ERR_INVALID_ARG, "negative size");
+    if (num_pairs > 0 && !h_pairs) return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    std::vector<int32_t> src, dst;
+    for (int p = 0; p < num_pairs; ++p) {
+        const int32_t a = h_pairs[2 * p], b = h_pairs[2 * p + 1];
+        if (a < 0 || a >= num_blocks || b < 0 || b >= num_blocks)
+            return fail(PKV_ERR_INVALID_ARG, "pair %d (%d, %d) outside [0, %d)", p, a, b, num_blocks);
+        if (a == b) continue;
+        src.push_back(a);
+        dst.push_back(b);
+    }
+    std::vector<int32_t> d = dst;
+    std::sort(d.begin(), d.end());
+    for (size_t i = 1; i < d.size(); ++i)
+        if (d[i] == d[i - 1]) return fail(PKV_ERR_INVALID_ARG, "destination block %d repeats", d[i]);
+    std::sort(src.begin(), src.end());
+    for (int32_t b : d)
+        if (std::binary_search(src.begin(), src.end(), b))
+            return fail(PKV_ERR_INVALID_ARG, "block %d is both a source and a destination", b);
+    return PKV_OK;
+}
+
+pkv_status pkv_device_error(int* code, int64_t* detail, pkv_stream_t stream) {
+    if (!code || !detail) return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    DeviceError* err = device_error_word();
+    if (!err) return fail(PKV_ERR_CUDA, "device error word unavailable");
+    DeviceError h{};
+    cudaError_t e = cudaMemcpyAsync(&h, err, sizeof h, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "device error read");
+    *code = h.code;
+    *detail = h.code ? h.detail : -1;
+    if (h.code) {
+        const DeviceError zero{};
+        e = cudaMemcpyAsync(err, &zero, sizeof zero, cudaMemcpyHostToDevice, (cudaStream_t)stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+        if (e != cudaSuccess) return cuda_fail(e, "device error clear");
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_profile_start(int capacity) {
+    if (capacity < 1) return fail(PKV_ERR_INVALID_ARG, "capacity < 1");
+    Profiler& p = t_prof;
+    for (cudaEvent_t e : p.ev) cudaEventDestroy(e);
+    p = Profiler{};
+    p.ev.resize(2 * (size_t)capacity);
+    p.kind.resize((size_t)capacity);
+    for (auto& e : p.ev) {
+        cudaError_t r = cudaEventCreate(&e);
+        if (r != cudaSuccess) {
+            p.ev.clear();
+            return cuda_fail(r, "profile event create");
+        }
+    }
+    p.on = true;
+    return PKV_OK;
+}
+
+pkv_status pkv_profile_stop(double* total_ms, int* launches, int* dropped) {
+    if (!total_ms || !launches || !dropped) return fail(PKV_ERR_INVALID_ARG, "null output");
+    Profiler& p = t_prof;
+    if (!p.on) return fail(PKV_ERR_INVALID_ARG, "profiling was not started");
+    for (int k = 0; k < PKV_KERNEL_KINDS; ++k) {
+        total_ms[k] = 0.0;
+        launches[k] = p.launches[k];
+    }
+    *dropped = p.dropped;
+    pkv_status st = PKV_OK;
+    for (int i = 0; i < p.used; ++i) {
+        cudaError_t r = cudaEventSynchronize(p.ev[2 * i + 1]);
+        float ms = 0.f;
+        if (r == cudaSuccess) r = cudaEventElapsedTime(&ms, p.ev[2 * i], p.ev[2 * i + 1]);
+        if (r != cudaSuccess) {
+            st = cuda_fail(r, "profile event read");
+            break;
+        }
+        total_ms[p.kind[i]] += ms;
+    }
+    for (cudaEvent_t e : p.ev) cudaEventDestroy(e);
+    p = Profiler{};
+    return st;
+}
+
+}  // extern "C"

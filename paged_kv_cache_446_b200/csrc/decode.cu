@@ -1,0 +1,459 @@
+// CUDA-core paged attention: split-K ("flash-decoding") over KV blocks with GQA packing, plus the
+// log-sum-exp merge of chunk partials.
+//
+// What it computes follows blog.mckayzhao.com/?p=56, "PagedAttention：操作系统课本里翻出来的灵感":
+// each KV block of a request is found through its block table and K and V are read block by block;
+// the result equals attention over contiguous storage. Rows of any length are served (decode rows
+// and, one row at a time with a causal limit, prefill rows that the tcgen05 path does not take).
+//
+// Design (B200): every warp is an independent persistent worker. It walks a static round-robin
+// share of the planner's work items (row, KV head, up to 8 query heads, block range) and streams
+// each (block, KV head) K and V chunk -- a contiguous 16*D run in the pool -- with one
+// cp.async.bulk (TMA engine, no tensor map) into a private ring of shared-memory stages,
+// completion tracked by an mbarrier per stage. The ring runs ahead across item boundaries, so
+// the copy engine is never idle between items. Each lane owns one 16-byte column chunk of a K/V
+// row: QK partial dots are fp32 FMAs on registers, reduced across the row's lanes with a
+// butterfly reduce-scatter of warp shuffles; the online softmax is per query head in fp32 (log2
+// domain, ex2.approx); P*V accumulates in fp32 registers. Items covering part of a row write
+// (unnormalised output, max, sum) partials; merge_kernel combines them by log-sum-exp.
+#include <type_traits>
+
+#include "common.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int log2i(int x) { return x <= 1 ? 0 : 1 + log2i(x / 2); }
+constexpr int round16(int x) { return (x + 15) / 16 * 16; }
+constexpr int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
+
+template <typename T, int D, int GP>
+struct Dec {
+    static constexpr int EB = sizeof(T);
+    static constexpr int ROW = D * EB;                 // bytes of one K/V row
+    static constexpr int CPR = ROW / 16;               // 16-byte chunks per row = lanes per row
+    static constexpr int LOG_CPR = log2i(CPR);
+    static constexpr int TPP = 32 / CPR;               // rows (tokens) handled per warp pass
+    static constexpr int EPC = 16 / EB;                // elements per chunk
+    static constexpr int PASSES = kBlockSize / TPP;    // passes per 16-token block
+    static constexpr int LOG_PASSES = log2i(PASSES);
+    static constexpr int NV = GP * PASSES;             // partial dots per lane per block
+    static constexpr int LOG_NV = log2i(NV);
+    static constexpr int SPLIT = LOG_CPR < LOG_NV ? LOG_CPR : LOG_NV;  // reduce-scatter rounds
+    static constexpr int NOWN = NV >> SPLIT;           // full dots owned per lane afterwards
+    static constexpr int BLK = kBlockSize * ROW;       // bytes of one (block, head) K or V chunk
+    static constexpr int QB = GP * ROW;                // bytes of an item's query rows
+    static constexpr int STAGE = 2 * BLK + QB;
+    static constexpr int STAGES = clampi((32 * 1024) / STAGE, 2, 4);
+    static constexpr int P_FLOATS = GP * TPP * PASSES; // softmax weights of one block
+    static constexpr int SCR = round16(P_FLOATS * 4 + GP * 4 + GP * 8);
+    static constexpr int WARP_SMEM = STAGES * STAGE + SCR + round16(STAGES * 8);
+    static_assert(CPR >= 8 && CPR <= 32, "K/V rows of 128..512 bytes");
+    static_assert(GP <= CPR, "query group larger than the lanes of a row");
+    static_assert(PASSES % 4 == 0, "weights are read four at a time");
+};
+
+constexpr int kDecodeWarps = 2;  // independent warps per CTA
+
+__device__ __forceinline__ DecodeItem load_item(const DecodeItem* items, int i) {
+    const int4* p = reinterpret_cast<const int4*>(items + i);
+    const int4 a = __ldg(p), b = __ldg(p + 1);
+    DecodeItem it;
+    it.row = a.x; it.req = a.y; it.kv_head = a.z; it.head0 = a.w;
+    it.blk_begin = b.x; it.blk_end = b.y; it.limit = b.z; it.partial = b.w;
+    return it;
+}
+
+template <typename T, int D, int GP>
+__global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeArgs a) {
+    using C = Dec<T, D, GP>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    unsigned char* wbase = smem + warp * C::WARP_SMEM;
+    float* p_s = reinterpret_cast<float*>(wbase + C::STAGES * C::STAGE);
+    float* alpha_s = p_s + C::P_FLOATS;
+    float* ml_s = alpha_s + GP;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + C::STAGES * C::STAGE + C::SCR);
+
+    if (lane == 0) {
+        for (int s = 0; s < C::STAGES; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    const int W = gridDim.x * kDecodeWarps;
+    const int gw = blockIdx.x * kDecodeWarps + warp;
+    if (gw >= a.num_items) return;
+
+    const int sub = lane >> C::LOG_CPR;       // token slot inside a pass
+    const int chunk = lane & (C::CPR - 1);    // 16-byte column chunk of a row
+    const size_t head_stride = (size_t)C::BLK;
+    const unsigned char* kp = static_cast<const unsigned char*>(a.k_pool);
+    const unsigned char* vp = static_cast<const unsigned char*>(a.v_pool);
+    const unsigned char* qp = static_cast<const unsigned char*>(a.q);
+
+    // ---------------- producer (runs up to STAGES blocks ahead of the consumer) ----------------
+    int p_it = gw;
+    DecodeItem pi = load_item(a.items, p_it);
+    int p_blk = pi.blk_begin;
+    int p_base = p_blk;
+    int p_ids = (p_blk + lane < pi.blk_end) ? __ldg(a.block_tables + (size_t)pi.req * a.max_blocks_per_seq + p_blk + lane) : 0;
+    bool p_done = false;
+    uint32_t issued = 0;
+
+    auto issue = [&](int stage) {
+        const int id_raw = __shfl_sync(FULL_MASK, p_ids, p_blk - p_base);
+        if (lane == 0) {
+            int id = id_raw;
+            if (id < 0 || id >= a.num_blocks) {
+                record_error(a.err, 6 /*PKV_ERR_DEVICE_RANGE*/, (long long)pi.req * a.max_blocks_per_seq + p_blk);
+                id = 0;
+            }
+            unsigned char* st = wbase + stage * C::STAGE;
+            const bool first = (p_blk == pi.blk_begin);
+            const int nh = min(GP, a.group - pi.head0);
+            const uint32_t qbytes = first ? (uint32_t)(nh * C::ROW) : 0u;
+            mbar_arrive_expect_tx(&bars[stage], 2u * C::BLK + qbytes);
+            const size_t off = ((size_t)id * a.num_kv_heads + pi.kv_head) * head_stride;
+            bulk_g2s(st, kp + off, C::BLK, &bars[stage]);
+            bulk_g2s(st + C::BLK, vp + off, C::BLK, &bars[stage]);
+            if (first) {
+                const size_t qoff = ((size_t)pi.row * a.num_q_heads + (size_t)pi.kv_head * a.group + pi.head0) * C::ROW;
+                bulk_g2s(st + 2 * C::BLK, qp + qoff, qbytes, &bars[stage]);
+            }
+        }
+        ++issued;
+        // advance to the next (item, block)
+        ++p_blk;
+        if (p_blk == pi.blk_end) {
+            p_it += W;
+            if (p_it < a.num_items) {
+                pi = load_item(a.items, p_it);
+                p_blk = pi.blk_begin;
+                p_base = p_blk;
+                p_ids = (p_blk + lane < pi.blk_end)
+                            ? __ldg(a.block_tables + (size_t)pi.req * a.max_blocks_per_seq + p_blk + lane) : 0;
+            } else {
+                p_done = true;
+            }
+        } else if (p_blk - p_base == 32) {
+            p_base = p_blk;
+            p_ids = (p_blk + lane < pi.blk_end)
+                        ? __ldg(a.block_tables + (size_t)pi.req * a.max_blocks_per_seq + p_blk + lane) : 0;
+        }
+    };
+
+    for (int s = 0; s < C::STAGES && !p_done; ++s) issue(s);
+
+    // ---------------- consumer ----------------
+    int c_it = gw;
+    DecodeItem ci = load_item(a.items, c_it);
+    int c_blk = ci.blk_begin;
+    uint32_t consumed = 0;
+
+    float q[GP][C::EPC];
+    float acc[GP][C::EPC];
+    float m_own = -INFINITY, l_own = 0.f;
+
+    // Owned dots after the reduce-scatter: indices base .. base+NOWN-1 of (g * PASSES + i).
+    int base = 0;
+#pragma unroll
+    for (int r = 0; r < C::SPLIT; ++r)
+        if (lane & (C::CPR >> (r + 1))) base += C::NV >> (r + 1);
+    const int g_own = base / C::PASSES;
+    const int i_own0 = base % C::PASSES;
+
+    while (true) {
+        const int stage = consumed % C::STAGES;
+        const uint32_t parity = (consumed / C::STAGES) & 1u;
+        if (!mbar_wait(&bars[stage], parity)) {
+            if (lane == 0) record_error(a.err, 5 /*PKV_ERR_DEVICE_TIMEOUT*/, c_it);
+            // Drain the copies still in flight (bounded) before leaving.
+            for (uint32_t k = consumed; k < issued; ++k)
+                (void)mbar_wait(&bars[k % C::STAGES], (k / C::STAGES) & 1u);
+            return;
+        }
+        const unsigned char* st = wbase + stage * C::STAGE;
+        const unsigned char* Ks = st;
+        const unsigned char* Vs = st + C::BLK;
+        const int nh = min(GP, a.group - ci.head0);
+
+        if (c_blk == ci.blk_begin) {
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+                if (g < nh) {
+                    Chunk<T>::unpack(lds128(st + 2 * C::BLK + g * C::ROW + chunk * 16), q[g]);
+#pragma unroll
+                    for (int e = 0; e < C::EPC; ++e) q[g][e] *= a.scale_log2;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < C::EPC; ++e) q[g][e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < C::EPC; ++e) acc[g][e] = 0.f;
+            }
+            m_own = -INFINITY;
+            l_own = 0.f;
+        }
+        const int valid = min(kBlockSize, ci.limit - c_blk * kBlockSize);
+
+        // ---- QK: partial dots of this lane's chunk for every (head, pass) ----
+        float dots[C::NV];
+#pragma unroll
+        for (int i = 0; i < C::PASSES; ++i) {
+            float k[C::EPC];
+            Chunk<T>::unpack(lds128(Ks + (i * C::TPP + sub) * C::ROW + chunk * 16), k);
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+                float d = 0.f;
+#pragma unroll
+                for (int e = 0; e < C::EPC; ++e) d = fmaf(q[g][e], k[e], d);
+                dots[g * C::PASSES + i] = d;
+            }
+        }
+        // ---- reduce-scatter across the CPR lanes of a row ----
+#pragma unroll
+        for (int r = 0; r < C::LOG_CPR; ++r) {
+            const int o = C::CPR >> (r + 1);
+            if (r < C::LOG_NV) {
+                const int h = C::NV >> (r + 1);
+                const bool upper = (lane & o) != 0;
+#pragma unroll
+                for (int k = 0; k < h; ++k) {
+                    const float send = upper ? dots[k] : dots[k + h];
+                    const float keep = upper ? dots[k + h] : dots[k];
+                    dots[k] = keep + __shfl_xor_sync(FULL_MASK, send, o);
+                }
+            } else {
+                dots[0] += __shfl_xor_sync(FULL_MASK, dots[0], o);
+            }
+        }
+        // ---- online softmax for head g_own over this block's tokens ----
+        float mb = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < C::NOWN; ++k) {
+            const int t = (i_own0 + k) * C::TPP + sub;
+            if (t >= valid) dots[k] = -INFINITY;
+            mb = fmaxf(mb, dots[k]);
+        }
+#pragma unroll
+        for (int r = 0; r < C::SPLIT; ++r)
+            if (C::LOG_NV - 1 - r < C::LOG_PASSES) mb = fmaxf(mb, __shfl_xor_sync(FULL_MASK, mb, C::CPR >> (r + 1)));
+#pragma unroll
+        for (int o = C::CPR; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(FULL_MASK, mb, o));
+        const float m_new = fmaxf(m_own, mb);
+        const float alpha = fast_exp2(m_own - m_new);
+        float ps = 0.f;
+        float* prow = p_s + (g_own * C::TPP + sub) * C::PASSES;
+#pragma unroll
+        for (int k = 0; k < C::NOWN; ++k) {
+            const float p = fast_exp2(dots[k] - m_new);
+            ps += p;
+            prow[i_own0 + k] = p;
+        }
+#pragma unroll
+        for (int r = 0; r < C::SPLIT; ++r)
+            if (C::LOG_NV - 1 - r < C::LOG_PASSES) ps += __shfl_xor_sync(FULL_MASK, ps, C::CPR >> (r + 1));
+#pragma unroll
+        for (int o = C::CPR; o < 32; o <<= 1) ps += __shfl_xor_sync(FULL_MASK, ps, o);
+        l_own = l_own * alpha + ps;
+        m_own = m_new;
+        alpha_s[g_own] = alpha;
+        __syncwarp();
+
+        // ---- P*V ----
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+            const float al = alpha_s[g];
+#pragma unroll
+            for (int e = 0; e < C::EPC; ++e) acc[g][e] *= al;
+        }
+#pragma unroll
+        for (int i4 = 0; i4 < C::PASSES; i4 += 4) {
+            float4 pw[GP];
+#pragma unroll
+            for (int g = 0; g < GP; ++g)
+                pw[g] = *reinterpret_cast<const float4*>(p_s + (g * C::TPP + sub) * C::PASSES + i4);
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                const int t = (i4 + ii) * C::TPP + sub;
+                float v[C::EPC];
+                Chunk<T>::unpack(lds128(Vs + t * C::ROW + chunk * 16), v);
+                if (t >= valid) {
+#pragma unroll
+                    for (int e = 0; e < C::EPC; ++e) v[e] = 0.f;  // slots past the context may hold anything
+                }
+#pragma unroll
+                for (int g = 0; g < GP; ++g) {
+                    const float p = ii == 0 ? pw[g].x : ii == 1 ? pw[g].y : ii == 2 ? pw[g].z : pw[g].w;
+#pragma unroll
+                    for (int e = 0; e < C::EPC; ++e) acc[g][e] = fmaf(p, v[e], acc[g][e]);
+                }
+            }
+        }
+        __syncwarp();
+        ++consumed;
+
+        // Refill this stage with the producer's next block.
+        if (!p_done) {
+            fence_proxy_async_smem();
+            issue(stage);
+        }
+
+        if (c_blk + 1 == ci.blk_end) {
+            // ---- item done: combine token slots, then write the output or the partial ----
+#pragma unroll
+            for (int o = C::CPR; o < 32; o <<= 1)
+#pragma unroll
+                for (int g = 0; g < GP; ++g)
+#pragma unroll
+                    for (int e = 0; e < C::EPC; ++e) acc[g][e] += __shfl_xor_sync(FULL_MASK, acc[g][e], o);
+            ml_s[2 * g_own] = m_own;
+            ml_s[2 * g_own + 1] = l_own;
+            __syncwarp();
+            if (sub == 0) {
+#pragma unroll
+                for (int g = 0; g < GP; ++g) {
+                    if (g < nh) {
+                        const size_t qh = (size_t)ci.row * a.num_q_heads + (size_t)ci.kv_head * a.group + ci.head0 + g;
+                        if (ci.partial < 0) {
+                            const float inv = 1.f / ml_s[2 * g + 1];
+                            float o[C::EPC];
+#pragma unroll
+                            for (int e = 0; e < C::EPC; ++e) o[e] = acc[g][e] * inv;
+                            *reinterpret_cast<uint4*>(static_cast<unsigned char*>(a.out) + qh * C::ROW + chunk * 16) =
+                                Chunk<T>::pack(o);
+                        } else {
+                            float* po = a.part_o + ((size_t)ci.partial * kMaxGroupPerItem + g) * D + chunk * C::EPC;
+#pragma unroll
+                            for (int e = 0; e < C::EPC; e += 4)
+                                *reinterpret_cast<float4*>(po + e) = make_float4(acc[g][e], acc[g][e + 1], acc[g][e + 2], acc[g][e + 3]);
+                            if (chunk == 0) {
+                                float* pm = a.part_ml + ((size_t)ci.partial * kMaxGroupPerItem + g) * 2;
+                                pm[0] = ml_s[2 * g];
+                                pm[1] = ml_s[2 * g + 1];
+                            }
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            c_it += W;
+            if (c_it >= a.num_items) break;
+            ci = load_item(a.items, c_it);
+            c_blk = ci.blk_begin;
+        } else {
+            ++c_blk;
+        }
+    }
+}
+
+// One warp per (merge row, head): out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
+    constexpr int PER = D / 32;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int entry = gw / kMaxGroupPerItem;
+    const int g = gw % kMaxGroupPerItem;
+    if (entry >= a.num_rows) return;
+    const MergeRow mr = a.rows[entry];
+    if (g >= mr.num_heads) return;
+    float M = -INFINITY;
+    for (int i = 0; i < mr.count; ++i)
+        M = fmaxf(M, a.part_ml[((size_t)(mr.first_partial + i) * kMaxGroupPerItem + g) * 2]);
+    float L = 0.f;
+    float o[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[e] = 0.f;
+    for (int i = 0; i < mr.count; ++i) {
+        const size_t p = (size_t)(mr.first_partial + i) * kMaxGroupPerItem + g;
+        const float w = fast_exp2(a.part_ml[p * 2] - M);
+        L = fmaf(w, a.part_ml[p * 2 + 1], L);
+        const float* po = a.part_o + p * D + lane * PER;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] = fmaf(w, po[e], o[e]);
+    }
+    const float inv = 1.f / L;
+    T* out = static_cast<T*>(a.out) + ((size_t)mr.row * a.num_q_heads + mr.q_head0 + g) * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        if constexpr (sizeof(T) == 4) out[e] = o[e] * inv;
+        else if constexpr (std::is_same<T, __half>::value) out[e] = __float2half_rn(o[e] * inv);
+        else out[e] = __float2bfloat16_rn(o[e] * inv);
+    }
+}
+
+template <typename T, int D, int GP>
+cudaError_t launch_decode_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    using C = Dec<T, D, GP>;
+    const int smem = kDecodeWarps * C::WARP_SMEM;
+    // The shared-memory attribute and the occupancy are per device; cache both per instantiation.
+    static int per_sm_cache[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int per_sm = (dev >= 0 && dev < 64) ? per_sm_cache[dev] : 0;
+    if (per_sm == 0) {
+        e = cudaFuncSetAttribute(decode_kernel<T, D, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<T, D, GP>, kDecodeWarps * 32, smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+        if (dev >= 0 && dev < 64) per_sm_cache[dev] = per_sm;
+    }
+    const int need = (a.num_items + kDecodeWarps - 1) / kDecodeWarps;
+    int grid = num_sms * per_sm;
+    if (grid > need) grid = need;
+    if (grid < 1) return cudaSuccess;
+    decode_kernel<T, D, GP><<<grid, kDecodeWarps * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_decode_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    const int g = a.group < kMaxGroupPerItem ? a.group : kMaxGroupPerItem;
+    if (g <= 1) return launch_decode_t<T, D, 1>(a, num_sms, s);
+    if (g <= 2) return launch_decode_t<T, D, 2>(a, num_sms, s);
+    if (g <= 4) return launch_decode_t<T, D, 4>(a, num_sms, s);
+    return launch_decode_t<T, D, 8>(a, num_sms, s);
+}
+
+template <typename T>
+cudaError_t launch_decode_d(int head_dim, const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    if (head_dim == 64) return launch_decode_g<T, 64>(a, num_sms, s);
+    return launch_decode_g<T, 128>(a, num_sms, s);
+}
+
+template <typename T>
+cudaError_t launch_merge_d(int head_dim, const MergeArgs& a, cudaStream_t s) {
+    const long long warps = (long long)a.num_rows * kMaxGroupPerItem;
+    const int grid = (int)((warps * 32 + 127) / 128);
+    if (grid < 1) return cudaSuccess;
+    if (head_dim == 64) merge_kernel<T, 64><<<grid, 128, 0, s>>>(a);
+    else merge_kernel<T, 128><<<grid, 128, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(int dtype, int head_dim, const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    if (a.num_items <= 0) return cudaSuccess;
+    switch (dtype) {
+        case 0: return launch_decode_d<float>(head_dim, a, num_sms, s);
+        case 1: return launch_decode_d<__half>(head_dim, a, num_sms, s);
+        default: return launch_decode_d<__nv_bfloat16>(head_dim, a, num_sms, s);
+    }
+}
+
+cudaError_t launch_merge(int dtype, int head_dim, const MergeArgs& a, cudaStream_t s) {
+    if (a.num_rows <= 0) return cudaSuccess;
+    switch (dtype) {
+        case 0: return launch_merge_d<float>(head_dim, a, s);
+        case 1: return launch_merge_d<__half>(head_dim, a, s);
+        default: return launch_merge_d<__nv_bfloat16>(head_dim, a, s);
+    }
+}
+
+}  // namespace pkv

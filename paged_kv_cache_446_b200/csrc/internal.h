@@ -1,0 +1,119 @@
+// Internal declarations shared by the library's translation units (host and device).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pkv {
+
+constexpr int kBlockSize = 16;      // tokens per KV block
+constexpr int kMaxGroupPerItem = 8; // query heads one CUDA-core work item serves (GQA packing)
+
+// First device-side error and its detail (an index); zero when none happened.
+struct DeviceError {
+    int code;
+    int pad;
+    long long detail;
+};
+
+// One unit of CUDA-core work: a query row, a KV head, up to 8 query heads of its group and a
+// contiguous range of the row's KV blocks.
+struct DecodeItem {
+    int32_t row;        // query row (index into q/out)
+    int32_t req;        // request (row of the block table)
+    int32_t kv_head;
+    int32_t head0;      // first query head of the group served here (offset inside the group)
+    int32_t blk_begin;  // KV block range [blk_begin, blk_end) of the request
+    int32_t blk_end;
+    int32_t limit;      // the row sees keys at positions < limit
+    int32_t partial;    // partial-result slot, or -1 when the item covers the whole row
+};
+static_assert(sizeof(DecodeItem) == 32, "DecodeItem layout");
+
+// One tcgen05 tile: 128 packed (query row, query head) rows of one request and KV head.
+struct PrefillTile {
+    int32_t req;
+    int32_t kv_head;
+    int32_t tok0;       // first query row of the tile, relative to the request's first row
+    int32_t key_tiles;  // 128-key tiles this tile iterates (planner's estimate, for ordering)
+};
+static_assert(sizeof(PrefillTile) == 16, "PrefillTile layout");
+
+// A (row, query-head range) whose chunks the log-sum-exp merge combines.
+struct MergeRow {
+    int32_t row;
+    int32_t q_head0;       // first query head
+    int32_t num_heads;     // heads in this entry (<= 8)
+    int32_t first_partial; // partial slots first_partial .. first_partial + count - 1
+    int32_t count;
+    int32_t pad[3];
+};
+static_assert(sizeof(MergeRow) == 32, "MergeRow layout");
+
+struct DecodeArgs {
+    const void* q;
+    void* out;
+    const void* k_pool;
+    const void* v_pool;
+    const int32_t* block_tables;
+    const DecodeItem* items;
+    float* part_o;       // [num_partials][8][D]
+    float* part_ml;      // [num_partials][8][2] (max in log2 units, sum)
+    DeviceError* err;
+    int num_items;
+    int max_blocks_per_seq;
+    int num_blocks;
+    int num_q_heads;
+    int num_kv_heads;
+    int group;           // Hq / Hkv
+    float scale_log2;    // scale * log2(e)
+};
+
+struct MergeArgs {
+    void* out;
+    const MergeRow* rows;
+    const float* part_o;
+    const float* part_ml;
+    int num_rows;
+    int num_q_heads;
+};
+
+struct PrefillArgs {
+    const void* q;
+    void* out;
+    const void* k_pool;
+    const void* v_pool;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* query_start_loc;
+    const PrefillTile* tiles;
+    DeviceError* err;
+    int num_tiles;
+    int max_blocks_per_seq;
+    int num_blocks;
+    int num_q_heads;
+    int num_kv_heads;
+    int group;
+    int num_q_tokens;
+    float scale_log2;
+};
+
+// Launchers (return the launch error, if any).
+cudaError_t launch_decode(int dtype, int head_dim, const DecodeArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_merge(int dtype, int head_dim, const MergeArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_tc(int dtype, const PrefillArgs& a, int num_sms, cudaStream_t s);
+bool prefill_tc_supported(int dtype, int head_dim, int group);
+cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, const int32_t* qsl, const int32_t* ctx,
+                                int num_reqs, int num_blocks, int64_t* slots, int num_tokens, DeviceError* err,
+                                cudaStream_t s);
+cudaError_t launch_kv_write(const void* k_new, const void* v_new, void* k_pool, void* v_pool, const int64_t* slots,
+                            int num_tokens, int num_blocks, int num_kv_heads, int row_bytes, DeviceError* err,
+                            cudaStream_t s);
+cudaError_t launch_copy_blocks(void* const* k_pools, void* const* v_pools, int num_layers, const int32_t* pairs,
+                               int num_pairs, int num_blocks, long long block_bytes, DeviceError* err,
+                               cudaStream_t s);
+
+// Device error word of the current device.
+DeviceError* device_error_word();
+
+}  // namespace pkv

@@ -1,0 +1,268 @@
+"""Python binding of libpkv.so (include/pkv.h): argument marshalling only.
+
+Every step of the hot path runs in the library's sm_100a kernels; torch supplies device memory and
+the current CUDA stream. There is no fallback: if the shared library is missing or cannot be loaded,
+importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m paged_kv_cache_446_b200.build` "
+                      "(or __graft_entry__.build())")
+_lib = ctypes.CDLL(LIB_PATH)
+
+PKV_OK = 0
+STATUS = {0: "PKV_OK", 1: "PKV_ERR_INVALID_ARG", 2: "PKV_ERR_UNSUPPORTED", 3: "PKV_ERR_CUDA",
+          4: "PKV_ERR_WORKSPACE_TOO_SMALL", 5: "PKV_ERR_DEVICE_TIMEOUT", 6: "PKV_ERR_DEVICE_RANGE"}
+DTYPE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+DTYPE_NAME = {"f32": 0, "f16": 1, "bf16": 2}
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+
+class PlanOptions(ctypes.Structure):
+    _fields_ = [("split_blocks", ctypes.c_int32), ("no_split", ctypes.c_int32),
+                ("cuda_core_only", ctypes.c_int32), ("num_sms", ctypes.c_int32)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("magic", ctypes.c_uint32)] + [(n, ctypes.c_int32) for n in (
+        "num_reqs", "num_q_tokens", "num_q_heads", "num_kv_heads", "head_dim", "dtype", "num_decode_rows",
+        "num_prefill_rows", "num_items", "num_tiles", "num_merge_rows", "num_partials", "split_blocks",
+        "max_blocks")] + [(n, ctypes.c_int64) for n in (
+        "off_items", "off_tiles", "off_merge", "off_part_o", "off_part_ml", "meta_bytes", "ws_bytes", "kv_bytes",
+        "attn_flops")]
+
+
+def _sig(name, restype, argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = argtypes
+    return f
+
+
+_lib.pkv_status_string.restype = ctypes.c_char_p
+_lib.pkv_status_string.argtypes = [_I]
+_lib.pkv_last_error.restype = ctypes.c_char_p
+_lib.pkv_version.restype = ctypes.c_char_p
+_slot_mapping = _sig("pkv_slot_mapping", _I, [_P, _I, _P, _P, _I, _I, _P, _I, _P])
+_kv_cache_write = _sig("pkv_kv_cache_write", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P])
+_copy_blocks = _sig("pkv_copy_blocks", _I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P])
+_ws_size = _sig("pkv_attention_workspace_size", _I, [_P, _P, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_SZ)])
+_plan_host = _sig("pkv_attention_plan_host", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, ctypes.POINTER(Plan)])
+_plan = _sig("pkv_attention_plan", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, ctypes.POINTER(Plan), _P])
+_attention = _sig("pkv_paged_attention", _I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _F, ctypes.POINTER(Plan), _P, _SZ, _P])
+_validate_tables = _sig("pkv_validate_tables", _I, [_P, _P, _I, _I, _I])
+_validate_slots = _sig("pkv_validate_slots", _I, [_P, _I, _I])
+_validate_pairs = _sig("pkv_validate_copy_pairs", _I, [_P, _I, _I])
+_device_error = _sig("pkv_device_error", _I, [ctypes.POINTER(_I), ctypes.POINTER(_I64), _P])
+_profile_start = _sig("pkv_profile_start", _I, [_I])
+_profile_stop = _sig("pkv_profile_stop", _I, [_P, _P, _P])
+KERNEL_KINDS = ("slot_mapping", "kv_write", "copy_blocks", "decode", "merge", "prefill_tc")
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.pkv_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {msg}")
+
+
+def _check(status: int, where: str):
+    if status != PKV_OK:
+        raise PkvError(status, where)
+
+
+def version() -> str:
+    return _lib.pkv_version().decode()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _np_ptr(a: np.ndarray):
+    return a.ctypes.data_as(_P)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in DTYPE:
+        raise TypeError(f"unsupported element type {t.dtype}")
+    return DTYPE[t.dtype]
+
+
+def _opts(split_blocks=0, no_split=False, cuda_core_only=False, num_sms=0) -> PlanOptions:
+    return PlanOptions(int(split_blocks), int(bool(no_split)), int(bool(cuda_core_only)), int(num_sms))
+
+
+# ---- a13: mixed-batch flattening -------------------------------------------------------------
+
+def flatten_batch(batch: dict, prior_lens) -> tuple[np.ndarray, np.ndarray]:
+    """{request_id: num_tokens} (dict order) + each request's prior context ->
+    (query_start_loc int32 [R+1], context_lens int32 [R]) on the host."""
+    counts = np.fromiter((int(v) for v in batch.values()), dtype=np.int64, count=len(batch))
+    qsl = np.zeros(len(batch) + 1, dtype=np.int64)
+    np.cumsum(counts, out=qsl[1:])
+    ctx = np.asarray(prior_lens, dtype=np.int64).reshape(-1) + counts
+    return qsl.astype(np.int32), ctx.astype(np.int32)
+
+
+# ---- a1 / a2 / a12 -----------------------------------------------------------------------------
+
+def slot_mapping(block_tables: torch.Tensor, query_start_loc: torch.Tensor, context_lens: torch.Tensor,
+                 num_blocks: int, num_tokens: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Physical slot (int64) of every token the step appends; device tensors in and out."""
+    if out is None:
+        out = torch.empty(num_tokens, dtype=torch.int64, device=block_tables.device)
+    R = context_lens.shape[0]
+    mb = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    _check(_slot_mapping(_ptr(block_tables), mb, _ptr(query_start_loc), _ptr(context_lens), R, int(num_blocks),
+                         _ptr(out), int(num_tokens), _stream(stream)), "pkv_slot_mapping")
+    return out
+
+
+def kv_cache_write(k_new: torch.Tensor, v_new: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                   slot_mapping: torch.Tensor, stream=None) -> None:
+    """k_pool[slot // 16, h, slot % 16] = k_new[t, h] (and V) for every slot >= 0."""
+    NB, Hkv, BS, D = k_pool.shape
+    T = slot_mapping.shape[0]
+    _check(_kv_cache_write(_ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(slot_mapping), T, NB, Hkv, D,
+                           BS, _dtype_code(k_pool), _stream(stream)), "pkv_kv_cache_write")
+
+
+def copy_blocks(k_pools: list, v_pools: list, block_mapping: torch.Tensor, stream=None) -> None:
+    """Copy-on-write: for every layer, block dst := block src for each (src, dst) row of block_mapping."""
+    L = len(k_pools)
+    NB, Hkv, BS, D = k_pools[0].shape
+    kp = (_P * L)(*[_ptr(p) for p in k_pools])
+    vp = (_P * L)(*[_ptr(p) for p in v_pools])
+    P = block_mapping.shape[0]
+    _check(_copy_blocks(kp, vp, L, _ptr(block_mapping), P, NB, Hkv, D, BS, _dtype_code(k_pools[0]), _stream(stream)),
+           "pkv_copy_blocks")
+
+
+# ---- paged attention ---------------------------------------------------------------------------
+
+def plan_host(query_start_loc: np.ndarray, context_lens: np.ndarray, num_q_heads: int, num_kv_heads: int,
+              head_dim: int, dtype: str, with_meta: bool = True, **opts) -> tuple[Plan, np.ndarray | None]:
+    """Host-only planning (no CUDA): the plan and the metadata image the upload would copy."""
+    qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+    plan = Plan()
+    o = _opts(**opts)
+    _check(_plan_host(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], num_q_heads, num_kv_heads, head_dim,
+                      DTYPE_NAME[dtype], ctypes.byref(o), None, 0, ctypes.byref(plan)), "pkv_attention_plan_host")
+    meta = None
+    if with_meta:
+        meta = np.zeros(plan.meta_bytes, dtype=np.uint8)
+        _check(_plan_host(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], num_q_heads, num_kv_heads, head_dim,
+                          DTYPE_NAME[dtype], ctypes.byref(o), _np_ptr(meta), meta.nbytes, ctypes.byref(plan)),
+               "pkv_attention_plan_host")
+    return plan, meta
+
+
+class AttentionPlan:
+    """A planned batch: host plan, device workspace and device copies of the batch description."""
+
+    def __init__(self, batch: dict, prior_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                 dtype: torch.dtype, device, workspace: torch.Tensor | None = None, stream=None, **opts):
+        qsl, ctx = flatten_batch(batch, prior_lens)
+        self.h_query_start_loc, self.h_context_lens = qsl, ctx
+        self.num_q_heads, self.num_kv_heads, self.head_dim, self.dtype = num_q_heads, num_kv_heads, head_dim, dtype
+        self.num_q_tokens = int(qsl[-1])
+        o = _opts(**opts)
+        size = _SZ(0)
+        _check(_ws_size(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], num_q_heads, num_kv_heads, head_dim,
+                        _dtype_code(torch.empty(0, dtype=dtype)), ctypes.byref(o), ctypes.byref(size)),
+               "pkv_attention_workspace_size")
+        if workspace is None or workspace.numel() < size.value:
+            workspace = torch.empty(max(size.value, 256), dtype=torch.uint8, device=device)
+        self.workspace = workspace
+        self.plan = Plan()
+        _check(_plan(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], num_q_heads, num_kv_heads, head_dim,
+                     _dtype_code(torch.empty(0, dtype=dtype)), ctypes.byref(o), _ptr(workspace), workspace.numel(),
+                     ctypes.byref(self.plan), _stream(stream)), "pkv_attention_plan")
+        # Pinned staging keeps the uploads asynchronous; torch's host allocator keeps each staging
+        # buffer alive until its copy has run.
+        self.query_start_loc = torch.from_numpy(qsl).pin_memory().to(device, non_blocking=True)
+        self.context_lens = torch.from_numpy(ctx).pin_memory().to(device, non_blocking=True)
+
+
+def paged_attention(plan: AttentionPlan, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                    block_tables: torch.Tensor, scale: float, out: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """Attention of every row of the planned batch; q/out [T, Hq, D], pools [NB, Hkv, 16, D]."""
+    if out is None:
+        out = torch.empty_like(q)
+    NB = k_pool.shape[0]
+    _check(_attention(_ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+                      _ptr(plan.context_lens), _ptr(plan.query_start_loc), NB, float(scale), ctypes.byref(plan.plan),
+                      _ptr(plan.workspace), plan.workspace.numel(), _stream(stream)), "pkv_paged_attention")
+    return out
+
+
+# ---- host validators and the device error word -----------------------------------------------
+
+def validate_tables(block_tables: np.ndarray, context_lens: np.ndarray, num_blocks: int) -> None:
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+    _check(_validate_tables(_np_ptr(bt), _np_ptr(ctx), ctx.shape[0], bt.shape[1] if bt.ndim == 2 else 0,
+                            int(num_blocks)), "pkv_validate_tables")
+
+
+def validate_slots(slots: np.ndarray, num_blocks: int) -> None:
+    s = np.ascontiguousarray(slots, dtype=np.int64)
+    _check(_validate_slots(_np_ptr(s), s.shape[0], int(num_blocks)), "pkv_validate_slots")
+
+
+def validate_copy_pairs(pairs: np.ndarray, num_blocks: int) -> None:
+    p = np.ascontiguousarray(pairs, dtype=np.int32).reshape(-1, 2)
+    _check(_validate_pairs(_np_ptr(p), p.shape[0], int(num_blocks)), "pkv_validate_copy_pairs")
+
+
+def device_error(stream=None) -> tuple[int, int]:
+    """(code, detail) of the first device-side error since the last read; (0, -1) when none."""
+    code = _I(0)
+    detail = _I64(0)
+    _check(_device_error(ctypes.byref(code), ctypes.byref(detail), _stream(stream)), "pkv_device_error")
+    return code.value, detail.value
+
+
+def profile_start(capacity: int = 4096) -> None:
+    """Time every library kernel launched from this thread with CUDA events on its stream."""
+    _check(_profile_start(int(capacity)), "pkv_profile_start")
+
+
+def profile_stop() -> dict:
+    """{kind: (total_ms, launches)} since profile_start; also 'dropped' (launches not timed)."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int * n)()
+    dropped = ctypes.c_int(0)
+    _check(_profile_stop(ms, cnt, ctypes.byref(dropped)), "pkv_profile_stop")
+    out = {k: (ms[i], cnt[i]) for i, k in enumerate(KERNEL_KINDS)}
+    out["dropped"] = dropped.value
+    return out

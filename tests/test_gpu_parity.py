@@ -1,0 +1,210 @@
+"""GPU parity: the sm_100a library against the CPU oracle on the same seeded inputs.
+
+Bit-exact for slot mapping, KV append and block copies (whole pools, sentinel-filled so a stray write
+shows); within the stated max |err| for attention. Small cases are checked element by element; the
+full-size configurations run in the launch configuration the benchmark times and are checked on
+sampled rows the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_harness import TOL, host_inputs, make_step, max_err, oracle_step, storage
+from paged_kv_cache_446_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from paged_kv_cache_446_b200 import pkv  # noqa: F401  (fails loudly if the library is missing)
+    return torch.device("cuda:0")
+
+
+@pytest.fixture(autouse=True)
+def no_device_error(dev):
+    from paged_kv_cache_446_b200 import pkv
+    pkv.device_error()
+    yield
+    code, detail = pkv.device_error()
+    assert code == 0, f"device error word set: code {code}, detail {detail}"
+
+
+def run_and_compare(wl, dev, rows=None, **opts):
+    h = host_inputs(wl)
+    step = make_step(wl, dev, **opts)
+    out = step.run(wl.q, wl.k_pool, wl.v_pool, wl.scale, wl.k_new, wl.v_new)
+    torch.cuda.synchronize()
+    ref = oracle_step(wl, h, rows=rows)
+    got = out if rows is None else out[torch.as_tensor(rows, device=out.device, dtype=torch.long)]
+    err = max_err(got, ref)
+    assert err <= TOL[wl.dtype], f"{wl.name}: max |err| {err:.3g} > {TOL[wl.dtype]}"
+    return err, step
+
+
+@pytest.mark.parametrize("config", W.CONFIGS)
+def test_step_small_all_outputs(dev, config):
+    wl = W.make(config, device=dev, small=True)
+    run_and_compare(wl, dev)
+
+
+@pytest.mark.parametrize("config", W.CONFIGS)
+def test_step_full_size_sampled(dev, config):
+    wl = W.make(config, device=dev)
+    qsl, ctx = oracle.flatten_batch(wl.batch, wl.prior_lens)
+    T = int(qsl[-1])
+    rng = np.random.default_rng(7)
+    rows = set(rng.choice(T, size=min(T, 24), replace=False).tolist())
+    # always include the longest decode row, and every prefill request's first and last row
+    dec = [r for r, n in enumerate(wl.batch.values()) if n == 1]
+    if dec:
+        rows.add(int(qsl[max(dec, key=lambda r: ctx[r])]))
+    for r, n in enumerate(wl.batch.values()):
+        if n > 1:
+            rows.update([int(qsl[r]), int(qsl[r + 1]) - 1])
+    run_and_compare(wl, dev, rows=np.asarray(sorted(rows), np.int32))
+
+
+@pytest.mark.parametrize("opts", [{"no_split": True}, {"split_blocks": 1}, {"split_blocks": 2},
+                                  {"split_blocks": 5}, {}])
+def test_split_count_independence(dev, opts):
+    wl = W.make("c3", device=dev, small=True)
+    run_and_compare(wl, dev, **opts)
+
+
+def test_cuda_core_path_on_prefill_rows(dev):
+    """The CUDA-core path serves chunked-prefill rows too (one row at a time, causal limit)."""
+    wl = W.make("c5", device=dev, small=True)
+    run_and_compare(wl, dev, cuda_core_only=True)
+
+
+def sentinel_pool(shape, dtype, dev, seed):
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    bits = torch.randint(-32768, 32767, shape, generator=g, device=dev, dtype=torch.int16)
+    if dtype == torch.float32:
+        bits = torch.randint(-2**31, 2**31 - 1, shape, generator=g, device=dev, dtype=torch.int32)
+    return bits.view(dtype)
+
+
+@pytest.mark.parametrize("config,small", [("c2", True), ("c3", True), ("c5", True), ("c4", True), ("c2", False),
+                                          ("c5", False)])
+def test_slot_mapping_and_kv_write_bit_exact(dev, config, small):
+    from paged_kv_cache_446_b200 import pkv
+    wl = W.make(config, device=dev, small=small)
+    shape = tuple(wl.k_pool.shape)
+    dt = W.TORCH_DTYPES[wl.dtype]
+    kp = sentinel_pool(shape, dt, dev, 1)
+    vp = sentinel_pool(shape, dt, dev, 2)
+    hk, hv = storage(kp), storage(vp)
+    step = make_step(wl, dev)
+    pkv.slot_mapping(step.block_tables, step.write_qsl, step.write_ctx, wl.num_blocks, step.num_write, out=step.slots)
+    pkv.kv_cache_write(wl.k_new, wl.v_new, kp, vp, step.slots)
+    torch.cuda.synchronize()
+    counts = np.asarray(list(wl.batch.values()), dtype=np.int64)
+    ctx_after = np.asarray(wl.prior_lens, dtype=np.int64) + counts
+    wcounts = np.asarray([wl.write_batch.get(r, 0) for r in wl.batch.keys()], dtype=np.int64)
+    wqsl, wctx = oracle.flatten_batch(dict(zip(wl.batch.keys(), wcounts)), ctx_after - wcounts)
+    slots = oracle.slot_mapping(wl.block_tables, wqsl, wctx)
+    assert np.array_equal(step.slots.cpu().numpy(), slots)
+    oracle.kv_cache_write(storage(wl.k_new), storage(wl.v_new), hk, hv, slots)
+    assert np.array_equal(storage(kp), hk)
+    assert np.array_equal(storage(vp), hv)
+
+
+@pytest.mark.parametrize("layers", [1, 3])
+def test_copy_blocks_bit_exact(dev, layers):
+    from paged_kv_cache_446_b200 import pkv
+    wl = W.make("c4", device=dev, small=False, with_tensors=False)
+    shape = (wl.num_blocks, wl.num_kv_heads, 16, wl.head_dim)
+    kps = [sentinel_pool(shape, torch.float16, dev, 10 + i) for i in range(layers)]
+    vps = [sentinel_pool(shape, torch.float16, dev, 20 + i) for i in range(layers)]
+    hk = [storage(p) for p in kps]
+    hv = [storage(p) for p in vps]
+    pairs = torch.from_numpy(wl.copy_pairs).to(dev)
+    pkv.validate_copy_pairs(wl.copy_pairs, wl.num_blocks)
+    pkv.copy_blocks(kps, vps, pairs)
+    torch.cuda.synchronize()
+    oracle.copy_blocks(hk, hv, wl.copy_pairs)
+    for i in range(layers):
+        assert np.array_equal(storage(kps[i]), hk[i])
+        assert np.array_equal(storage(vps[i]), hv[i])
+
+
+def test_block_permutation_bit_identical(dev):
+    """Relabelling physical blocks (pool and tables together) leaves every output bit unchanged."""
+    wl = W.make("c3", device=dev, small=True)
+    wl.write_batch = {}
+    step = make_step(wl, dev)
+    base = step.run(wl.q, wl.k_pool, wl.v_pool, wl.scale).clone()
+    perm = torch.randperm(wl.num_blocks, generator=torch.Generator().manual_seed(3))
+    kp = torch.empty_like(wl.k_pool)
+    vp = torch.empty_like(wl.v_pool)
+    kp[perm.to(dev)] = wl.k_pool
+    vp[perm.to(dev)] = wl.v_pool
+    bt = wl.block_tables.copy()
+    pn = perm.numpy()
+    bt[bt >= 0] = pn[bt[bt >= 0]]
+    wl.block_tables = bt
+    out = make_step(wl, dev).run(wl.q, kp, vp, wl.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out, base)
+
+
+def custom(dev, dtype, Hq, Hkv, D, specs, seed=5):
+    """A workload with explicit (prior, num_tokens) rows over a shuffled pool."""
+    rng = np.random.default_rng(seed)
+    ctx = np.asarray([p + n for p, n in specs], np.int64)
+    need = [int(-(-c // 16)) for c in ctx]
+    NB = max(1, int(math.ceil(1.2 * sum(need))) + 1)
+    perm = rng.permutation(NB).astype(np.int32)
+    bt = np.full((len(specs), max(max(need), 1)), -1, np.int32)
+    pos = 0
+    for r, k in enumerate(need):
+        bt[r, :k] = perm[pos:pos + k]
+        pos += k
+    batch = {r: n for r, (_, n) in enumerate(specs)}
+    wl = W.Workload(name="custom", dtype=dtype, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                    scale=float(np.float32(1 / math.sqrt(D))), batch=batch,
+                    prior_lens=np.asarray([p for p, _ in specs], np.int32), block_tables=bt, num_blocks=NB,
+                    write_batch={}, copy_pairs=np.zeros((0, 2), np.int32), seed=seed)
+    W._draw_tensors(wl, dev)
+    return wl
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,specs", [
+    ("f16", 8, 8, 128, [(0, 1)]),                                  # context of one token
+    ("bf16", 32, 2, 128, [(31, 1), (16, 1), (200, 1)]),            # group of 16 query heads
+    ("f16", 16, 8, 64, [(100, 1), (15, 1), (47, 3)]),              # head_dim 64, 16-bit
+    ("f32", 16, 4, 128, [(90, 1), (7, 2)]),                        # fp32, head_dim 128
+    ("bf16", 12, 4, 128, [(50, 1), (3, 1)]),                       # group of 3 (padded to 4)
+    ("f16", 8, 8, 128, [(0, 0), (20, 1), (0, 0), (63, 1)]),       # requests with no rows this step
+    ("bf16", 64, 8, 128, [(16 * 2080 - 1, 1)]),                    # 33280-token context
+    ("f16", 8, 2, 128, [(0, 17), (5, 130)]),                       # prefill rows, ragged tiles
+])
+def test_edge_cases(dev, dtype, Hq, Hkv, D, specs):
+    run_and_compare(custom(dev, dtype, Hq, Hkv, D, specs), dev)
+
+
+def test_empty_batch(dev):
+    from paged_kv_cache_446_b200 import pkv
+    plan = pkv.AttentionPlan({}, [], 8, 8, 128, torch.float16, dev)
+    q = torch.empty(0, 8, 128, dtype=torch.float16, device=dev)
+    pool = torch.zeros(1, 8, 16, 128, dtype=torch.float16, device=dev)
+    bt = torch.zeros(1, 1, dtype=torch.int32, device=dev)
+    out = pkv.paged_attention(plan, q, pool, pool, bt, 0.1)
+    assert out.shape == (0, 8, 128)
+
+
+def test_device_error_on_out_of_range_table_entry(dev):
+    """A table entry outside the pool is skipped by the kernel and reported through the error word."""
+    from paged_kv_cache_446_b200 import pkv
+    wl = custom(dev, "f16", 8, 8, 128, [(40, 1), (10, 1)])
+    wl.block_tables[1, 0] = wl.num_blocks + 5
+    make_step(wl, dev).run(wl.q, wl.k_pool, wl.v_pool, wl.scale)
+    code, detail = pkv.device_error()
+    assert code == 6 and detail >= 0
