@@ -217,6 +217,32 @@ pkv_status pkv_validate_copy_pairs(const int32_t* h_pairs, int num_pairs, int nu
 pkv_status pkv_device_error(int* code, int64_t* detail, pkv_stream_t stream);
 
 /*
+ * pkv_paged_attention_static_ws -- plan and run paged attention with no device allocation at all.
+ * The pages have no counterpart to this call; it exists for callers that cannot call cudaMalloc
+ * where they run attention (an engine whose memory manager already owns nearly all of HBM, a
+ * plugin inside a runtime that owns every allocation, code running where allocation calls are
+ * forbidden or would stall). Instead of a caller workspace it uses one library-owned device array
+ * of PKV_STATIC_WS_BYTES, held by every GPU that loads the library until the process exits.
+ * Arguments: the host batch description and options of pkv_attention_plan, then the device
+ * tensors and scale of pkv_paged_attention (same layouts and meaning); out receives the result.
+ * The array's device address is looked up on the first call made on each device, so make that
+ * first call before any stream capture begins. Every call reuses the same array, which keeps the
+ * last call's contents; calls that may overlap on the GPU (other streams or host threads) race on
+ * it and must be serialised by the caller. No part of it has to start zeroed: each call writes
+ * what its kernels read.
+ * Errors: those of pkv_attention_plan and pkv_paged_attention, and WORKSPACE_TOO_SMALL when the
+ * batch needs more scratch than PKV_STATIC_WS_BYTES (checked on the host before any launch).
+ */
+#define PKV_STATIC_WS_BYTES (32u << 20)
+pkv_status pkv_paged_attention_static_ws(const int32_t* h_query_start_loc, const int32_t* h_context_lens,
+                                         int num_reqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                         pkv_dtype dtype, const pkv_plan_options* opts, void* out, const void* q,
+                                         const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                                         int max_blocks_per_seq, const int32_t* context_lens,
+                                         const int32_t* query_start_loc, int num_blocks, float scale,
+                                         pkv_stream_t stream);
+
+/*
  * Kernel timing (no counterpart on the pages; a measurement aid). Between pkv_profile_start and
  * pkv_profile_stop, every kernel the library launches on the calling host thread is bracketed by
  * a pair of CUDA events recorded on the launch stream. pkv_profile_stop synchronises those events,

@@ -213,6 +213,8 @@ struct ProfileScope {
 
 }  // namespace
 
+void set_last_error(const char* msg) { t_last_error = msg ? msg : ""; }
+
 DeviceError* device_error_word() {
     static std::mutex mu;
     static DeviceError* addr[64] = {nullptr};

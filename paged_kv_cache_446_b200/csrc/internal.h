@@ -116,4 +116,7 @@ cudaError_t launch_copy_blocks(void* const* k_pools, void* const* v_pools, int n
 // Device error word of the current device.
 DeviceError* device_error_word();
 
+// Replaces the calling thread's pkv_last_error() message.
+void set_last_error(const char* msg);
+
 }  // namespace pkv
