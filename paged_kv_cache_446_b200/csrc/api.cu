@@ -136,8 +136,16 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     std::stable_sort(L->items.begin(), L->items.end(), [](const DecodeItem& a, const DecodeItem& b) {
         return (a.blk_end - a.blk_begin) > (b.blk_end - b.blk_begin);
     });
-    std::stable_sort(L->tiles.begin(), L->tiles.end(),
-                     [](const PrefillTile& a, const PrefillTile& b) { return a.key_tiles > b.key_tiles; });
+    // Tiles: longest requests first; a (request, KV head)'s tiles stay adjacent (longest first) so
+    // the CTAs running at the same time share that head's K/V through L2.
+    std::vector<int> req_keys(R > 0 ? R : 1, 0);
+    for (const PrefillTile& t : L->tiles) req_keys[t.req] = std::max(req_keys[t.req], t.key_tiles);
+    std::stable_sort(L->tiles.begin(), L->tiles.end(), [&](const PrefillTile& a, const PrefillTile& b) {
+        if (req_keys[a.req] != req_keys[b.req]) return req_keys[a.req] > req_keys[b.req];
+        if (a.req != b.req) return a.req < b.req;
+        if (a.kv_head != b.kv_head) return a.kv_head < b.kv_head;
+        return a.tok0 > b.tok0;
+    });
 
     std::memset(plan, 0, sizeof *plan);
     plan->magic = PKV_PLAN_MAGIC;

@@ -1,10 +1,480 @@
-// tcgen05 chunked-prefill tiles (not yet enabled: every row goes to the CUDA-core kernel).
+// Chunked-prefill attention tiles on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// What it computes: for a request with n > 1 query rows at prior context P (blog.mckayzhao.com/?p=56,
+// "进阶特性：让推理再快一点" -- chunked prefill; "V1 架构：推倒重来的勇气" -- one mixed batch), row j
+// attends keys 0 .. P+j of the request's cache, read block by block through its block table
+// ("PagedAttention：操作系统课本里翻出来的灵感"). Here QK^T and PV are dense contractions, so they run
+// on tcgen05 with fp32 accumulation in tensor memory; softmax stays in fp32 on the CUDA cores and
+// P is rounded to the input type for the PV product.
+//
+// Tile: 128 MMA rows = (128/G) consecutive query rows x the G query heads of one KV head (GQA
+// packing: each K/V tile is loaded once for all G heads). Key tiles of 128 = 8 blocks.
+// Warp roles (320 threads):
+//   warps 0-7  softmax: two threads per row (64 key columns / 64 output columns each)
+//   warp  8    TMA producer: Q once (3-D tensor map, SWIZZLE_128B), then per key tile 8 blocks x
+//              2 column halves of K and of V (2-D tensor map over the pool rows), double-buffered
+//   warp  9    MMA issuer (one thread): S = Q K^T into one of two TMEM S buffers (so the next
+//              tile's QK^T overlaps this tile's softmax), O_tile = P V into TMEM; completion is
+//              signalled to mbarriers with tcgen05.commit
+// Softmax threads fold each O_tile into fp32 registers with the running-max correction.
+// Blocks past the context are fetched at an out-of-range coordinate (TMA fills zeros); V rows past
+// the context inside the last block are zeroed before PV (stale slots may hold anything).
+// Every wait is bounded; on expiry the CTA records PKV_ERR_DEVICE_TIMEOUT, drains its own copies
+// and MMAs (bounded), frees its tensor memory and returns. No TMA multicast.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace pkv {
+namespace {
 
-bool prefill_tc_supported(int, int, int) { return false; }
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kHalf = 128 * 128;        // 128 rows x 64 elements x 2 bytes
+constexpr int kTile = 2 * kHalf;        // 128 x 128 x 2 bytes
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + kTile;    // 2 stages
+constexpr int OFF_V = OFF_K + 2 * kTile;
+constexpr int OFF_P = OFF_V + 2 * kTile;
+constexpr int OFF_BAR = OFF_P + kTile;
+// barrier slots (8 bytes each)
+enum { B_Q = 0, B_KF0 = 1, B_VF0 = 3, B_KE0 = 5, B_SF0 = 7, B_PF = 9, B_OF = 10, B_DRAIN = 11, NUM_BARS = 12 };
+constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;     // tcgen05.alloc result
+constexpr int OFF_ABORT = OFF_TMEM + 4;
+constexpr int OFF_MAXX = OFF_BAR + 128;              // [2 parity][2 half][128 rows] floats
+constexpr int OFF_SUMX = OFF_MAXX + 2 * 2 * 128 * 4; // [2 half][128 rows]
+constexpr int SMEM_USED = OFF_SUMX + 2 * 128 * 4;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;         // slack to align the base to 1024 bytes
+constexpr uint32_t kTmemCols = 512;                  // S0 [0,128), S1 [128,256), O [256,384)
 
-cudaError_t launch_prefill_tc(int, const PrefillArgs&, int, cudaStream_t) { return cudaErrorNotSupported; }
+// ---- tcgen05 / TMA primitives ---------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc)
+        : "memory");
+}
+// 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives TMEM lane (base lane + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, SWIZZLE_128B (layout type 2), descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo, uint32_t sbo) {
+    const uint32_t a = smem_u32(p);
+    return (uint64_t)((a >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor of kind::f16 with fp32 accumulation, M = N = 128.
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_format, uint32_t b_mn_major) {
+    return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (b_mn_major << 16) | ((128u >> 3) << 17) |
+           ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ bool bar_or(bool v) {  // named barrier 1 over the 256 softmax threads
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Bounded wait that also gives up when another role has aborted the CTA.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag, DeviceError* err,
+                                              int where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > WAIT_BUDGET_CYCLES) {
+            *abort_flag = 1;
+            record_error(err, 5 /*PKV_ERR_DEVICE_TIMEOUT*/, where);
+            return false;
+        }
+    }
+    return true;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+    float* maxx = reinterpret_cast<float*>(smem + OFF_MAXX);
+    float* sumx = reinterpret_cast<float*>(smem + OFF_SUMX);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const PrefillTile tile = a.tiles[blockIdx.x];
+    const int req = tile.req, kvh = tile.kv_head, tok0 = tile.tok0;
+    const int q0 = a.query_start_loc[req];
+    const int n = a.query_start_loc[req + 1] - q0;
+    const int ctx = a.context_lens[req];
+    const int prior = ctx - n;
+    const int G = a.group;
+    const int tt = 128 / G;
+    const int last = min(n, tok0 + tt);
+    const int keys = min(ctx, prior + last);
+    const int nkt = (keys + 127) / 128;
+    const int nblk_ctx = (ctx + kBlockSize - 1) / kBlockSize;
+    const int rows_total = a.num_blocks * a.num_kv_heads * kBlockSize;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[B_Q], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[B_KF0 + s], 1);
+            mbar_init(&bars[B_VF0 + s], 1);
+            mbar_init(&bars[B_KE0 + s], 1);
+            mbar_init(&bars[B_SF0 + s], 1);
+        }
+        mbar_init(&bars[B_PF], kSoftmaxThreads);
+        mbar_init(&bars[B_OF], 1);
+        mbar_init(&bars[B_DRAIN], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem + OFF_TMEM)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
+    const bool sane = nkt >= 1 && n > 1 && tok0 < n;
+
+    if (warp == 8 && sane) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bars[B_Q], kTile);
+            tma_load_3d(smem + OFF_Q, &tm_q, 0, kvh * G, q0 + tok0, &bars[B_Q]);
+            tma_load_3d(smem + OFF_Q + kHalf, &tm_q, 64, kvh * G, q0 + tok0, &bars[B_Q]);
+        }
+        int ids = -1, ids_base = -1;
+        int issued_k[2] = {-1, -1};
+        bool ok = true;
+        for (int kt = 0; kt < nkt && ok; ++kt) {
+            const int s = kt & 1;
+            if (kt >= 2) ok = wait_or_abort(&bars[B_KE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 100 + kt);
+            if (!ok) break;
+            if (ids_base < 0 || kt * 8 >= ids_base + 32) {
+                ids_base = kt * 8;
+                const int b = ids_base + lane;
+                ids = b < nblk_ctx ? __ldg(a.block_tables + (size_t)req * a.max_blocks_per_seq + b) : -2;
+            }
+            int y[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int id = __shfl_sync(FULL_MASK, ids, kt * 8 - ids_base + i);
+                if (id == -2) y[i] = rows_total;                       // past the context: zero fill
+                else if (id < 0 || id >= a.num_blocks) {
+                    if (lane == 0) record_error(a.err, 6 /*PKV_ERR_DEVICE_RANGE*/, (long long)req * a.max_blocks_per_seq + kt * 8 + i);
+                    y[i] = rows_total;
+                } else y[i] = (id * a.num_kv_heads + kvh) * kBlockSize;
+            }
+            if (lane == 0) {
+                unsigned char* ks = smem + OFF_K + s * kTile;
+                unsigned char* vs = smem + OFF_V + s * kTile;
+                mbar_arrive_expect_tx(&bars[B_KF0 + s], kTile);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    tma_load_2d(ks + i * 2048, &tm_k, 0, y[i], &bars[B_KF0 + s]);
+                    tma_load_2d(ks + kHalf + i * 2048, &tm_k, 64, y[i], &bars[B_KF0 + s]);
+                }
+                mbar_arrive_expect_tx(&bars[B_VF0 + s], kTile);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    tma_load_2d(vs + i * 2048, &tm_v, 0, y[i], &bars[B_VF0 + s]);
+                    tma_load_2d(vs + kHalf + i * 2048, &tm_v, 64, y[i], &bars[B_VF0 + s]);
+                }
+            }
+            issued_k[s] = kt;
+            __syncwarp();
+        }
+        if (!ok && lane == 0) {
+            // Drain: wait (bounded) for the last loads issued into each stage.
+            for (int s = 0; s < 2; ++s)
+                if (issued_k[s] >= 0) {
+                    (void)mbar_wait(&bars[B_KF0 + s], (issued_k[s] >> 1) & 1);
+                    (void)mbar_wait(&bars[B_VF0 + s], (issued_k[s] >> 1) & 1);
+                }
+            (void)mbar_wait(&bars[B_Q], 0);
+        }
+    } else if (warp == 9 && sane) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            const uint32_t fmt = sizeof(T) == 2 && !std::is_same<T, __half>::value ? 1u : 0u;
+            const uint32_t id_qk = idesc_f16(fmt, 0);
+            const uint32_t id_pv = idesc_f16(fmt, 1);
+            bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, a.err, 200);
+            auto issue_qk = [&](int kt) {
+                const int s = kt & 1;
+                const unsigned char* ks = smem + OFF_K + s * kTile;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int half = k >> 2, off = (k & 3) * 32;
+                    tc_mma(tmem + s * 128, smem_desc(smem + OFF_Q + half * kHalf + off, 16, 1024),
+                           smem_desc(ks + half * kHalf + off, 16, 1024), id_qk, k > 0);
+                }
+                tc_commit(&bars[B_SF0 + s]);
+            };
+            if (ok) ok = wait_or_abort(&bars[B_KF0], 0, abort_flag, a.err, 201);
+            if (ok) {
+                tc_fence_after();
+                issue_qk(0);
+            }
+            for (int kt = 0; kt < nkt && ok; ++kt) {
+                if (kt + 1 < nkt) {
+                    ok = wait_or_abort(&bars[B_KF0 + ((kt + 1) & 1)], ((kt + 1) >> 1) & 1, abort_flag, a.err, 202);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk(kt + 1);
+                }
+                ok = wait_or_abort(&bars[B_PF], kt & 1, abort_flag, a.err, 203);
+                if (ok) ok = wait_or_abort(&bars[B_VF0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 204);
+                if (!ok) break;
+                tc_fence_after();
+                const unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int half = k >> 2, off = (k & 3) * 32;
+                    tc_mma(tmem + 256, smem_desc(smem + OFF_P + half * kHalf + off, 16, 1024),
+                           smem_desc(vs + k * 2048, kHalf, 1024), id_pv, k > 0);
+                }
+                tc_commit(&bars[B_OF]);
+                tc_commit(&bars[B_KE0 + (kt & 1)]);
+            }
+            if (ok) {
+                (void)wait_or_abort(&bars[B_KE0 + ((nkt - 1) & 1)], ((nkt - 1) >> 1) & 1, abort_flag, a.err, 205);
+            } else {
+                tc_commit(&bars[B_DRAIN]);
+                (void)mbar_wait(&bars[B_DRAIN], 0);
+            }
+        }
+    } else if (warp < 8 && sane) {
+        // ------------------------------ softmax ------------------------------
+        const int row = (warp & 3) * 32 + lane;
+        const int half = warp >> 2;
+        const int t_local = row / G, g = row % G;
+        const int j = tok0 + t_local;
+        const bool row_valid = j < n;
+        const int limit = row_valid ? prior + j + 1 : prior + 1;  // keys visible: [0, limit)
+        const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        float acc[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+        float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+        bool failed = false;
+        for (int kt = 0; kt < nkt; ++kt) {
+            const int sb = kt & 1;
+            bool ok = wait_or_abort(&bars[B_SF0 + sb], (kt >> 1) & 1, abort_flag, a.err, 300);
+            float s[64];
+            float mx = -INFINITY;
+            if (ok) {
+                tc_fence_after();
+                tmem_ld32(tl + sb * 128 + half * 64, s);
+                tmem_ld32(tl + sb * 128 + half * 64 + 32, s + 32);
+                tmem_wait_ld();
+                const int key0 = kt * 128 + half * 64;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const float v = (key0 + i < limit) ? s[i] * a.scale_log2 : -INFINITY;
+                    s[i] = v;
+                    mx = fmaxf(mx, v);
+                }
+                maxx[(sb * 2 + half) * 128 + row] = mx;
+            }
+            if (ok && kt >= 1) ok = wait_or_abort(&bars[B_OF], (kt - 1) & 1, abort_flag, a.err, 301);
+            const bool zero_v = (kt == nkt - 1) && (kt + 1) * 128 > ctx;
+            if (ok && zero_v) ok = wait_or_abort(&bars[B_VF0 + sb], (kt >> 1) & 1, abort_flag, a.err, 302);
+            if (bar_or(!ok)) {
+                failed = true;
+                break;
+            }
+            const float m_new = fmaxf(m, fmaxf(mx, maxx[(sb * 2 + (half ^ 1)) * 128 + row]));
+            const float alpha = fast_exp2(m - m_new);
+            float ps = 0.f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                s[i] = fast_exp2(s[i] - m_new);
+                ps += s[i];
+            }
+            l = l * alpha + ps;
+            if (kt >= 1) {
+                tc_fence_after();
+                float o[32];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    tmem_ld32(tl + 256 + half * 64 + c * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(acc[c * 32 + i], alpha_prev, o[i]);
+                }
+            }
+            alpha_prev = alpha;
+            m = m_new;
+            // P (rounded to T) into the SWIZZLE_128B K-major operand layout.
+            unsigned char* prow = smem + OFF_P + half * kHalf + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = Chunk<T>::pack(s + c * 8);
+            if (zero_v) {
+                unsigned char* vs = smem + OFF_V + sb * kTile;
+                const int r0 = ctx - kt * 128;  // first V row past the context
+                const int chunks = (128 - r0) * 16;  // 16-byte chunks over both halves
+                for (int c = threadIdx.x; c < chunks; c += kSoftmaxThreads) {
+                    const int r = r0 + (c >> 4), h = (c >> 3) & 1, k = c & 7;
+                    *reinterpret_cast<uint4*>(vs + h * kHalf + r * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_PF]);
+        }
+        if (!failed) {
+            bool ok = wait_or_abort(&bars[B_OF], (nkt - 1) & 1, abort_flag, a.err, 303);
+            if (ok) {
+                tc_fence_after();
+                float o[32];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    tmem_ld32(tl + 256 + half * 64 + c * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(acc[c * 32 + i], alpha_prev, o[i]);
+                }
+                sumx[half * 128 + row] = l;
+            }
+            if (!bar_or(!ok) && row_valid) {
+                const float inv = 1.f / (l + sumx[(half ^ 1) * 128 + row]);
+                unsigned char* dst = static_cast<unsigned char*>(a.out) +
+                                     ((size_t)(q0 + j) * a.num_q_heads + (size_t)kvh * G + g) * 256 + half * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = acc[c * 8 + e] * inv;
+                    *reinterpret_cast<uint4*>(dst + c * 16) = Chunk<T>::pack(v);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// ---- host side: tensor maps ------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode(CUtensorMap* m, CUtensorMapDataType t, int rank, const void* base, const cuuint64_t* dims,
+            const cuuint64_t* strides, const cuuint32_t* box) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, t, rank, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
+    const CUtensorMapDataType dt =
+        std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int G = a.group;
+    CUtensorMap mq, mk, mv;
+    const cuuint64_t qdims[3] = {128, (cuuint64_t)a.num_q_heads, (cuuint64_t)a.num_q_tokens};
+    const cuuint64_t qstr[2] = {128 * 2, (cuuint64_t)a.num_q_heads * 128 * 2};
+    const cuuint32_t qbox[3] = {64, (cuuint32_t)G, (cuuint32_t)(128 / G)};
+    const long long rows = (long long)a.num_blocks * a.num_kv_heads * kBlockSize;
+    const cuuint64_t kdims[2] = {128, (cuuint64_t)rows};
+    const cuuint64_t kstr[1] = {128 * 2};
+    const cuuint32_t kbox[2] = {64, (cuuint32_t)kBlockSize};
+    if (!encode(&mq, dt, 3, a.q, qdims, qstr, qbox) || !encode(&mk, dt, 2, a.k_pool, kdims, kstr, kbox) ||
+        !encode(&mv, dt, 2, a.v_pool, kdims, kstr, kbox))
+        return cudaErrorInvalidValue;
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(prefill_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = 1;
+    }
+    prefill_tc_kernel<T><<<a.num_tiles, kThreads, SMEM_BYTES, s>>>(a, mq, mk, mv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int dtype, int head_dim, int group) {
+    return (dtype == 1 || dtype == 2) && head_dim == 128 && group >= 1 && group <= 16 && (128 % group) == 0;
+}
+
+cudaError_t launch_prefill_tc(int dtype, const PrefillArgs& a, int /*num_sms*/, cudaStream_t s) {
+    if (a.num_tiles <= 0) return cudaSuccess;
+    if ((long long)a.num_blocks * a.num_kv_heads * kBlockSize >= (1LL << 31) - 1) return cudaErrorInvalidValue;
+    if (((uintptr_t)a.q | (uintptr_t)a.k_pool | (uintptr_t)a.v_pool) & 15) return cudaErrorInvalidValue;
+    return dtype == 1 ? launch_t<__half>(a, s) : launch_t<__nv_bfloat16>(a, s);
+}
 
 }  // namespace pkv

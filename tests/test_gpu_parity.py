@@ -208,3 +208,32 @@ def test_device_error_on_out_of_range_table_entry(dev):
     make_step(wl, dev).run(wl.q, wl.k_pool, wl.v_pool, wl.scale)
     code, detail = pkv.device_error()
     assert code == 6 and detail >= 0
+
+
+PREFILL_CASES = [
+    ("bf16", 64, 8, 128, [(0, 512)]),                              # first 512-row chunk, G = 8
+    ("bf16", 64, 8, 128, [(300, 80), (0, 1), (17, 33)]),           # mixed rows, ragged tiles
+    ("f16", 32, 32, 128, [(0, 200), (129, 130)]),                  # G = 1: 128 rows per tile
+    ("bf16", 32, 2, 128, [(5, 40)]),                               # G = 16: 8 rows per tile
+    ("f16", 16, 8, 128, [(1000, 3)]),                              # few rows, long prior
+    ("bf16", 8, 8, 128, [(0, 2)]),                                 # two rows
+    ("f16", 64, 16, 128, [(4096 - 7, 45), (250, 1)]),              # prior not block aligned
+]
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,specs", PREFILL_CASES)
+def test_prefill_tiles_tcgen05(dev, dtype, Hq, Hkv, D, specs):
+    wl = custom(dev, dtype, Hq, Hkv, D, specs, seed=11)
+    _, step = run_and_compare(wl, dev)
+    assert step.plan.plan.num_tiles > 0, "expected the tcgen05 tile path"
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,specs", PREFILL_CASES[:4])
+def test_prefill_tiles_match_cuda_core_path(dev, dtype, Hq, Hkv, D, specs):
+    """The tcgen05 tiles and the CUDA-core kernel agree on the same prefill rows."""
+    wl = custom(dev, dtype, Hq, Hkv, D, specs, seed=12)
+    a = make_step(wl, dev).run(wl.q, wl.k_pool, wl.v_pool, wl.scale).clone()
+    b = make_step(wl, dev, cuda_core_only=True).run(wl.q, wl.k_pool, wl.v_pool, wl.scale)
+    torch.cuda.synchronize()
+    err = (a.double() - b.double()).abs().max().item()
+    assert err <= TOL[wl.dtype], err
