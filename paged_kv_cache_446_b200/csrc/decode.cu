@@ -16,6 +16,7 @@
 // butterfly reduce-scatter of warp shuffles; the online softmax is per query head in fp32 (log2
 // domain, ex2.approx); P*V accumulates in fp32 registers. Items covering part of a row write
 // (unnormalised output, max, sum) partials; merge_kernel combines them by log-sum-exp.
+#include <cstdlib>
 #include <type_traits>
 
 #include "common.cuh"
@@ -27,7 +28,7 @@ constexpr int log2i(int x) { return x <= 1 ? 0 : 1 + log2i(x / 2); }
 constexpr int round16(int x) { return (x + 15) / 16 * 16; }
 constexpr int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
 
-template <typename T, int D, int GP>
+template <typename T, int D, int GP, int NSTAGE>
 struct Dec {
     static constexpr int EB = sizeof(T);
     static constexpr int ROW = D * EB;                 // bytes of one K/V row
@@ -35,6 +36,7 @@ struct Dec {
     static constexpr int LOG_CPR = log2i(CPR);
     static constexpr int TPP = 32 / CPR;               // rows (tokens) handled per warp pass
     static constexpr int EPC = 16 / EB;                // elements per chunk
+    static constexpr int E2 = EPC / 2;                 // element pairs per chunk
     static constexpr int PASSES = kBlockSize / TPP;    // passes per 16-token block
     static constexpr int LOG_PASSES = log2i(PASSES);
     static constexpr int NV = GP * PASSES;             // partial dots per lane per block
@@ -44,7 +46,7 @@ struct Dec {
     static constexpr int BLK = kBlockSize * ROW;       // bytes of one (block, head) K or V chunk
     static constexpr int QB = GP * ROW;                // bytes of an item's query rows
     static constexpr int STAGE = 2 * BLK + QB;
-    static constexpr int STAGES = clampi((32 * 1024) / STAGE, 2, 4);
+    static constexpr int STAGES = NSTAGE;
     static constexpr int P_FLOATS = GP * TPP * PASSES; // softmax weights of one block
     static constexpr int SCR = round16(P_FLOATS * 4 + GP * 4 + GP * 8);
     static constexpr int WARP_SMEM = STAGES * STAGE + SCR + round16(STAGES * 8);
@@ -55,6 +57,11 @@ struct Dec {
 
 constexpr int kDecodeWarps = 2;  // independent warps per CTA
 
+// Default ring depth: three stages for small groups (pure streaming), two for large groups
+// (more resident warps matter more there, the kernel being issue-bound).
+template <int GP>
+constexpr int default_stages() { return GP >= 4 ? 2 : 3; }
+
 __device__ __forceinline__ DecodeItem load_item(const DecodeItem* items, int i) {
     const int4* p = reinterpret_cast<const int4*>(items + i);
     const int4 a = __ldg(p), b = __ldg(p + 1);
@@ -64,9 +71,9 @@ __device__ __forceinline__ DecodeItem load_item(const DecodeItem* items, int i) 
     return it;
 }
 
-template <typename T, int D, int GP>
+template <typename T, int D, int GP, int NSTAGE>
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeArgs a) {
-    using C = Dec<T, D, GP>;
+    using C = Dec<T, D, GP, NSTAGE>;
     extern __shared__ __align__(128) unsigned char smem[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -152,17 +159,23 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
     int c_blk = ci.blk_begin;
     uint32_t consumed = 0;
 
-    float q[GP][C::EPC];
-    float acc[GP][C::EPC];
-    float m_own = -INFINITY, l_own = 0.f;
-
-    // Owned dots after the reduce-scatter: indices base .. base+NOWN-1 of (g * PASSES + i).
-    int base = 0;
+    // Dots are indexed x = head * PASSES + pass. The butterfly reduce-scatter halves the index range
+    // each round, the lane keeping the half selected by its own lane bit. Storing slot s as logical
+    // index s ^ M (M = the lane's kept bits) puts the kept half always in the low slots, so a round
+    // is one shuffle and one add per value. M is applied by loading q heads in permuted order and by
+    // permuting which token each pass reads.
+    int M = 0;
 #pragma unroll
     for (int r = 0; r < C::SPLIT; ++r)
-        if (lane & (C::CPR >> (r + 1))) base += C::NV >> (r + 1);
-    const int g_own = base / C::PASSES;
-    const int i_own0 = base % C::PASSES;
+        if (lane & (C::CPR >> (r + 1))) M |= C::NV >> (r + 1);
+    const int g_own = M / C::PASSES;           // head whose scores this lane owns after the rounds
+    const int i_own0 = M % C::PASSES;          // first owned pass
+    const int gm = M / C::PASSES;              // head-slot permutation
+    const int im = M % C::PASSES;              // pass permutation
+
+    float2 q2[GP][C::E2];                      // q (scaled, log2 domain), head slots permuted by gm
+    float2 acc2[GP][C::E2];                    // output accumulator, logical head order
+    float m_own = -INFINITY, l_own = 0.f;
 
     while (true) {
         const int stage = consumed % C::STAGES;
@@ -181,50 +194,47 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
 
         if (c_blk == ci.blk_begin) {
 #pragma unroll
-            for (int g = 0; g < GP; ++g) {
+            for (int gs = 0; gs < GP; ++gs) {
+                const int g = gs ^ gm;
                 if (g < nh) {
-                    Chunk<T>::unpack(lds128(st + 2 * C::BLK + g * C::ROW + chunk * 16), q[g]);
+                    float f[C::EPC];
+                    Chunk<T>::unpack(lds128(st + 2 * C::BLK + g * C::ROW + chunk * 16), f);
 #pragma unroll
-                    for (int e = 0; e < C::EPC; ++e) q[g][e] *= a.scale_log2;
+                    for (int e = 0; e < C::E2; ++e) q2[gs][e] = make_float2(f[2 * e] * a.scale_log2, f[2 * e + 1] * a.scale_log2);
                 } else {
 #pragma unroll
-                    for (int e = 0; e < C::EPC; ++e) q[g][e] = 0.f;
+                    for (int e = 0; e < C::E2; ++e) q2[gs][e] = make_float2(0.f, 0.f);
                 }
 #pragma unroll
-                for (int e = 0; e < C::EPC; ++e) acc[g][e] = 0.f;
+                for (int e = 0; e < C::E2; ++e) acc2[gs][e] = make_float2(0.f, 0.f);
             }
             m_own = -INFINITY;
             l_own = 0.f;
         }
         const int valid = min(kBlockSize, ci.limit - c_blk * kBlockSize);
 
-        // ---- QK: partial dots of this lane's chunk for every (head, pass) ----
+        // ---- QK: partial dots of this lane's chunk for every (head slot, pass slot) ----
         float dots[C::NV];
 #pragma unroll
-        for (int i = 0; i < C::PASSES; ++i) {
+        for (int is = 0; is < C::PASSES; ++is) {
             float k[C::EPC];
-            Chunk<T>::unpack(lds128(Ks + (i * C::TPP + sub) * C::ROW + chunk * 16), k);
+            Chunk<T>::unpack(lds128(Ks + ((is ^ im) * C::TPP + sub) * C::ROW + chunk * 16), k);
 #pragma unroll
-            for (int g = 0; g < GP; ++g) {
-                float d = 0.f;
+            for (int gs = 0; gs < GP; ++gs) {
+                float2 d2 = __fmul2_rn(q2[gs][0], make_float2(k[0], k[1]));
 #pragma unroll
-                for (int e = 0; e < C::EPC; ++e) d = fmaf(q[g][e], k[e], d);
-                dots[g * C::PASSES + i] = d;
+                for (int e = 1; e < C::E2; ++e) d2 = __ffma2_rn(q2[gs][e], make_float2(k[2 * e], k[2 * e + 1]), d2);
+                dots[gs * C::PASSES + is] = d2.x + d2.y;
             }
         }
-        // ---- reduce-scatter across the CPR lanes of a row ----
+        // ---- reduce-scatter across the CPR lanes of a row (kept half always in the low slots) ----
 #pragma unroll
         for (int r = 0; r < C::LOG_CPR; ++r) {
             const int o = C::CPR >> (r + 1);
             if (r < C::LOG_NV) {
                 const int h = C::NV >> (r + 1);
-                const bool upper = (lane & o) != 0;
 #pragma unroll
-                for (int k = 0; k < h; ++k) {
-                    const float send = upper ? dots[k] : dots[k + h];
-                    const float keep = upper ? dots[k + h] : dots[k];
-                    dots[k] = keep + __shfl_xor_sync(FULL_MASK, send, o);
-                }
+                for (int k = 0; k < h; ++k) dots[k] += __shfl_xor_sync(FULL_MASK, dots[k + h], o);
             } else {
                 dots[0] += __shfl_xor_sync(FULL_MASK, dots[0], o);
             }
@@ -262,12 +272,17 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
         alpha_s[g_own] = alpha;
         __syncwarp();
 
-        // ---- P*V ----
+        // ---- P*V (logical head order) ----
+        bool rescale = false;
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-            const float al = alpha_s[g];
+        for (int g = 0; g < GP; ++g) rescale |= alpha_s[g] != 1.f;
+        if (rescale) {  // warp-uniform: every lane reads the same alphas
 #pragma unroll
-            for (int e = 0; e < C::EPC; ++e) acc[g][e] *= al;
+            for (int g = 0; g < GP; ++g) {
+                const float al = alpha_s[g];
+#pragma unroll
+                for (int e = 0; e < C::E2; ++e) acc2[g][e] = __fmul2_rn(acc2[g][e], make_float2(al, al));
+            }
         }
 #pragma unroll
         for (int i4 = 0; i4 < C::PASSES; i4 += 4) {
@@ -287,8 +302,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
 #pragma unroll
                 for (int g = 0; g < GP; ++g) {
                     const float p = ii == 0 ? pw[g].x : ii == 1 ? pw[g].y : ii == 2 ? pw[g].z : pw[g].w;
+                    const float2 p2 = make_float2(p, p);
 #pragma unroll
-                    for (int e = 0; e < C::EPC; ++e) acc[g][e] = fmaf(p, v[e], acc[g][e]);
+                    for (int e = 0; e < C::E2; ++e) acc2[g][e] = __ffma2_rn(p2, make_float2(v[2 * e], v[2 * e + 1]), acc2[g][e]);
                 }
             }
         }
@@ -308,7 +324,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
 #pragma unroll
                 for (int g = 0; g < GP; ++g)
 #pragma unroll
-                    for (int e = 0; e < C::EPC; ++e) acc[g][e] += __shfl_xor_sync(FULL_MASK, acc[g][e], o);
+                    for (int e = 0; e < C::E2; ++e) {
+                        acc2[g][e].x += __shfl_xor_sync(FULL_MASK, acc2[g][e].x, o);
+                        acc2[g][e].y += __shfl_xor_sync(FULL_MASK, acc2[g][e].y, o);
+                    }
             ml_s[2 * g_own] = m_own;
             ml_s[2 * g_own + 1] = l_own;
             __syncwarp();
@@ -321,14 +340,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
                             const float inv = 1.f / ml_s[2 * g + 1];
                             float o[C::EPC];
 #pragma unroll
-                            for (int e = 0; e < C::EPC; ++e) o[e] = acc[g][e] * inv;
+                            for (int e = 0; e < C::E2; ++e) {
+                                o[2 * e] = acc2[g][e].x * inv;
+                                o[2 * e + 1] = acc2[g][e].y * inv;
+                            }
                             *reinterpret_cast<uint4*>(static_cast<unsigned char*>(a.out) + qh * C::ROW + chunk * 16) =
                                 Chunk<T>::pack(o);
                         } else {
                             float* po = a.part_o + ((size_t)ci.partial * kMaxGroupPerItem + g) * D + chunk * C::EPC;
 #pragma unroll
-                            for (int e = 0; e < C::EPC; e += 4)
-                                *reinterpret_cast<float4*>(po + e) = make_float4(acc[g][e], acc[g][e + 1], acc[g][e + 2], acc[g][e + 3]);
+                            for (int e = 0; e < C::E2; e += 2)
+                                *reinterpret_cast<float4*>(po + 2 * e) =
+                                    make_float4(acc2[g][e].x, acc2[g][e].y, acc2[g][e + 1].x, acc2[g][e + 1].y);
                             if (chunk == 0) {
                                 float* pm = a.part_ml + ((size_t)ci.partial * kMaxGroupPerItem + g) * 2;
                                 pm[0] = ml_s[2 * g];
@@ -385,9 +408,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
     }
 }
 
-template <typename T, int D, int GP>
+template <typename T, int D, int GP, int NSTAGE>
 cudaError_t launch_decode_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
-    using C = Dec<T, D, GP>;
+    using C = Dec<T, D, GP, NSTAGE>;
     const int smem = kDecodeWarps * C::WARP_SMEM;
     // The shared-memory attribute and the occupancy are per device; cache both per instantiation.
     static int per_sm_cache[64] = {0};
@@ -396,9 +419,9 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < 64) ? per_sm_cache[dev] : 0;
     if (per_sm == 0) {
-        e = cudaFuncSetAttribute(decode_kernel<T, D, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(decode_kernel<T, D, GP, NSTAGE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<T, D, GP>, kDecodeWarps * 32, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<T, D, GP, NSTAGE>, kDecodeWarps * 32, smem);
         if (e != cudaSuccess) return e;
         if (per_sm < 1) per_sm = 1;
         if (dev >= 0 && dev < 64) per_sm_cache[dev] = per_sm;
@@ -407,17 +430,36 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     int grid = num_sms * per_sm;
     if (grid > need) grid = need;
     if (grid < 1) return cudaSuccess;
-    decode_kernel<T, D, GP><<<grid, kDecodeWarps * 32, smem, s>>>(a);
+    decode_kernel<T, D, GP, NSTAGE><<<grid, kDecodeWarps * 32, smem, s>>>(a);
     return cudaGetLastError();
+}
+
+// Ring depth: the default per group size, or PKV_DECODE_STAGES (2..4) as a tuning override.
+inline int stage_override() {
+    static const int v = [] {
+        const char* e = getenv("PKV_DECODE_STAGES");
+        const int x = e ? atoi(e) : 0;
+        return (x >= 2 && x <= 4) ? x : 0;
+    }();
+    return v;
+}
+
+template <typename T, int D, int GP>
+cudaError_t launch_decode_s(const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    switch (stage_override() ? stage_override() : default_stages<GP>()) {
+        case 2: return launch_decode_t<T, D, GP, 2>(a, num_sms, s);
+        case 4: return launch_decode_t<T, D, GP, 4>(a, num_sms, s);
+        default: return launch_decode_t<T, D, GP, 3>(a, num_sms, s);
+    }
 }
 
 template <typename T, int D>
 cudaError_t launch_decode_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     const int g = a.group < kMaxGroupPerItem ? a.group : kMaxGroupPerItem;
-    if (g <= 1) return launch_decode_t<T, D, 1>(a, num_sms, s);
-    if (g <= 2) return launch_decode_t<T, D, 2>(a, num_sms, s);
-    if (g <= 4) return launch_decode_t<T, D, 4>(a, num_sms, s);
-    return launch_decode_t<T, D, 8>(a, num_sms, s);
+    if (g <= 1) return launch_decode_s<T, D, 1>(a, num_sms, s);
+    if (g <= 2) return launch_decode_s<T, D, 2>(a, num_sms, s);
+    if (g <= 4) return launch_decode_s<T, D, 4>(a, num_sms, s);
+    return launch_decode_s<T, D, 8>(a, num_sms, s);
 }
 
 template <typename T>
