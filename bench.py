@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU work of the oracle sample")
     ap.add_argument("--split-blocks", type=int, default=0)
+    ap.add_argument("--part", default="all", choices=["all", "prefill", "decode"],
+                    help="time only the prefill or decode requests of the workload")
     return ap.parse_args()
 
 
@@ -195,7 +197,7 @@ def reference_arm(args, rank, world):
     if rank != 0:
         return
     from paged_kv_cache_446_b200 import workloads as W
-    wl = W.make(args.config, device="cpu")
+    wl = W.make(args.config, device="cpu", part=args.part)
     h = {k: storage(getattr(wl, k)) for k in ("q", "k_pool", "v_pool", "k_new", "v_new")}
     per_step = max(1.0, 150.0 / max(1, args.steps + args.warmup))
     samples = []
@@ -241,7 +243,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     seed = 1000 + int(args.config[1]) + 100 * rank
-    wl = W.make(args.config, device=dev, seed=seed)
+    wl = W.make(args.config, device=dev, seed=seed, part=args.part)
     dt = W.TORCH_DTYPES[wl.dtype]
     opts = {"split_blocks": args.split_blocks} if args.split_blocks else {}
     step = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,

@@ -39,10 +39,9 @@ constexpr int kTile = 2 * kHalf;        // 128 x 128 x 2 bytes
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + kTile;    // 2 stages
 constexpr int OFF_V = OFF_K + 2 * kTile;
-constexpr int OFF_P = OFF_V + 2 * kTile;
-constexpr int OFF_BAR = OFF_P + kTile;
+constexpr int OFF_BAR = OFF_V + 2 * kTile;
 // barrier slots (8 bytes each)
-enum { B_Q = 0, B_KF0 = 1, B_VF0 = 3, B_KE0 = 5, B_SF0 = 7, B_PF = 9, B_OF = 10, B_DRAIN = 11, NUM_BARS = 12 };
+enum { B_Q = 0, B_KF0 = 1, B_VF0 = 3, B_KE0 = 5, B_VE0 = 7, B_SF0 = 9, B_PF = 11, B_OF = 12, B_DRAIN = 13, NUM_BARS = 14 };
 constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;     // tcgen05.alloc result
 constexpr int OFF_ABORT = OFF_TMEM + 4;
 constexpr int OFF_MAXX = OFF_BAR + 128;              // [2 parity][2 half][128 rows] floats
@@ -50,6 +49,9 @@ constexpr int OFF_SUMX = OFF_MAXX + 2 * 2 * 128 * 4; // [2 half][128 rows]
 constexpr int SMEM_USED = OFF_SUMX + 2 * 128 * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;         // slack to align the base to 1024 bytes
 constexpr uint32_t kTmemCols = 512;                  // S0 [0,128), S1 [128,256), O [256,384)
+// A row's exponentials use a reference max that is only raised when the tile max exceeds it by
+// more than this (log2 units); the result is exact (softmax is shift invariant) and p <= 2^8.
+constexpr float kRescaleThreshold = 8.f;
 
 // ---- tcgen05 / TMA primitives ---------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -79,6 +81,27 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc)
         : "memory");
 }
+// Same MMA with the A operand (M x K, K-major, two 16-bit elements per 32-bit column) in TMEM.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc)
+        : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns from registers (thread i writes TMEM lane base + i).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives TMEM lane (base lane + i).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     uint32_t r[32];
@@ -167,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars[B_KF0 + s], 1);
             mbar_init(&bars[B_VF0 + s], 1);
             mbar_init(&bars[B_KE0 + s], 1);
+            mbar_init(&bars[B_VE0 + s], 1);
             mbar_init(&bars[B_SF0 + s], 1);
         }
         mbar_init(&bars[B_PF], kSoftmaxThreads);
@@ -195,12 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(smem + OFF_Q + kHalf, &tm_q, 64, kvh * G, q0 + tok0, &bars[B_Q]);
         }
         int ids = -1, ids_base = -1;
-        int issued_k[2] = {-1, -1};
+        int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
         bool ok = true;
         for (int kt = 0; kt < nkt && ok; ++kt) {
             const int s = kt & 1;
-            if (kt >= 2) ok = wait_or_abort(&bars[B_KE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 100 + kt);
-            if (!ok) break;
             if (ids_base < 0 || kt * 8 >= ids_base + 32) {
                 ids_base = kt * 8;
                 const int b = ids_base + lane;
@@ -216,15 +238,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     y[i] = rows_total;
                 } else y[i] = (id * a.num_kv_heads + kvh) * kBlockSize;
             }
+            // K of tile kt may land once QK^T of tile kt-2 is done; V once PV of tile kt-2 is done.
+            if (kt >= 2) ok = wait_or_abort(&bars[B_KE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 100 + kt);
+            if (!ok) break;
             if (lane == 0) {
                 unsigned char* ks = smem + OFF_K + s * kTile;
-                unsigned char* vs = smem + OFF_V + s * kTile;
                 mbar_arrive_expect_tx(&bars[B_KF0 + s], kTile);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     tma_load_2d(ks + i * 2048, &tm_k, 0, y[i], &bars[B_KF0 + s]);
                     tma_load_2d(ks + kHalf + i * 2048, &tm_k, 64, y[i], &bars[B_KF0 + s]);
                 }
+            }
+            issued_k[s] = kt;
+            if (kt >= 2) ok = wait_or_abort(&bars[B_VE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 150 + kt);
+            if (!ok) break;
+            if (lane == 0) {
+                unsigned char* vs = smem + OFF_V + s * kTile;
                 mbar_arrive_expect_tx(&bars[B_VF0 + s], kTile);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -232,16 +262,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(vs + kHalf + i * 2048, &tm_v, 64, y[i], &bars[B_VF0 + s]);
                 }
             }
-            issued_k[s] = kt;
+            issued_v[s] = kt;
             __syncwarp();
         }
         if (!ok && lane == 0) {
             // Drain: wait (bounded) for the last loads issued into each stage.
-            for (int s = 0; s < 2; ++s)
-                if (issued_k[s] >= 0) {
-                    (void)mbar_wait(&bars[B_KF0 + s], (issued_k[s] >> 1) & 1);
-                    (void)mbar_wait(&bars[B_VF0 + s], (issued_k[s] >> 1) & 1);
-                }
+            for (int s = 0; s < 2; ++s) {
+                if (issued_k[s] >= 0) (void)mbar_wait(&bars[B_KF0 + s], (issued_k[s] >> 1) & 1);
+                if (issued_v[s] >= 0) (void)mbar_wait(&bars[B_VF0 + s], (issued_v[s] >> 1) & 1);
+            }
             (void)mbar_wait(&bars[B_Q], 0);
         }
     } else if (warp == 9 && sane) {
@@ -261,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            smem_desc(ks + half * kHalf + off, 16, 1024), id_qk, k > 0);
                 }
                 tc_commit(&bars[B_SF0 + s]);
+                tc_commit(&bars[B_KE0 + s]);
             };
             if (ok) ok = wait_or_abort(&bars[B_KF0], 0, abort_flag, a.err, 201);
             if (ok) {
@@ -279,17 +309,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
+                // P(kt) sits as packed 16-bit pairs in the first 64 columns of S buffer kt & 1;
+                // each K step of 16 keys is 8 columns.
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int half = k >> 2, off = (k & 3) * 32;
-                    tc_mma(tmem + 256, smem_desc(smem + OFF_P + half * kHalf + off, 16, 1024),
-                           smem_desc(vs + k * 2048, kHalf, 1024), id_pv, k > 0);
-                }
+                for (int k = 0; k < 8; ++k)
+                    tc_mma_ts(tmem + 256, tmem + (kt & 1) * 128 + k * 8, smem_desc(vs + k * 2048, kHalf, 1024), id_pv,
+                              kt > 0 || k > 0);
                 tc_commit(&bars[B_OF]);
-                tc_commit(&bars[B_KE0 + (kt & 1)]);
+                tc_commit(&bars[B_VE0 + (kt & 1)]);
             }
             if (ok) {
-                (void)wait_or_abort(&bars[B_KE0 + ((nkt - 1) & 1)], ((nkt - 1) >> 1) & 1, abort_flag, a.err, 205);
+                (void)wait_or_abort(&bars[B_VE0 + ((nkt - 1) & 1)], ((nkt - 1) >> 1) & 1, abort_flag, a.err, 205);
             } else {
                 tc_commit(&bars[B_DRAIN]);
                 (void)mbar_wait(&bars[B_DRAIN], 0);
@@ -304,14 +334,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool row_valid = j < n;
         const int limit = row_valid ? prior + j + 1 : prior + 1;  // keys visible: [0, limit)
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        float acc[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-        float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
-        bool failed = false;
+        // Keys below this bound are visible to every row of the tile: no masking needed there.
+        const int all_visible = prior + tok0 + 1;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true, failed = false;
         for (int kt = 0; kt < nkt; ++kt) {
             const int sb = kt & 1;
-            bool ok = wait_or_abort(&bars[B_SF0 + sb], (kt >> 1) & 1, abort_flag, a.err, 300);
+            if (ok) ok = wait_or_abort(&bars[B_SF0 + sb], (kt >> 1) & 1, abort_flag, a.err, 300);
             float s[64];
             float mx = -INFINITY;
             if (ok) {
@@ -320,48 +349,78 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(tl + sb * 128 + half * 64 + 32, s + 32);
                 tmem_wait_ld();
                 const int key0 = kt * 128 + half * 64;
+                if (kt * 128 + 128 <= all_visible) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float v = (key0 + i < limit) ? s[i] * a.scale_log2 : -INFINITY;
-                    s[i] = v;
-                    mx = fmaxf(mx, v);
+                    for (int i = 0; i < 64; ++i) {
+                        s[i] *= a.scale_log2;
+                        mx = fmaxf(mx, s[i]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const float v = (key0 + i < limit) ? s[i] * a.scale_log2 : -INFINITY;
+                        s[i] = v;
+                        mx = fmaxf(mx, v);
+                    }
                 }
                 maxx[(sb * 2 + half) * 128 + row] = mx;
             }
-            if (ok && kt >= 1) ok = wait_or_abort(&bars[B_OF], (kt - 1) & 1, abort_flag, a.err, 301);
-            const bool zero_v = (kt == nkt - 1) && (kt + 1) * 128 > ctx;
-            if (ok && zero_v) ok = wait_or_abort(&bars[B_VF0 + sb], (kt >> 1) & 1, abort_flag, a.err, 302);
             if (bar_or(!ok)) {
                 failed = true;
                 break;
             }
-            const float m_new = fmaxf(m, fmaxf(mx, maxx[(sb * 2 + (half ^ 1)) * 128 + row]));
-            const float alpha = fast_exp2(m - m_new);
-            float ps = 0.f;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                s[i] = fast_exp2(s[i] - m_new);
-                ps += s[i];
+            // Lazy reference max: raised only when this tile's max exceeds it by the threshold.
+            const float tile_max = fmaxf(mx, maxx[(sb * 2 + (half ^ 1)) * 128 + row]);
+            float alpha = 1.f;
+            if (tile_max > m + kRescaleThreshold) {
+                alpha = fast_exp2(m - tile_max);  // 0 on the first tile
+                m = tile_max;
             }
-            l = l * alpha + ps;
-            if (kt >= 1) {
-                tc_fence_after();
-                float o[32];
+            float ps = 0.f;
+            uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    tmem_ld32(tl + 256 + half * 64 + c * 32, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(acc[c * 32 + i], alpha_prev, o[i]);
+            for (int i = 0; i < 32; ++i) {
+                const float p0 = fast_exp2(s[2 * i] - m), p1 = fast_exp2(s[2 * i + 1] - m);
+                ps += p0 + p1;
+                if constexpr (std::is_same<T, __half>::value) {
+                    const __half2 h = __floats2half2_rn(p0, p1);
+                    pk[i] = *reinterpret_cast<const uint32_t*>(&h);
+                } else {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    pk[i] = *reinterpret_cast<const uint32_t*>(&h);
                 }
             }
-            alpha_prev = alpha;
-            m = m_new;
-            // P (rounded to T) into the SWIZZLE_128B K-major operand layout.
-            unsigned char* prow = smem + OFF_P + half * kHalf + (row >> 3) * 1024 + (row & 7) * 128;
+            l = l * alpha + ps;
+            // P(kt) replaces S(kt) in its TMEM buffer: keys half*64.. go to columns half*32.. .
+            tmem_st32(tl + sb * 128 + half * 32, pk);
+            tmem_wait_st();
+            // Rescale O in tensor memory when some row of this warp moved its reference (rare after
+            // the first tiles). PV(kt-1) must be complete before O is read.
+            if (kt >= 1 && __any_sync(FULL_MASK, alpha != 1.f)) {
+                ok = wait_or_abort(&bars[B_OF], (kt - 1) & 1, abort_flag, a.err, 301);
+                if (__all_sync(FULL_MASK, ok)) {
+                    tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = Chunk<T>::pack(s + c * 8);
+                    for (int c = 0; c < 2; ++c) {
+                        float o[32];
+                        tmem_ld32(tl + 256 + half * 64 + c * 32, o);
+                        tmem_wait_ld();
+                        uint32_t w[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
+                        tmem_st32(tl + 256 + half * 64 + c * 32, w);
+                    }
+                    tmem_wait_st();
+                } else {
+                    ok = false;
+                }
+            }
+            const bool zero_v = (kt == nkt - 1) && (kt + 1) * 128 > ctx;
+            if (zero_v && ok) ok = wait_or_abort(&bars[B_VF0 + sb], (kt >> 1) & 1, abort_flag, a.err, 302);
+            if (zero_v && bar_or(!ok)) {  // every softmax thread takes this branch or none does
+                failed = true;
+                break;
+            }
             if (zero_v) {
                 unsigned char* vs = smem + OFF_V + sb * kTile;
                 const int r0 = ctx - kt * 128;  // first V row past the context
@@ -370,23 +429,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int r = r0 + (c >> 4), h = (c >> 3) & 1, k = c & 7;
                     *reinterpret_cast<uint4*>(vs + h * kHalf + r * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                 }
+                fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[B_PF]);
         }
         if (!failed) {
-            bool ok = wait_or_abort(&bars[B_OF], (nkt - 1) & 1, abort_flag, a.err, 303);
+            if (ok) ok = wait_or_abort(&bars[B_OF], (nkt - 1) & 1, abort_flag, a.err, 303);
+            float acc[64];
             if (ok) {
                 tc_fence_after();
-                float o[32];
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    tmem_ld32(tl + 256 + half * 64 + c * 32, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(acc[c * 32 + i], alpha_prev, o[i]);
-                }
+                tmem_ld32(tl + 256 + half * 64, acc);
+                tmem_ld32(tl + 256 + half * 64 + 32, acc + 32);
+                tmem_wait_ld();
                 sumx[half * 128 + row] = l;
             }
             if (!bar_or(!ok) && row_valid) {

@@ -108,8 +108,13 @@ def _tables_from_permutation(rng, lens_blocks: list[int], num_blocks: int) -> np
 
 
 def make(config: str, device: str | torch.device = "cpu", small: bool = False, seed: int | None = None,
-         with_tensors: bool = True) -> Workload:
-    """Build configuration `config` ("c1".."c5"); seed defaults to 1000 + the configuration number."""
+         with_tensors: bool = True, part: str = "all") -> Workload:
+    """Build configuration `config` ("c1".."c5"); seed defaults to 1000 + the configuration number.
+
+    part="prefill" / "decode" keeps only the requests with more than one / exactly one row this
+    step (their tables are relabelled onto a pool sized 1.2x their blocks, keeping the seeded
+    placement order), so each half of a mixed batch can be timed on its own.
+    """
     if config not in CONFIGS:
         raise ValueError(f"unknown configuration {config!r}")
     seed = 1000 + int(config[1]) if seed is None else int(seed)
@@ -117,9 +122,34 @@ def make(config: str, device: str | torch.device = "cpu", small: bool = False, s
     builder = {"c1": _c1, "c2": _c2, "c3": _c3, "c4": _c4, "c5": _c5}[config]
     wl = builder(rng, small)
     wl.seed = seed
+    if part != "all":
+        _keep_part(wl, part)
     if with_tensors:
         _draw_tensors(wl, device)
     return wl
+
+
+def _keep_part(wl: Workload, part: str) -> None:
+    if part not in ("prefill", "decode"):
+        raise ValueError(f"unknown part {part!r}")
+    if len(wl.copy_pairs):
+        raise ValueError("parts are defined for workloads without copy-on-write pairs")
+    keys = list(wl.batch.keys())
+    keep = [i for i, r in enumerate(keys) if (wl.batch[r] > 1) == (part == "prefill")]
+    if not keep:
+        raise ValueError(f"{wl.name} has no {part} rows")
+    bt = wl.block_tables[keep]
+    used = np.unique(bt[bt >= 0])
+    order = np.argsort(np.argsort(used))            # rank of each used id: keeps the placement order
+    remap = np.full(wl.num_blocks, -1, dtype=np.int64)
+    remap[used] = order
+    nb = int(math.ceil(1.2 * len(used)))
+    wl.block_tables = np.where(bt >= 0, remap[np.maximum(bt, 0)], -1).astype(np.int32)
+    wl.num_blocks = max(nb, 1)
+    wl.prior_lens = np.asarray(wl.prior_lens)[keep].astype(np.int32)
+    wl.batch = {keys[i]: wl.batch[keys[i]] for i in keep}
+    wl.write_batch = {r: n for r, n in wl.write_batch.items() if r in wl.batch}
+    wl.name = f"{wl.name}-{part}"
 
 
 def _draw_tensors(wl: Workload, device) -> None:
