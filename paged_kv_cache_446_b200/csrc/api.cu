@@ -54,8 +54,8 @@ struct PlanLists {
     int num_partials = 0;
 };
 
-// Query rows per tcgen05 tile: the 128 MMA rows hold (128 / G) consecutive query rows x G heads.
-int tile_tokens(int group) { return 128 / group; }
+// Query rows per tcgen05 CTA: two 128-row MMA tiles, each (128 / G) consecutive query rows x G heads.
+int tile_tokens(int group) { return 2 * (128 / group); }
 
 pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int Hkv, int D, pkv_dtype dt,
                       const pkv_plan_options* opts, int num_sms, PlanLists* L, pkv_plan* plan) {

@@ -7,16 +7,19 @@
 // on tcgen05 with fp32 accumulation in tensor memory; softmax stays in fp32 on the CUDA cores and
 // P is rounded to the input type for the PV product.
 //
-// Tile: 128 MMA rows = (128/G) consecutive query rows x the G query heads of one KV head (GQA
-// packing: each K/V tile is loaded once for all G heads). Key tiles of 128 = 8 blocks.
-// Warp roles (320 threads):
-//   warps 0-7  softmax: two threads per row (64 key columns / 64 output columns each)
-//   warp  8    TMA producer: Q once (3-D tensor map, SWIZZLE_128B), then per key tile 8 blocks x
-//              2 column halves of K and of V (2-D tensor map over the pool rows), double-buffered
-//   warp  9    MMA issuer (one thread): S = Q K^T into one of two TMEM S buffers (so the next
-//              tile's QK^T overlaps this tile's softmax), O_tile = P V into TMEM; completion is
-//              signalled to mbarriers with tcgen05.commit
-// Softmax threads fold each O_tile into fp32 registers with the running-max correction.
+// CTA: two 128-row MMA tiles (A, B), each (128/G) consecutive query rows x the G query heads of one
+// KV head (GQA packing), sharing one stream of 128-key K/V tiles (8 blocks), so every K/V byte
+// fetched from L2 serves 256 rows. Warp roles (320 threads):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: one thread per row
+//   warp  8    TMA producer: both Q tiles once (3-D tensor map, SWIZZLE_128B), then per key tile
+//              8 blocks x 2 column halves of K and of V (2-D tensor map over the pool rows),
+//              double-buffered, K and V released separately
+//   warp  9    MMA issuer (one thread): S_X = Q_X K^T into TMEM; after softmax X has written
+//              P_X (16-bit, over the first 64 columns of S_X), O_X += P_X V with A read from TMEM.
+//              The two tiles ping-pong: one tile's softmax overlaps the other tile's MMAs.
+// O accumulates in TMEM across key tiles. A row's exponentials use a reference maximum that is
+// raised only when a tile's maximum exceeds it by 2^8; O is then rescaled in TMEM (exact: softmax is
+// shift invariant, and p stays <= 2^8).
 // Blocks past the context are fetched at an out-of-range coordinate (TMA fills zeros); V rows past
 // the context inside the last block are zeroed before PV (stale slots may hold anything).
 // Every wait is bounded; on expiry the CTA records PKV_ERR_DEVICE_TIMEOUT, drains its own copies
@@ -33,22 +36,22 @@ namespace pkv {
 namespace {
 
 constexpr int kThreads = 320;
-constexpr int kSoftmaxThreads = 256;
 constexpr int kHalf = 128 * 128;        // 128 rows x 64 elements x 2 bytes
 constexpr int kTile = 2 * kHalf;        // 128 x 128 x 2 bytes
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + kTile;    // 2 stages
-constexpr int OFF_V = OFF_K + 2 * kTile;
+constexpr int OFF_Q = 0;                // Q_A, Q_B
+constexpr int OFF_K = OFF_Q + 2 * kTile;    // 2 stages
+constexpr int OFF_V = OFF_K + 2 * kTile;    // 2 stages
 constexpr int OFF_BAR = OFF_V + 2 * kTile;
-// barrier slots (8 bytes each)
-enum { B_Q = 0, B_KF0 = 1, B_VF0 = 3, B_KE0 = 5, B_VE0 = 7, B_SF0 = 9, B_PF = 11, B_OF = 12, B_DRAIN = 13, NUM_BARS = 14 };
+// barrier slots (8 bytes each); per-tile barriers are indexed by tile 0 (A) / 1 (B)
+enum {
+    B_Q = 0, B_KF0 = 1, B_VF0 = 3, B_KE0 = 5, B_VE0 = 7, B_SF0 = 9, B_PF0 = 11, B_OF0 = 13, B_DRAIN = 15,
+    NUM_BARS = 16
+};
 constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;     // tcgen05.alloc result
 constexpr int OFF_ABORT = OFF_TMEM + 4;
-constexpr int OFF_MAXX = OFF_BAR + 128;              // [2 parity][2 half][128 rows] floats
-constexpr int OFF_SUMX = OFF_MAXX + 2 * 2 * 128 * 4; // [2 half][128 rows]
-constexpr int SMEM_USED = OFF_SUMX + 2 * 128 * 4;
+constexpr int SMEM_USED = OFF_ABORT + 12;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;         // slack to align the base to 1024 bytes
-constexpr uint32_t kTmemCols = 512;                  // S0 [0,128), S1 [128,256), O [256,384)
+constexpr uint32_t kTmemCols = 512;                  // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 // A row's exponentials use a reference max that is only raised when the tile max exceeds it by
 // more than this (log2 units); the result is exact (softmax is shift invariant) and p <= 2^8.
 constexpr float kRescaleThreshold = 8.f;
@@ -100,6 +103,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
         "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
+// 32 lanes x 16 consecutive 32-bit columns from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives TMEM lane (base lane + i).
@@ -131,17 +143,6 @@ __host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_format, uint32_t b_
            ((128u >> 4) << 24);
 }
 
-__device__ __forceinline__ bool bar_or(bool v) {  // named barrier 1 over the 256 softmax threads
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(r)
-        : "r"((uint32_t)v)
-        : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
 // Bounded wait that also gives up when another role has aborted the CTA.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag, DeviceError* err,
                                               int where) {
@@ -158,6 +159,20 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     return true;
 }
 
+// Warp-uniform "all succeeded" for the lanes of one warp.
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(FULL_MASK, v); }
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    if constexpr (std::is_same<T, __half>::value) {
+        const __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
@@ -166,8 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
-    float* maxx = reinterpret_cast<float*>(smem + OFF_MAXX);
-    float* sumx = reinterpret_cast<float*>(smem + OFF_SUMX);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const PrefillTile tile = a.tiles[blockIdx.x];
@@ -177,10 +190,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ctx = a.context_lens[req];
     const int prior = ctx - n;
     const int G = a.group;
-    const int tt = 128 / G;
-    const int last = min(n, tok0 + tt);
-    const int keys = min(ctx, prior + last);
-    const int nkt = (keys + 127) / 128;
+    const int tt = 128 / G;                      // query rows of one MMA tile
+    const bool has_b = tok0 + tt < n;
+    // key tiles each MMA tile needs: keys visible to its last valid row
+    const int nkt_x[2] = {(min(ctx, prior + min(n, tok0 + tt)) + 127) / 128,
+                          has_b ? (min(ctx, prior + min(n, tok0 + 2 * tt)) + 127) / 128 : 0};
+    const int nkt = max(nkt_x[0], nkt_x[1]);
     const int nblk_ctx = (ctx + kBlockSize - 1) / kBlockSize;
     const int rows_total = a.num_blocks * a.num_kv_heads * kBlockSize;
 
@@ -192,9 +207,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars[B_KE0 + s], 1);
             mbar_init(&bars[B_VE0 + s], 1);
             mbar_init(&bars[B_SF0 + s], 1);
+            mbar_init(&bars[B_PF0 + s], 128);
+            mbar_init(&bars[B_OF0 + s], 1);
         }
-        mbar_init(&bars[B_PF], kSoftmaxThreads);
-        mbar_init(&bars[B_OF], 1);
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -214,9 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 8 && sane) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
-            mbar_arrive_expect_tx(&bars[B_Q], kTile);
-            tma_load_3d(smem + OFF_Q, &tm_q, 0, kvh * G, q0 + tok0, &bars[B_Q]);
-            tma_load_3d(smem + OFF_Q + kHalf, &tm_q, 64, kvh * G, q0 + tok0, &bars[B_Q]);
+            mbar_arrive_expect_tx(&bars[B_Q], has_b ? 2 * kTile : kTile);
+            for (int x = 0; x < (has_b ? 2 : 1); ++x) {
+                tma_load_3d(smem + OFF_Q + x * kTile, &tm_q, 0, kvh * G, q0 + tok0 + x * tt, &bars[B_Q]);
+                tma_load_3d(smem + OFF_Q + x * kTile + kHalf, &tm_q, 64, kvh * G, q0 + tok0 + x * tt, &bars[B_Q]);
+            }
         }
         int ids = -1, ids_base = -1;
         int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
@@ -238,8 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     y[i] = rows_total;
                 } else y[i] = (id * a.num_kv_heads + kvh) * kBlockSize;
             }
-            // K of tile kt may land once QK^T of tile kt-2 is done; V once PV of tile kt-2 is done.
-            if (kt >= 2) ok = wait_or_abort(&bars[B_KE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 100 + kt);
+            // K of tile kt may land once both QK^T of tile kt-2 are done; V once both PV of tile kt-2.
+            if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_KE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 100));
             if (!ok) break;
             if (lane == 0) {
                 unsigned char* ks = smem + OFF_K + s * kTile;
@@ -251,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             issued_k[s] = kt;
-            if (kt >= 2) ok = wait_or_abort(&bars[B_VE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 150 + kt);
+            if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_VE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 101));
             if (!ok) break;
             if (lane == 0) {
                 unsigned char* vs = smem + OFF_V + s * kTile;
@@ -276,184 +293,179 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 9 && sane) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
-            const uint32_t fmt = sizeof(T) == 2 && !std::is_same<T, __half>::value ? 1u : 0u;
+            const uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
             const uint32_t id_qk = idesc_f16(fmt, 0);
             const uint32_t id_pv = idesc_f16(fmt, 1);
-            bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, a.err, 200);
-            auto issue_qk = [&](int kt) {
-                const int s = kt & 1;
-                const unsigned char* ks = smem + OFF_K + s * kTile;
+            auto issue_qk = [&](int x, int kt) {
+                const unsigned char* ks = smem + OFF_K + (kt & 1) * kTile;
+                const unsigned char* qs = smem + OFF_Q + x * kTile;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int half = k >> 2, off = (k & 3) * 32;
-                    tc_mma(tmem + s * 128, smem_desc(smem + OFF_Q + half * kHalf + off, 16, 1024),
+                    tc_mma(tmem + x * 128, smem_desc(qs + half * kHalf + off, 16, 1024),
                            smem_desc(ks + half * kHalf + off, 16, 1024), id_qk, k > 0);
                 }
-                tc_commit(&bars[B_SF0 + s]);
-                tc_commit(&bars[B_KE0 + s]);
+                tc_commit(&bars[B_SF0 + x]);
             };
+            auto issue_pv = [&](int x, int kt) {
+                const unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
+                // P_X(kt) sits as packed 16-bit pairs in the first 64 columns of S_X; each K step of
+                // 16 keys is 8 columns.
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    tc_mma_ts(tmem + 256 + x * 128, tmem + x * 128 + k * 8, smem_desc(vs + k * 2048, kHalf, 1024),
+                              id_pv, kt > 0 || k > 0);
+                tc_commit(&bars[B_OF0 + x]);
+            };
+            bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, a.err, 200);
             if (ok) ok = wait_or_abort(&bars[B_KF0], 0, abort_flag, a.err, 201);
             if (ok) {
                 tc_fence_after();
-                issue_qk(0);
+                issue_qk(0, 0);
+                if (has_b) issue_qk(1, 0);
+                tc_commit(&bars[B_KE0]);
             }
             for (int kt = 0; kt < nkt && ok; ++kt) {
-                if (kt + 1 < nkt) {
-                    ok = wait_or_abort(&bars[B_KF0 + ((kt + 1) & 1)], ((kt + 1) >> 1) & 1, abort_flag, a.err, 202);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_qk(kt + 1);
+                const int s = kt & 1;
+                const bool next = kt + 1 < nkt;
+                bool k_ready = false, v_ready = false;
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (kt < nkt_x[x]) {
+                        ok = wait_or_abort(&bars[B_PF0 + x], kt & 1, abort_flag, a.err, 202 + x);
+                        if (ok && !v_ready) ok = v_ready = wait_or_abort(&bars[B_VF0 + s], (kt >> 1) & 1, abort_flag, a.err, 204);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(x, kt);
+                    }
+                    if (kt + 1 < nkt_x[x]) {
+                        if (!k_ready) ok = k_ready = wait_or_abort(&bars[B_KF0 + (s ^ 1)], ((kt + 1) >> 1) & 1, abort_flag, a.err, 206);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_qk(x, kt + 1);
+                    }
                 }
-                ok = wait_or_abort(&bars[B_PF], kt & 1, abort_flag, a.err, 203);
-                if (ok) ok = wait_or_abort(&bars[B_VF0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 204);
                 if (!ok) break;
-                tc_fence_after();
-                const unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
-                // P(kt) sits as packed 16-bit pairs in the first 64 columns of S buffer kt & 1;
-                // each K step of 16 keys is 8 columns.
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    tc_mma_ts(tmem + 256, tmem + (kt & 1) * 128 + k * 8, smem_desc(vs + k * 2048, kHalf, 1024), id_pv,
-                              kt > 0 || k > 0);
-                tc_commit(&bars[B_OF]);
-                tc_commit(&bars[B_VE0 + (kt & 1)]);
+                tc_commit(&bars[B_VE0 + s]);
+                if (next) tc_commit(&bars[B_KE0 + (s ^ 1)]);
             }
             if (ok) {
-                (void)wait_or_abort(&bars[B_VE0 + ((nkt - 1) & 1)], ((nkt - 1) >> 1) & 1, abort_flag, a.err, 205);
+                (void)wait_or_abort(&bars[B_VE0 + ((nkt - 1) & 1)], ((nkt - 1) >> 1) & 1, abort_flag, a.err, 207);
             } else {
                 tc_commit(&bars[B_DRAIN]);
                 (void)mbar_wait(&bars[B_DRAIN], 0);
             }
         }
-    } else if (warp < 8 && sane) {
-        // ------------------------------ softmax ------------------------------
+    } else if (warp < 8 && sane && (warp < 4 || has_b)) {
+        // ------------------------------ softmax (one thread per row) ------------------------------
+        const int x = warp >> 2;                 // tile
         const int row = (warp & 3) * 32 + lane;
-        const int half = warp >> 2;
         const int t_local = row / G, g = row % G;
-        const int j = tok0 + t_local;
+        const int j = tok0 + x * tt + t_local;
         const bool row_valid = j < n;
         const int limit = row_valid ? prior + j + 1 : prior + 1;  // keys visible: [0, limit)
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t ts = tl + x * 128, to = tl + 256 + x * 128;
         // Keys below this bound are visible to every row of the tile: no masking needed there.
-        const int all_visible = prior + tok0 + 1;
+        const int all_visible = prior + tok0 + x * tt + 1;
+        const int my_nkt = nkt_x[x];
         float m = -INFINITY, l = 0.f;
-        bool ok = true, failed = false;
-        for (int kt = 0; kt < nkt; ++kt) {
-            const int sb = kt & 1;
-            if (ok) ok = wait_or_abort(&bars[B_SF0 + sb], (kt >> 1) & 1, abort_flag, a.err, 300);
-            float s[64];
+        bool ok = true;
+        for (int kt = 0; kt < my_nkt && ok; ++kt) {
+            ok = warp_all(wait_or_abort(&bars[B_SF0 + x], kt & 1, abort_flag, a.err, 300));
+            if (!ok) break;
+            tc_fence_after();
+            const bool full = kt * 128 + 128 <= all_visible;
+            // pass 1: row maximum of this tile
             float mx = -INFINITY;
-            if (ok) {
-                tc_fence_after();
-                tmem_ld32(tl + sb * 128 + half * 64, s);
-                tmem_ld32(tl + sb * 128 + half * 64 + 32, s + 32);
+#pragma unroll
+            for (int c = 0; c < 4; c += 2) {
+                float sv[64];
+                tmem_ld32(ts + c * 32, sv);
+                tmem_ld32(ts + c * 32 + 32, sv + 32);
                 tmem_wait_ld();
-                const int key0 = kt * 128 + half * 64;
-                if (kt * 128 + 128 <= all_visible) {
+                const int key0 = kt * 128 + c * 32;
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        s[i] *= a.scale_log2;
-                        mx = fmaxf(mx, s[i]);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        const float v = (key0 + i < limit) ? s[i] * a.scale_log2 : -INFINITY;
-                        s[i] = v;
-                        mx = fmaxf(mx, v);
-                    }
-                }
-                maxx[(sb * 2 + half) * 128 + row] = mx;
+                for (int i = 0; i < 64; ++i) mx = fmaxf(mx, (full || key0 + i < limit) ? sv[i] * a.scale_log2 : -INFINITY);
             }
-            if (bar_or(!ok)) {
-                failed = true;
-                break;
-            }
-            // Lazy reference max: raised only when this tile's max exceeds it by the threshold.
-            const float tile_max = fmaxf(mx, maxx[(sb * 2 + (half ^ 1)) * 128 + row]);
             float alpha = 1.f;
-            if (tile_max > m + kRescaleThreshold) {
-                alpha = fast_exp2(m - tile_max);  // 0 on the first tile
-                m = tile_max;
+            if (mx > m + kRescaleThreshold) {
+                alpha = fast_exp2(m - mx);  // 0 on the first tile
+                m = mx;
             }
+            // pass 2: p = 2^(s*scale - m), rounded to T, written over S as the A operand of PV.
+            // Chunk c's P goes to columns 16c.., which pass 2 has already read.
             float ps = 0.f;
-            uint32_t pk[32];
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float sv[32];
+                tmem_ld32(ts + c * 32, sv);
+                tmem_wait_ld();
+                const int key0 = kt * 128 + c * 32;
+                uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float p0 = fast_exp2(s[2 * i] - m), p1 = fast_exp2(s[2 * i + 1] - m);
-                ps += p0 + p1;
-                if constexpr (std::is_same<T, __half>::value) {
-                    const __half2 h = __floats2half2_rn(p0, p1);
-                    pk[i] = *reinterpret_cast<const uint32_t*>(&h);
-                } else {
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                    pk[i] = *reinterpret_cast<const uint32_t*>(&h);
+                for (int i = 0; i < 16; ++i) {
+                    const float p0 = (full || key0 + 2 * i < limit) ? fast_exp2(fmaf(sv[2 * i], a.scale_log2, -m)) : 0.f;
+                    const float p1 = (full || key0 + 2 * i + 1 < limit) ? fast_exp2(fmaf(sv[2 * i + 1], a.scale_log2, -m)) : 0.f;
+                    ps += p0 + p1;
+                    pk[i] = pack2<T>(p0, p1);
                 }
+                tmem_st16(ts + c * 16, pk);
             }
             l = l * alpha + ps;
-            // P(kt) replaces S(kt) in its TMEM buffer: keys half*64.. go to columns half*32.. .
-            tmem_st32(tl + sb * 128 + half * 32, pk);
-            tmem_wait_st();
-            // Rescale O in tensor memory when some row of this warp moved its reference (rare after
-            // the first tiles). PV(kt-1) must be complete before O is read.
+            // Rescale O in TMEM when a row of this warp raised its reference (rare after the first
+            // tiles). PV(kt-1) must be complete before O is read.
             if (kt >= 1 && __any_sync(FULL_MASK, alpha != 1.f)) {
-                ok = wait_or_abort(&bars[B_OF], (kt - 1) & 1, abort_flag, a.err, 301);
-                if (__all_sync(FULL_MASK, ok)) {
-                    tc_fence_after();
+                ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (kt - 1) & 1, abort_flag, a.err, 301));
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float o[32];
+                    tmem_ld32(to + c * 32, o);
+                    tmem_wait_ld();
+                    uint32_t w[32];
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float o[32];
-                        tmem_ld32(tl + 256 + half * 64 + c * 32, o);
-                        tmem_wait_ld();
-                        uint32_t w[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
-                        tmem_st32(tl + 256 + half * 64 + c * 32, w);
-                    }
-                    tmem_wait_st();
-                } else {
-                    ok = false;
+                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
+                    tmem_st32(to + c * 32, w);
                 }
             }
-            const bool zero_v = (kt == nkt - 1) && (kt + 1) * 128 > ctx;
-            if (zero_v && ok) ok = wait_or_abort(&bars[B_VF0 + sb], (kt >> 1) & 1, abort_flag, a.err, 302);
-            if (zero_v && bar_or(!ok)) {  // every softmax thread takes this branch or none does
-                failed = true;
-                break;
-            }
-            if (zero_v) {
-                unsigned char* vs = smem + OFF_V + sb * kTile;
+            tmem_wait_st();
+            // V rows past the context (only possible in the CTA's final key tile) are zeroed by the
+            // tile whose PV of that key tile is issued first: A when it reaches it, else B.
+            if (kt == nkt - 1 && (kt + 1) * 128 > ctx && x == (nkt_x[0] == nkt ? 0 : 1)) {
+                ok = warp_all(wait_or_abort(&bars[B_VF0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 302));
+                if (!ok) break;
+                unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
                 const int r0 = ctx - kt * 128;  // first V row past the context
                 const int chunks = (128 - r0) * 16;  // 16-byte chunks over both halves
-                for (int c = threadIdx.x; c < chunks; c += kSoftmaxThreads) {
+                for (int c = (warp & 3) * 32 + lane; c < chunks; c += 128) {
                     const int r = r0 + (c >> 4), h = (c >> 3) & 1, k = c & 7;
                     *reinterpret_cast<uint4*>(vs + h * kHalf + r * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
             }
             tc_fence_before();
-            mbar_arrive(&bars[B_PF]);
+            mbar_arrive(&bars[B_PF0 + x]);
         }
-        if (!failed) {
-            if (ok) ok = wait_or_abort(&bars[B_OF], (nkt - 1) & 1, abort_flag, a.err, 303);
-            float acc[64];
-            if (ok) {
-                tc_fence_after();
-                tmem_ld32(tl + 256 + half * 64, acc);
-                tmem_ld32(tl + 256 + half * 64 + 32, acc + 32);
+        if (ok) ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (my_nkt - 1) & 1, abort_flag, a.err, 303));
+        if (ok) {
+            tc_fence_after();
+            const float inv = 1.f / l;
+            unsigned char* dst = static_cast<unsigned char*>(a.out) +
+                                 ((size_t)(q0 + (row_valid ? j : 0)) * a.num_q_heads + (size_t)kvh * G + g) * 256;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float o[32];
+                tmem_ld32(to + c * 32, o);
                 tmem_wait_ld();
-                sumx[half * 128 + row] = l;
-            }
-            if (!bar_or(!ok) && row_valid) {
-                const float inv = 1.f / (l + sumx[(half ^ 1) * 128 + row]);
-                unsigned char* dst = static_cast<unsigned char*>(a.out) +
-                                     ((size_t)(q0 + j) * a.num_q_heads + (size_t)kvh * G + g) * 256 + half * 128;
+                if (row_valid) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float v[8];
+                    for (int q = 0; q < 4; ++q) {
+                        float v[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = acc[c * 8 + e] * inv;
-                    *reinterpret_cast<uint4*>(dst + c * 16) = Chunk<T>::pack(v);
+                        for (int e = 0; e < 8; ++e) v[e] = o[q * 8 + e] * inv;
+                        *reinterpret_cast<uint4*>(dst + c * 64 + q * 16) = Chunk<T>::pack(v);
+                    }
                 }
             }
         }

@@ -128,7 +128,7 @@ def test_planner_covers_every_block_once(pkv, seed, opts):
             for b in range(b0, b1):
                 key = (row, kvh * G + h, b)
                 cover[key] = cover.get(key, 0) + 1
-    tile_rows = 128 // G
+    tile_rows = 2 * (128 // G)      # two 128-row MMA tiles per CTA
     for req, kvh, tok0, _ in tiles:
         nreq = qsl[req + 1] - qsl[req]
         for j in range(tok0, min(nreq, tok0 + tile_rows)):
