@@ -374,18 +374,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = warp_all(wait_or_abort(&bars[B_SF0 + x], kt & 1, abort_flag, a.err, 300));
             if (!ok) break;
             tc_fence_after();
-            const bool full = kt * 128 + 128 <= all_visible;
-            // pass 1: row maximum of this tile
+            const bool full = kt * 128 + 128 <= all_visible;   // no masking anywhere in this key tile
+            // pass 1: row maximum of scale * s over the visible keys
             float mx = -INFINITY;
+            if (full && a.scale_log2 >= 0.f) {
 #pragma unroll
-            for (int c = 0; c < 4; c += 2) {
-                float sv[64];
-                tmem_ld32(ts + c * 32, sv);
-                tmem_ld32(ts + c * 32 + 32, sv + 32);
-                tmem_wait_ld();
-                const int key0 = kt * 128 + c * 32;
+                for (int c = 0; c < 4; c += 2) {
+                    float sv[64];
+                    tmem_ld32(ts + c * 32, sv);
+                    tmem_ld32(ts + c * 32 + 32, sv + 32);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 64; ++i) mx = fmaxf(mx, (full || key0 + i < limit) ? sv[i] * a.scale_log2 : -INFINITY);
+                    for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+                }
+                mx *= a.scale_log2;
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float sv[32];
+                    tmem_ld32(ts + c * 32, sv);
+                    tmem_wait_ld();
+                    const int key0 = kt * 128 + c * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, key0 + i < limit ? sv[i] * a.scale_log2 : -INFINITY);
+                }
             }
             float alpha = 1.f;
             if (mx > m + kRescaleThreshold) {
@@ -394,23 +406,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // pass 2: p = 2^(s*scale - m), rounded to T, written over S as the A operand of PV.
             // Chunk c's P goes to columns 16c.., which pass 2 has already read.
-            float ps = 0.f;
+            float2 ps2 = make_float2(0.f, 0.f);
+            const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 float sv[32];
                 tmem_ld32(ts + c * 32, sv);
                 tmem_wait_ld();
-                const int key0 = kt * 128 + c * 32;
                 uint32_t pk[16];
+                if (full) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = (full || key0 + 2 * i < limit) ? fast_exp2(fmaf(sv[2 * i], a.scale_log2, -m)) : 0.f;
-                    const float p1 = (full || key0 + 2 * i + 1 < limit) ? fast_exp2(fmaf(sv[2 * i + 1], a.scale_log2, -m)) : 0.f;
-                    ps += p0 + p1;
-                    pk[i] = pack2<T>(p0, p1);
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
+                        const float2 p = make_float2(fast_exp2(e.x), fast_exp2(e.y));
+                        ps2 = __fadd2_rn(ps2, p);
+                        pk[i] = pack2<T>(p.x, p.y);
+                    }
+                } else {
+                    const int key0 = kt * 128 + c * 32;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
+                        const float p0 = key0 + 2 * i < limit ? fast_exp2(e.x) : 0.f;
+                        const float p1 = key0 + 2 * i + 1 < limit ? fast_exp2(e.y) : 0.f;
+                        ps2 = __fadd2_rn(ps2, make_float2(p0, p1));
+                        pk[i] = pack2<T>(p0, p1);
+                    }
                 }
                 tmem_st16(ts + c * 16, pk);
             }
+            const float ps = ps2.x + ps2.y;
             l = l * alpha + ps;
             // Rescale O in TMEM when a row of this warp raised its reference (rare after the first
             // tiles). PV(kt-1) must be complete before O is read.
