@@ -275,15 +275,23 @@ def main():
     if world > 1:
         dist.barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    pkv.profile_start(capacity=16 * args.steps + 16)
     ev0.record()
     for _ in range(args.steps):
         run_step()
     ev1.record()
     torch.cuda.synchronize()
-    prof = pkv.profile_stop()
     ms_total = ev0.elapsed_time(ev1)
     clocks = sampler.stop() if sampler else None
+    # Per-kernel times: a second timed region of the same length with CUDA events around every
+    # library launch, on the launch stream (the event pairs serialise back-to-back kernels, so the
+    # step time above is taken without them).
+    if world > 1:
+        dist.barrier()
+    pkv.profile_start(capacity=16 * args.steps + 16)
+    for _ in range(args.steps):
+        run_step()
+    torch.cuda.synchronize()
+    prof = pkv.profile_stop()
     t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

@@ -435,6 +435,7 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         m.part_ml = reinterpret_cast<const float*>(ws + plan->off_part_ml);
         m.num_rows = plan->num_merge_rows;
         m.num_q_heads = plan->num_q_heads;
+        m.heads_per_entry = G < kMaxGroupPerItem ? G : kMaxGroupPerItem;
         ProfileScope prof(PKV_KERNEL_MERGE, s);
         cudaError_t e = launch_merge(plan->dtype, plan->head_dim, m, s);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");

@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
         fence_mbar_init();
     }
     __syncwarp();
+    griddep_wait();
 
     const int W = gridDim.x * kDecodeWarps;
     const int gw = blockIdx.x * kDecodeWarps + warp;
@@ -378,8 +379,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
     constexpr int PER = D / 32;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    const int entry = gw / kMaxGroupPerItem;
-    const int g = gw % kMaxGroupPerItem;
+    const int entry = gw / a.heads_per_entry;
+    const int g = gw % a.heads_per_entry;
+    griddep_wait();
     if (entry >= a.num_rows) return;
     const MergeRow mr = a.rows[entry];
     if (g >= mr.num_heads) return;
@@ -430,8 +432,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     int grid = num_sms * per_sm;
     if (grid > need) grid = need;
     if (grid < 1) return cudaSuccess;
-    decode_kernel<T, D, GP, NSTAGE><<<grid, kDecodeWarps * 32, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(decode_kernel<T, D, GP, NSTAGE>, dim3(grid), dim3(kDecodeWarps * 32), smem, s, a);
 }
 
 // Ring depth: the default per group size, or PKV_DECODE_STAGES (2..4) as a tuning override.
@@ -470,12 +471,11 @@ cudaError_t launch_decode_d(int head_dim, const DecodeArgs& a, int num_sms, cuda
 
 template <typename T>
 cudaError_t launch_merge_d(int head_dim, const MergeArgs& a, cudaStream_t s) {
-    const long long warps = (long long)a.num_rows * kMaxGroupPerItem;
+    const long long warps = (long long)a.num_rows * a.heads_per_entry;
     const int grid = (int)((warps * 32 + 127) / 128);
     if (grid < 1) return cudaSuccess;
-    if (head_dim == 64) merge_kernel<T, 64><<<grid, 128, 0, s>>>(a);
-    else merge_kernel<T, 128><<<grid, 128, 0, s>>>(a);
-    return cudaGetLastError();
+    if (head_dim == 64) return launch_pdl(merge_kernel<T, 64>, dim3(grid), dim3(128), 0, s, a);
+    return launch_pdl(merge_kernel<T, 128>, dim3(grid), dim3(128), 0, s, a);
 }
 
 }  // namespace

@@ -76,6 +76,7 @@ struct MergeArgs {
     const float* part_ml;
     int num_rows;
     int num_q_heads;
+    int heads_per_entry;  // min(Hq / Hkv, 8): warps launched per merge row
 };
 
 struct PrefillArgs {

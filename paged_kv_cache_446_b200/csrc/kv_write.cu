@@ -19,6 +19,7 @@ __global__ void __launch_bounds__(128) slot_mapping_kernel(const int32_t* __rest
                                                            const int32_t* __restrict__ ctx, int num_blocks,
                                                            int64_t* __restrict__ slots, int num_tokens,
                                                            DeviceError* err) {
+    griddep_wait();
     const int r = blockIdx.x;
     const int begin = qsl[r], end = qsl[r + 1];
     const int n = end - begin;
@@ -47,6 +48,7 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const uint4* __restrict__
                                                        const int64_t* __restrict__ slots, long long num_chunks,
                                                        int num_kv_heads, int cpr, long long num_slots,
                                                        DeviceError* err) {
+    griddep_wait();
     const long long per_token = (long long)num_kv_heads * cpr;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < num_chunks;
          i += (long long)gridDim.x * blockDim.x) {
@@ -77,6 +79,7 @@ struct LayerPtrs {
 __global__ void __launch_bounds__(256) copy_blocks_kernel(const LayerPtrs ptrs, const int32_t* __restrict__ pairs,
                                                           int num_blocks, long long chunks_per_block,
                                                           DeviceError* err) {
+    griddep_wait();
     const int p = blockIdx.x;
     const int src = pairs[2 * p], dst = pairs[2 * p + 1];
     if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) {
@@ -96,8 +99,8 @@ cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, const int32_t
                                 int num_reqs, int num_blocks, int64_t* slots, int num_tokens, DeviceError* err,
                                 cudaStream_t s) {
     if (num_reqs <= 0 || num_tokens <= 0) return cudaSuccess;
-    slot_mapping_kernel<<<num_reqs, 128, 0, s>>>(bt, max_blocks, qsl, ctx, num_blocks, slots, num_tokens, err);
-    return cudaGetLastError();
+    return launch_pdl(slot_mapping_kernel, dim3(num_reqs), dim3(128), 0, s, bt, max_blocks, qsl, ctx, num_blocks, slots,
+                      num_tokens, err);
 }
 
 cudaError_t launch_kv_write(const void* k_new, const void* v_new, void* k_pool, void* v_pool, const int64_t* slots,
@@ -108,10 +111,9 @@ cudaError_t launch_kv_write(const void* k_new, const void* v_new, void* k_pool, 
     if (chunks <= 0) return cudaSuccess;
     long long grid = (chunks + 255) / 256;
     if (grid > 148LL * 16) grid = 148LL * 16;
-    kv_write_kernel<<<(unsigned)grid, 256, 0, s>>>(static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-                                                   static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), slots,
-                                                   chunks, num_kv_heads, cpr, (long long)num_blocks * kBlockSize, err);
-    return cudaGetLastError();
+    return launch_pdl(kv_write_kernel, dim3((unsigned)grid), dim3(256), 0, s, static_cast<const uint4*>(k_new),
+                      static_cast<const uint4*>(v_new), static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), slots,
+                      chunks, num_kv_heads, cpr, (long long)num_blocks * kBlockSize, err);
 }
 
 cudaError_t launch_copy_blocks(void* const* k_pools, void* const* v_pools, int num_layers, const int32_t* pairs,
@@ -125,8 +127,8 @@ cudaError_t launch_copy_blocks(void* const* k_pools, void* const* v_pools, int n
             ptrs.k[i] = static_cast<uint4*>(k_pools[l0 + i]);
             ptrs.v[i] = static_cast<uint4*>(v_pools[l0 + i]);
         }
-        copy_blocks_kernel<<<dim3(num_pairs, nl, 2), 256, 0, s>>>(ptrs, pairs, num_blocks, block_bytes / 16, err);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(copy_blocks_kernel, dim3(num_pairs, nl, 2), dim3(256), 0, s, ptrs, pairs, num_blocks,
+                                   block_bytes / 16, err);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

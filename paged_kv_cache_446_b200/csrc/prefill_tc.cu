@@ -182,6 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    griddep_wait();
 
     const PrefillTile tile = a.tiles[blockIdx.x];
     const int req = tile.req, kvh = tile.kv_head, tok0 = tile.tok0;
@@ -552,8 +553,7 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = 1;
     }
-    prefill_tc_kernel<T><<<a.num_tiles, kThreads, SMEM_BYTES, s>>>(a, mq, mk, mv);
-    return cudaGetLastError();
+    return launch_pdl(prefill_tc_kernel<T>, dim3(a.num_tiles), dim3(kThreads), SMEM_BYTES, s, a, mq, mk, mv);
 }
 
 }  // namespace
