@@ -63,6 +63,24 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def rank_seed(config: str, rank: int) -> int:
+    """Each rank runs its own replica of the workload: same shapes, its own seeded data."""
+    return 1000 + int(config[1]) + 100 * rank
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The slowest rank's time: every rank contributes its own device time, all receive the max."""
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: all ranks' bytes divided by the slowest rank's step time."""
+    return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 def workload_desc(wl):
     ctx = np.asarray(wl.prior_lens, np.int64) + np.asarray(list(wl.batch.values()), np.int64)
     return ctx
@@ -242,8 +260,7 @@ def main():
     dev = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    seed = 1000 + int(args.config[1]) + 100 * rank
-    wl = W.make(args.config, device=dev, seed=seed, part=args.part)
+    wl = W.make(args.config, device=dev, seed=rank_seed(args.config, rank), part=args.part)
     dt = W.TORCH_DTYPES[wl.dtype]
     opts = {"split_blocks": args.split_blocks} if args.split_blocks else {}
     step = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,
@@ -292,10 +309,7 @@ def main():
         run_step()
     torch.cuda.synchronize()
     prof = pkv.profile_stop()
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_per_step = float(t.item()) / args.steps
+    ms_per_step = max_over_ranks(ms_total, dist, dev) / args.steps
     code, detail = pkv.device_error()
     assert code == 0, f"device error {code} at {detail}"
 
@@ -331,14 +345,11 @@ def main():
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item()) / args.steps
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.steps
         h2d = (hq.numel() * hq.element_size() + hkn.numel() * hkn.element_size() + hvn.numel() * hvn.element_size()
                + hbt.numel() * 4 + int(step.plan.plan.meta_bytes) + 2 * 4 * (len(wl.batch) + 1))
         d2h = hout.numel() * hout.element_size()
-        e2e = {"value": world * kv_bytes(wl) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+        e2e = {"value": whole_job_gbs(kv_bytes(wl), world, e2e_ms), "unit": "GB/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     if world > 1:
@@ -347,7 +358,7 @@ def main():
     if rank != 0:
         return
     peak, peak_kind = peaks()
-    value = world * kv_bytes(wl) / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gbs(kv_bytes(wl), world, ms_per_step)
     dec_ms, dec_n = prof["decode"]
     roof = None
     if dec_n:
