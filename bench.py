@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--split-blocks", type=int, default=0)
     ap.add_argument("--part", default="all", choices=["all", "prefill", "decode"],
                     help="time only the prefill or decode requests of the workload")
+    ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling subsets)")
     return ap.parse_args()
 
 
@@ -215,7 +216,7 @@ def reference_arm(args, rank, world):
     if rank != 0:
         return
     from paged_kv_cache_446_b200 import workloads as W
-    wl = W.make(args.config, device="cpu", part=args.part)
+    wl = W.make(args.config, device="cpu", part=args.part, max_requests=args.requests)
     h = {k: storage(getattr(wl, k)) for k in ("q", "k_pool", "v_pool", "k_new", "v_new")}
     per_step = max(1.0, 150.0 / max(1, args.steps + args.warmup))
     samples = []
@@ -260,7 +261,8 @@ def main():
     dev = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    wl = W.make(args.config, device=dev, seed=rank_seed(args.config, rank), part=args.part)
+    wl = W.make(args.config, device=dev, seed=rank_seed(args.config, rank), part=args.part,
+                max_requests=args.requests)
     dt = W.TORCH_DTYPES[wl.dtype]
     opts = {"split_blocks": args.split_blocks} if args.split_blocks else {}
     step = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,
@@ -322,15 +324,13 @@ def main():
         hbt = torch.from_numpy(wl.block_tables).pin_memory()
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         dq, dkn, dvn = torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new)
-        ws = step.plan.workspace
 
         def e2e_step():
             dq.copy_(hq, non_blocking=True)
             dkn.copy_(hkn, non_blocking=True)
             dvn.copy_(hvn, non_blocking=True)
             step.block_tables.copy_(hbt, non_blocking=True)
-            step.plan = pkv.AttentionPlan(wl.batch, wl.prior_lens, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, dt,
-                                          dev, workspace=ws, **opts)
+            step.plan.replan(wl.batch, wl.prior_lens)
             step.run(dq, wl.k_pool, wl.v_pool, wl.scale, dkn, dvn, out=out)
             hout.copy_(out, non_blocking=True)
 

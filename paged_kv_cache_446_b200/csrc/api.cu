@@ -46,13 +46,31 @@ int current_sm_count() {
     return n;
 }
 
-// Work lists of one batch, before they are written into the metadata image.
+// Work lists of one batch, before they are written into the metadata image. One instance per host
+// thread is reused across calls so the vectors keep their capacity (fresh large allocations would
+// be served from newly mapped pages and fault on every call).
 struct PlanLists {
     std::vector<DecodeItem> items;
     std::vector<PrefillTile> tiles;
     std::vector<MergeRow> merges;
+    std::vector<size_t> start;
+    std::vector<int> req_keys;
     int num_partials = 0;
+    void reset() {
+        items.clear();
+        tiles.clear();
+        merges.clear();
+        start.clear();
+        req_keys.clear();
+        num_partials = 0;
+    }
 };
+
+PlanLists& thread_lists() {
+    static thread_local PlanLists lists;
+    lists.reset();
+    return lists;
+}
 
 // Query rows per tcgen05 CTA: two 128-row MMA tiles, each (128 / G) consecutive query rows x G heads.
 int tile_tokens(int group) { return 2 * (128 / group); }
@@ -79,7 +97,9 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     const int eb = elem_bytes(dt);
 
     struct CoreRow { int row, req, limit; };
-    std::vector<CoreRow> core_rows;
+    static thread_local std::vector<CoreRow> core_rows;
+    core_rows.clear();
+    core_rows.reserve(R > 0 ? (size_t)qsl[R] : 0);
     int64_t kv_bytes = 0, flops = 0;
     int decode_rows = 0, prefill_rows = 0, max_blocks = 0;
     for (int r = 0; r < R; ++r) {
@@ -115,6 +135,40 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
         const int64_t workers = (int64_t)std::max(num_sms, 1) * 8;
         chunk = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(total_blocks, workers * 4), 8), 1 << 20);
     }
+    // Items are placed directly at their position in a stable order by length, longest first:
+    // this balances the static round-robin over the persistent warps. Pass 1 counts the items of
+    // each length from the row lengths alone; pass 2 writes every item to its slot.
+    size_t n_items = 0, n_merge = 0;
+    int max_len = 0;
+    for (const CoreRow& c : core_rows) {
+        const int nb = (int)ceil_div(c.limit, kBlockSize);
+        const int pieces = (int)ceil_div(nb, chunk);
+        n_items += (size_t)pieces * Hkv * groups;
+        if (pieces > 1) n_merge += (size_t)Hkv * groups;
+        max_len = std::max(max_len, std::min(nb, chunk));
+    }
+    std::vector<size_t>& start = L->start;
+    start.assign((size_t)max_len + 2, 0);
+    for (const CoreRow& c : core_rows) {
+        const int nb = (int)ceil_div(c.limit, kBlockSize);
+        const int pieces = (int)ceil_div(nb, chunk);
+        const size_t per = (size_t)Hkv * groups;
+        start[std::min(nb, chunk)] += per * (pieces > 1 ? pieces - 1 : 1);
+        if (pieces > 1) start[nb - (pieces - 1) * chunk] += per;
+    }
+    size_t acc = 0;
+    for (int len = max_len; len >= 1; --len) {
+        const size_t cnt = start[len];
+        start[len] = acc;
+        acc += cnt;
+    }
+    L->items.resize(n_items);
+    L->merges.resize(n_merge);
+    DecodeItem* items = L->items.data();
+    MergeRow* merges = L->merges.data();
+    size_t* pos = start.data();
+    size_t mi = 0;
+    int partials = 0;
     for (const CoreRow& c : core_rows) {
         const int nb = (int)ceil_div(c.limit, kBlockSize);
         const int pieces = (int)ceil_div(nb, chunk);
@@ -122,23 +176,21 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
             for (int g0 = 0; g0 < G; g0 += kMaxGroupPerItem) {
                 int first = -1;
                 if (pieces > 1) {
-                    first = L->num_partials;
-                    L->num_partials += pieces;
-                    L->merges.push_back(MergeRow{c.row, h * G + g0, std::min(kMaxGroupPerItem, G - g0), first, pieces, {0, 0, 0}});
+                    first = partials;
+                    partials += pieces;
+                    merges[mi++] = MergeRow{c.row, h * G + g0, std::min(kMaxGroupPerItem, G - g0), first, pieces, {0, 0, 0}};
                 }
                 for (int p = 0; p < pieces; ++p) {
                     const int b0 = p * chunk, b1 = std::min(nb, b0 + chunk);
-                    L->items.push_back(DecodeItem{c.row, c.req, h, g0, b0, b1, c.limit, pieces > 1 ? first + p : -1});
+                    items[pos[b1 - b0]++] = DecodeItem{c.row, c.req, h, g0, b0, b1, c.limit, pieces > 1 ? first + p : -1};
                 }
             }
     }
-    // Longest work first: balances the static round-robin over persistent warps / CTAs.
-    std::stable_sort(L->items.begin(), L->items.end(), [](const DecodeItem& a, const DecodeItem& b) {
-        return (a.blk_end - a.blk_begin) > (b.blk_end - b.blk_begin);
-    });
+    L->num_partials = partials;
     // Tiles: longest requests first; a (request, KV head)'s tiles stay adjacent (longest first) so
     // the CTAs running at the same time share that head's K/V through L2.
-    std::vector<int> req_keys(R > 0 ? R : 1, 0);
+    std::vector<int>& req_keys = L->req_keys;
+    req_keys.assign(R > 0 ? R : 1, 0);
     for (const PrefillTile& t : L->tiles) req_keys[t.req] = std::max(req_keys[t.req], t.key_tiles);
     std::stable_sort(L->tiles.begin(), L->tiles.end(), [&](const PrefillTile& a, const PrefillTile& b) {
         if (req_keys[a.req] != req_keys[b.req]) return req_keys[a.req] > req_keys[b.req];
@@ -325,7 +377,7 @@ pkv_status pkv_attention_workspace_size(const int32_t* h_query_start_loc, const 
                                         int num_reqs, int num_q_heads, int num_kv_heads, int head_dim,
                                         pkv_dtype dtype, const pkv_plan_options* opts, size_t* bytes) {
     if (!bytes) return fail(PKV_ERR_INVALID_ARG, "null bytes");
-    PlanLists L;
+    PlanLists& L = thread_lists();
     pkv_plan plan;
     const int sms = (opts && opts->num_sms > 0) ? opts->num_sms : current_sm_count();
     pkv_status s = plan_lists(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim,
@@ -339,7 +391,7 @@ pkv_status pkv_attention_plan_host(const int32_t* h_query_start_loc, const int32
                                    int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
                                    const pkv_plan_options* opts, void* h_meta, size_t meta_capacity,
                                    pkv_plan* plan) {
-    PlanLists L;
+    PlanLists& L = thread_lists();
     const int sms = (opts && opts->num_sms > 0) ? opts->num_sms : 148;
     pkv_status s = plan_lists(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim,
                               dtype, opts, sms, &L, plan);
@@ -356,7 +408,7 @@ pkv_status pkv_attention_plan(const int32_t* h_query_start_loc, const int32_t* h
                               int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
                               const pkv_plan_options* opts, void* d_workspace, size_t ws_bytes, pkv_plan* plan,
                               pkv_stream_t stream) {
-    PlanLists L;
+    PlanLists& L = thread_lists();
     const int sms = (opts && opts->num_sms > 0) ? opts->num_sms : current_sm_count();
     pkv_status s = plan_lists(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim,
                               dtype, opts, sms, &L, plan);

@@ -185,30 +185,47 @@ def plan_host(query_start_loc: np.ndarray, context_lens: np.ndarray, num_q_heads
 
 
 class AttentionPlan:
-    """A planned batch: host plan, device workspace and device copies of the batch description."""
+    """A planned batch: host plan, device workspace and device copies of the batch description.
+
+    The workspace is reused across plans; it grows (one more planner run) only when a batch needs
+    more than it holds.
+    """
 
     def __init__(self, batch: dict, prior_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
                  dtype: torch.dtype, device, workspace: torch.Tensor | None = None, stream=None, **opts):
-        qsl, ctx = flatten_batch(batch, prior_lens)
-        self.h_query_start_loc, self.h_context_lens = qsl, ctx
         self.num_q_heads, self.num_kv_heads, self.head_dim, self.dtype = num_q_heads, num_kv_heads, head_dim, dtype
-        self.num_q_tokens = int(qsl[-1])
-        o = _opts(**opts)
-        size = _SZ(0)
-        _check(_ws_size(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], num_q_heads, num_kv_heads, head_dim,
-                        _dtype_code(torch.empty(0, dtype=dtype)), ctypes.byref(o), ctypes.byref(size)),
-               "pkv_attention_workspace_size")
-        if workspace is None or workspace.numel() < size.value:
-            workspace = torch.empty(max(size.value, 256), dtype=torch.uint8, device=device)
+        self.device = torch.device(device)
+        self.opts = _opts(**opts)
         self.workspace = workspace
         self.plan = Plan()
-        _check(_plan(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], num_q_heads, num_kv_heads, head_dim,
-                     _dtype_code(torch.empty(0, dtype=dtype)), ctypes.byref(o), _ptr(workspace), workspace.numel(),
-                     ctypes.byref(self.plan), _stream(stream)), "pkv_attention_plan")
-        # Pinned staging keeps the uploads asynchronous; torch's host allocator keeps each staging
-        # buffer alive until its copy has run.
-        self.query_start_loc = torch.from_numpy(qsl).pin_memory().to(device, non_blocking=True)
-        self.context_lens = torch.from_numpy(ctx).pin_memory().to(device, non_blocking=True)
+        self.replan(batch, prior_lens, stream=stream)
+
+    def replan(self, batch: dict, prior_lens, stream=None) -> "AttentionPlan":
+        qsl, ctx = flatten_batch(batch, prior_lens)
+        self.h_query_start_loc, self.h_context_lens = qsl, ctx
+        self.num_q_tokens = int(qsl[-1])
+        code = _dtype_code(torch.empty(0, dtype=self.dtype))
+        st = _stream(stream)
+        for _ in range(2):
+            ws = self.workspace
+            status = _plan(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], self.num_q_heads, self.num_kv_heads,
+                           self.head_dim, code, ctypes.byref(self.opts), _ptr(ws) if ws is not None else None,
+                           ws.numel() if ws is not None else 0, ctypes.byref(self.plan), st)
+            if status == PKV_OK:
+                break
+            if status in (1, 4) and (ws is None or ws.numel() < self.plan.ws_bytes) and self.plan.ws_bytes > 0:
+                self.workspace = torch.empty(max(int(self.plan.ws_bytes), 256), dtype=torch.uint8, device=self.device)
+                continue
+            _check(status, "pkv_attention_plan")
+        _check(status, "pkv_attention_plan")
+        # One pinned staging buffer for both arrays keeps the upload asynchronous; torch's host
+        # allocator keeps it alive until the copy has run.
+        R = ctx.shape[0]
+        staged = torch.from_numpy(np.concatenate([qsl, ctx])).pin_memory()
+        dev = staged.to(self.device, non_blocking=True)
+        self.query_start_loc = dev[:R + 1]
+        self.context_lens = dev[R + 1:]
+        return self
 
 
 def paged_attention(plan: AttentionPlan, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,

@@ -108,12 +108,13 @@ def _tables_from_permutation(rng, lens_blocks: list[int], num_blocks: int) -> np
 
 
 def make(config: str, device: str | torch.device = "cpu", small: bool = False, seed: int | None = None,
-         with_tensors: bool = True, part: str = "all") -> Workload:
+         with_tensors: bool = True, part: str = "all", max_requests: int = 0) -> Workload:
     """Build configuration `config` ("c1".."c5"); seed defaults to 1000 + the configuration number.
 
     part="prefill" / "decode" keeps only the requests with more than one / exactly one row this
     step (their tables are relabelled onto a pool sized 1.2x their blocks, keeping the seeded
-    placement order), so each half of a mixed batch can be timed on its own.
+    placement order), so each half of a mixed batch can be timed on its own. max_requests > 0 then
+    keeps only the first that many requests (a smaller case of the same structure, for profiling).
     """
     if config not in CONFIGS:
         raise ValueError(f"unknown configuration {config!r}")
@@ -122,20 +123,22 @@ def make(config: str, device: str | torch.device = "cpu", small: bool = False, s
     builder = {"c1": _c1, "c2": _c2, "c3": _c3, "c4": _c4, "c5": _c5}[config]
     wl = builder(rng, small)
     wl.seed = seed
-    if part != "all":
-        _keep_part(wl, part)
+    if part != "all" or max_requests > 0:
+        _keep_part(wl, part, max_requests)
     if with_tensors:
         _draw_tensors(wl, device)
     return wl
 
 
-def _keep_part(wl: Workload, part: str) -> None:
-    if part not in ("prefill", "decode"):
+def _keep_part(wl: Workload, part: str, max_requests: int = 0) -> None:
+    if part not in ("all", "prefill", "decode"):
         raise ValueError(f"unknown part {part!r}")
     if len(wl.copy_pairs):
         raise ValueError("parts are defined for workloads without copy-on-write pairs")
     keys = list(wl.batch.keys())
-    keep = [i for i, r in enumerate(keys) if (wl.batch[r] > 1) == (part == "prefill")]
+    keep = [i for i, r in enumerate(keys) if part == "all" or (wl.batch[r] > 1) == (part == "prefill")]
+    if max_requests > 0:
+        keep = keep[:max_requests]
     if not keep:
         raise ValueError(f"{wl.name} has no {part} rows")
     bt = wl.block_tables[keep]
@@ -149,7 +152,7 @@ def _keep_part(wl: Workload, part: str) -> None:
     wl.prior_lens = np.asarray(wl.prior_lens)[keep].astype(np.int32)
     wl.batch = {keys[i]: wl.batch[keys[i]] for i in keep}
     wl.write_batch = {r: n for r, n in wl.write_batch.items() if r in wl.batch}
-    wl.name = f"{wl.name}-{part}"
+    wl.name = wl.name + ("" if part == "all" else f"-{part}") + (f"-first{max_requests}" if max_requests > 0 else "")
 
 
 def _draw_tensors(wl: Workload, device) -> None:
