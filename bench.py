@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--part", default="all", choices=["all", "prefill", "decode"],
                     help="time only the prefill or decode requests of the workload")
     ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling subsets)")
+    ap.add_argument("--heads-per-item", type=int, default=0, help="query heads per CUDA-core work item")
     return ap.parse_args()
 
 
@@ -265,6 +266,8 @@ def main():
                 max_requests=args.requests)
     dt = W.TORCH_DTYPES[wl.dtype]
     opts = {"split_blocks": args.split_blocks} if args.split_blocks else {}
+    if args.heads_per_item:
+        opts["heads_per_item"] = args.heads_per_item
     step = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,
                               wl.num_kv_heads, wl.head_dim, dt, dev, write_batch=wl.write_batch or None,
                               copy_pairs=wl.copy_pairs, **opts)

@@ -113,6 +113,9 @@ typedef struct pkv_plan_options {
     int32_t cuda_core_only;    /* 1: multi-row requests also go to the CUDA-core path (no tcgen05) */
     int32_t num_sms;           /* SM count the chunking targets; 0 = query the current device
                                   (pkv_attention_plan) or 148 (pkv_attention_plan_host) */
+    int32_t heads_per_item;    /* query heads of one group served by one CUDA-core work item
+                                  (1..8); 0 = min(Hq/Hkv, 8). Larger groups are split into items
+                                  that read the same K/V blocks */
 } pkv_plan_options;
 
 /*
@@ -130,6 +133,8 @@ typedef struct pkv_plan {
     int32_t num_partials;        /* chunk partial results in the workspace */
     int32_t split_blocks;        /* chunk length in blocks used for this batch */
     int32_t max_blocks;          /* longest context in blocks */
+    int32_t heads_per_item;      /* query heads per CUDA-core work item */
+    int32_t reserved;
     int64_t off_items, off_tiles, off_merge, off_part_o, off_part_ml; /* byte offsets into workspace */
     int64_t meta_bytes;          /* bytes uploaded by pkv_attention_plan (work lists) */
     int64_t ws_bytes;            /* total workspace bytes this plan needs */

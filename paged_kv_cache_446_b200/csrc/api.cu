@@ -124,8 +124,10 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
             for (int j = 0; j < n; ++j) core_rows.push_back(CoreRow{qsl[r] + j, r, P + j + 1});
         }
     }
+    const int hpi = (o.heads_per_item > 0 && o.heads_per_item <= kMaxGroupPerItem) ? o.heads_per_item
+                                                                                  : std::min(G, kMaxGroupPerItem);
     // Chunk length: enough items for ~4 per resident warp, but never below 8 blocks.
-    const int groups = (int)ceil_div(G, kMaxGroupPerItem);
+    const int groups = (int)ceil_div(G, hpi);
     int64_t total_blocks = 0;
     for (const CoreRow& c : core_rows) total_blocks += ceil_div(c.limit, kBlockSize) * Hkv * groups;
     int chunk;
@@ -173,12 +175,12 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
         const int nb = (int)ceil_div(c.limit, kBlockSize);
         const int pieces = (int)ceil_div(nb, chunk);
         for (int h = 0; h < Hkv; ++h)
-            for (int g0 = 0; g0 < G; g0 += kMaxGroupPerItem) {
+            for (int g0 = 0; g0 < G; g0 += hpi) {
                 int first = -1;
                 if (pieces > 1) {
                     first = partials;
                     partials += pieces;
-                    merges[mi++] = MergeRow{c.row, h * G + g0, std::min(kMaxGroupPerItem, G - g0), first, pieces, {0, 0, 0}};
+                    merges[mi++] = MergeRow{c.row, h * G + g0, std::min(hpi, G - g0), first, pieces, {0, 0, 0}};
                 }
                 for (int p = 0; p < pieces; ++p) {
                     const int b0 = p * chunk, b1 = std::min(nb, b0 + chunk);
@@ -215,6 +217,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->num_partials = L->num_partials;
     plan->split_blocks = chunk;
     plan->max_blocks = max_blocks;
+    plan->heads_per_item = hpi;
     int64_t off = 256;  // first 256 bytes reserved
     plan->off_items = off;
     off = align256(off + (int64_t)L->items.size() * sizeof(DecodeItem));
@@ -474,7 +477,7 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         a.part_ml = reinterpret_cast<float*>(ws + plan->off_part_ml);
         a.err = err; a.num_items = plan->num_items; a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks; a.num_q_heads = plan->num_q_heads; a.num_kv_heads = plan->num_kv_heads;
-        a.group = G; a.scale_log2 = scale_log2;
+        a.group = G; a.heads_per_item = plan->heads_per_item; a.scale_log2 = scale_log2;
         ProfileScope prof(PKV_KERNEL_DECODE, s);
         cudaError_t e = launch_decode(plan->dtype, plan->head_dim, a, sms, s);
         if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -487,7 +490,7 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         m.part_ml = reinterpret_cast<const float*>(ws + plan->off_part_ml);
         m.num_rows = plan->num_merge_rows;
         m.num_q_heads = plan->num_q_heads;
-        m.heads_per_entry = G < kMaxGroupPerItem ? G : kMaxGroupPerItem;
+        m.heads_per_entry = plan->heads_per_item;
         ProfileScope prof(PKV_KERNEL_MERGE, s);
         cudaError_t e = launch_merge(plan->dtype, plan->head_dim, m, s);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");

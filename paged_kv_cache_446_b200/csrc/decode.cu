@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
             }
             unsigned char* st = wbase + stage * C::STAGE;
             const bool first = (p_blk == pi.blk_begin);
-            const int nh = min(GP, a.group - pi.head0);
+            const int nh = min(a.heads_per_item, a.group - pi.head0);
             const uint32_t qbytes = first ? (uint32_t)(nh * C::ROW) : 0u;
             mbar_arrive_expect_tx(&bars[stage], 2u * C::BLK + qbytes);
             const size_t off = ((size_t)id * a.num_kv_heads + pi.kv_head) * head_stride;
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
         const unsigned char* st = wbase + stage * C::STAGE;
         const unsigned char* Ks = st;
         const unsigned char* Vs = st + C::BLK;
-        const int nh = min(GP, a.group - ci.head0);
+        const int nh = min(a.heads_per_item, a.group - ci.head0);
 
         if (c_blk == ci.blk_begin) {
 #pragma unroll
@@ -456,7 +456,7 @@ cudaError_t launch_decode_s(const DecodeArgs& a, int num_sms, cudaStream_t s) {
 
 template <typename T, int D>
 cudaError_t launch_decode_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
-    const int g = a.group < kMaxGroupPerItem ? a.group : kMaxGroupPerItem;
+    const int g = a.heads_per_item;
     if (g <= 1) return launch_decode_s<T, D, 1>(a, num_sms, s);
     if (g <= 2) return launch_decode_s<T, D, 2>(a, num_sms, s);
     if (g <= 4) return launch_decode_s<T, D, 4>(a, num_sms, s);

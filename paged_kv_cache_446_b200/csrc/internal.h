@@ -66,6 +66,7 @@ struct DecodeArgs {
     int num_q_heads;
     int num_kv_heads;
     int group;           // Hq / Hkv
+    int heads_per_item;  // query heads one item serves (<= 8)
     float scale_log2;    // scale * log2(e)
 };
 
@@ -76,7 +77,7 @@ struct MergeArgs {
     const float* part_ml;
     int num_rows;
     int num_q_heads;
-    int heads_per_entry;  // min(Hq / Hkv, 8): warps launched per merge row
+    int heads_per_entry;  // heads per merge row (the plan's heads per item): warps launched per row
 };
 
 struct PrefillArgs {

@@ -103,7 +103,7 @@ def parse_meta(plan, meta):
 
 @pytest.mark.parametrize("seed", range(6))
 @pytest.mark.parametrize("opts", [{}, {"split_blocks": 1}, {"split_blocks": 3}, {"no_split": True},
-                                  {"cuda_core_only": True}])
+                                  {"cuda_core_only": True}, {"heads_per_item": 4}, {"heads_per_item": 3}])
 def test_planner_covers_every_block_once(pkv, seed, opts):
     """Every (row, query head, visible KV block) is covered by exactly one work item or tile."""
     rng = np.random.default_rng(seed)
@@ -124,7 +124,7 @@ def test_planner_covers_every_block_once(pkv, seed, opts):
         j = row - qsl[req]
         assert limit == ctx[req] - (qsl[req + 1] - qsl[req]) + j + 1
         assert 0 <= b0 < b1 <= -(-limit // 16)
-        for h in range(head0, min(G, head0 + 8)):
+        for h in range(head0, min(G, head0 + plan.heads_per_item)):
             for b in range(b0, b1):
                 key = (row, kvh * G + h, b)
                 cover[key] = cover.get(key, 0) + 1
@@ -155,7 +155,7 @@ def test_planner_covers_every_block_once(pkv, seed, opts):
     assert len(owners) == plan.num_partials
     for row, req, kvh, head0, b0, b1, limit, part in items:
         if part >= 0:
-            assert owners[part] == (row, kvh * G + head0, min(8, G - head0))
+            assert owners[part] == (row, kvh * G + head0, min(plan.heads_per_item, G - head0))
     if opts.get("no_split"):
         assert plan.num_merge_rows == 0
 

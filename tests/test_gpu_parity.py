@@ -237,3 +237,11 @@ def test_prefill_tiles_match_cuda_core_path(dev, dtype, Hq, Hkv, D, specs):
     torch.cuda.synchronize()
     err = (a.double() - b.double()).abs().max().item()
     assert err <= TOL[wl.dtype], err
+
+
+@pytest.mark.parametrize("hpi", [1, 3, 4, 8])
+def test_heads_per_item(dev, hpi):
+    """A query group served by several work items (each re-reading the same K/V blocks) gives the
+    same result."""
+    wl = W.make("c5", device=dev, small=True)
+    run_and_compare(wl, dev, heads_per_item=hpi, cuda_core_only=True)
