@@ -248,6 +248,14 @@ pkv_status pkv_paged_attention_static_ws(const int32_t* h_query_start_loc, const
                                          pkv_stream_t stream);
 
 /*
+ * pkv_selftest_exp2 -- test aid with no counterpart on the pages: y[i] = 2^x[i] computed by the
+ * FMA-pipe exponential the prefill softmax uses for part of its elements (range reduction to
+ * [-1/2, 1/2] and a fitted degree-4 polynomial, relative error below 3e-6 for -126 <= x <= 127).
+ * x, y: device float arrays of n elements. Errors: INVALID_ARG, CUDA.
+ */
+pkv_status pkv_selftest_exp2(const float* x, float* y, int n, pkv_stream_t stream);
+
+/*
  * Kernel timing (no counterpart on the pages; a measurement aid). Between pkv_profile_start and
  * pkv_profile_stop, every kernel the library launches on the calling host thread is bracketed by
  * a pair of CUDA events recorded on the launch stream. pkv_profile_stop synchronises those events,

@@ -98,6 +98,30 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, for two values at once (offloads the MUFU unit, which the prefill softmax
+// saturates). Range reduction: x = n + f with n = round(x) and f in [-1/2, 1/2], n obtained by
+// adding 1.5 * 2^23 (the sum's low mantissa bits then hold n). 2^f comes from a degree-4 polynomial
+// fitted here to 2^f on [-1/2, 1/2] for minimum relative error (weighted least squares on
+// Chebyshev nodes with iterative reweighting); evaluated in fp32 its relative error is below
+// 3e-6. 2^n is added into the exponent field. Inputs are clamped to -126 (results below 2^-126
+// flush towards 0); inputs must be at most 127.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kC0 = 0.99999928474426270f, kC1 = 0.69312179088592530f, kC2 = 0.24024748802185059f,
+                    kC3 = 0.055917855352163315f, kC4 = 0.009569923393428326f;
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+    const float2 r = __fadd2_rn(t, make_float2(-kRound, -kRound));
+    const float2 f = __fadd2_rn(x, make_float2(-r.x, -r.y));
+    float2 p = __ffma2_rn(make_float2(kC4, kC4), f, make_float2(kC3, kC3));
+    p = __ffma2_rn(p, f, make_float2(kC2, kC2));
+    p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+    p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // ---- element types ------------------------------------------------------------------------
 // Unpack one 16-byte chunk into fp32 values.
 template <typename T>

@@ -27,6 +27,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 #include <type_traits>
 
@@ -55,6 +56,9 @@ constexpr uint32_t kTmemCols = 512;                  // S_A [0,128), S_B [128,25
 // A row's exponentials use a reference max that is only raised when the tile max exceeds it by
 // more than this (log2 units); the result is exact (softmax is shift invariant) and p <= 2^8.
 constexpr float kRescaleThreshold = 8.f;
+// Of each 32 exponentials of an unmasked key tile, 2 * POLY are computed by exp2_poly2 on the FMA
+// pipe (the kernel's template parameter; default kPolyPairs, PKV_PREFILL_POLY_PAIRS overrides it).
+constexpr int kPolyPairs = 2;
 
 // ---- tcgen05 / TMA primitives ---------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -173,7 +177,7 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     }
 }
 
-template <typename T>
+template <typename T, int POLY>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -419,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
-                        const float2 p = make_float2(fast_exp2(e.x), fast_exp2(e.y));
+                        const float2 p = i < POLY ? exp2_poly2(e) : make_float2(fast_exp2(e.x), fast_exp2(e.y));
                         ps2 = __fadd2_rn(ps2, p);
                         pk[i] = pack2<T>(p.x, p.y);
                     }
@@ -528,7 +532,7 @@ bool encode(CUtensorMap* m, CUtensorMapDataType t, int rank, const void* base, c
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T>
+template <typename T, int POLY>
 cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     const CUtensorMapDataType dt =
         std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -549,11 +553,28 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(prefill_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        e = cudaFuncSetAttribute(prefill_tc_kernel<T, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = 1;
     }
-    return launch_pdl(prefill_tc_kernel<T>, dim3(a.num_tiles), dim3(kThreads), SMEM_BYTES, s, a, mq, mk, mv);
+    return launch_pdl(prefill_tc_kernel<T, POLY>, dim3(a.num_tiles), dim3(kThreads), SMEM_BYTES, s, a, mq, mk, mv);
+}
+
+int poly_pairs() {
+    static const int v = [] {
+        const char* e = getenv("PKV_PREFILL_POLY_PAIRS");
+        return e ? atoi(e) : kPolyPairs;
+    }();
+    return v;
+}
+
+template <typename T>
+cudaError_t launch_p(const PrefillArgs& a, cudaStream_t s) {
+    switch (poly_pairs()) {
+        case 0: return launch_t<T, 0>(a, s);
+        case 4: return launch_t<T, 4>(a, s);
+        default: return launch_t<T, kPolyPairs>(a, s);
+    }
 }
 
 }  // namespace
@@ -566,7 +587,7 @@ cudaError_t launch_prefill_tc(int dtype, const PrefillArgs& a, int /*num_sms*/, 
     if (a.num_tiles <= 0) return cudaSuccess;
     if ((long long)a.num_blocks * a.num_kv_heads * kBlockSize >= (1LL << 31) - 1) return cudaErrorInvalidValue;
     if (((uintptr_t)a.q | (uintptr_t)a.k_pool | (uintptr_t)a.v_pool) & 15) return cudaErrorInvalidValue;
-    return dtype == 1 ? launch_t<__half>(a, s) : launch_t<__nv_bfloat16>(a, s);
+    return dtype == 1 ? launch_p<__half>(a, s) : launch_p<__nv_bfloat16>(a, s);
 }
 
 }  // namespace pkv
