@@ -65,6 +65,24 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.json), or None when there
+    is no record for this workload or the kernel's source changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+        if not rec or rec.get("workload") != workload:
+            return None
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def rank_seed(config: str, rank: int) -> int:
     """Each rank runs its own replica of the workload: same shapes, its own seeded data."""
     return 1000 + int(config[1]) + 100 * rank
@@ -367,8 +385,10 @@ def main():
     if dec_n:
         dec_avg_ms = dec_ms / dec_n
         achieved = decode_kernel_bytes(wl) / (dec_avg_ms * 1e-3) / 1e9
+        traffic = recorded_traffic("decode_kernel", wl.name)
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": None, "kernel": "decode_kernel (CUDA-core split-K)", "kernel_ms": dec_avg_ms,
+                "traffic": traffic, "algorithmic_bytes": decode_kernel_bytes(wl),
+                "kernel": "decode_kernel (CUDA-core split-K)", "kernel_ms": dec_avg_ms,
                 "peak_source": f"{peak_kind} hbm_gbs (burst copy)"}
     launches = sum(v[1] for k, v in prof.items() if k != "dropped")
     line = {
