@@ -46,7 +46,8 @@ typedef enum pkv_status {
     PKV_ERR_CUDA = 3,                 /* a CUDA runtime call failed; see pkv_last_error() */
     PKV_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below what the plan needs */
     PKV_ERR_DEVICE_TIMEOUT = 5,       /* a kernel's bounded wait expired (device error word only) */
-    PKV_ERR_DEVICE_RANGE = 6          /* a kernel met an out-of-range id (device error word only) */
+    PKV_ERR_DEVICE_RANGE = 6,         /* a kernel met an out-of-range id (device error word only) */
+    PKV_ERR_OUT_OF_BLOCKS = 7         /* the block pool has too few free blocks; nothing was changed */
 } pkv_status;
 
 typedef enum pkv_dtype { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
@@ -254,6 +255,86 @@ pkv_status pkv_paged_attention_static_ws(const int32_t* h_query_start_loc, const
  * x, y: device float arrays of n elements. Errors: INVALID_ARG, CUDA.
  */
 pkv_status pkv_selftest_exp2(const float* x, float* y, int n, pkv_stream_t stream);
+
+/*
+ * Host block manager (host memory only; no CUDA call). Owns the allocation state of one block pool:
+ * which physical blocks are free, each sequence's ordered block list and token count, and a
+ * reference count per block.
+ *   - 一文搞懂vLLM：为啥它能让一张GPU扛住几十倍用户？, "PagedAttention：核心思路": a sequence gets blocks
+ *     on demand (a new one only once its last block is full; any free block will do) and returns all
+ *     of them to the pool when it finishes.
+ *   - blog.mckayzhao.com/?p=56, "PagedAttention：操作系统课本里翻出来的灵感": N tokens hold
+ *     ceil(N / block_size) blocks, so at most block_size - 1 slots of a sequence are unused.
+ *   - same page, "还不止是分页：Copy-on-Write 和内存共享": forked sequences share blocks under a
+ *     reference count; before a sequence writes into a shared block, the block is copied and the
+ *     writer's table points at the copy (copy-on-write); the original is left as it was.
+ * Policy (not fixed by the pages, stated so results are reproducible): free blocks form a stack; a
+ * new pool hands out ids 0, 1, 2, ... in order, and a block whose count drops to 0 is pushed on
+ * top, so the most recently released block is reused first. A sequence's blocks are released last
+ * to first. Only the last block of a sequence can be partially filled, so only it can need a copy.
+ * Every call either succeeds completely or changes nothing. A manager is not thread-safe: callers
+ * serialise calls on one manager. Sequence ids are arbitrary int64 keys.
+ */
+typedef struct pkv_block_manager pkv_block_manager; /* opaque */
+
+typedef struct pkv_pool_stats {
+    int64_t num_blocks;     /* pool size */
+    int64_t free_blocks;    /* blocks with reference count 0 */
+    int64_t used_blocks;    /* num_blocks - free_blocks */
+    int64_t shared_blocks;  /* blocks with reference count > 1 */
+    int64_t num_sequences;  /* live sequences */
+    int64_t logical_tokens; /* sum of sequence lengths (a shared token counts once per sharer) */
+    int64_t stored_tokens;  /* filled slots of used blocks (a shared slot counts once) */
+    int64_t wasted_slots;   /* used_blocks * block_size - stored_tokens: reserved but unfilled */
+    int64_t cow_copies;     /* copy-on-write copies requested since creation */
+} pkv_pool_stats;
+
+/* Creates a manager for a pool of num_blocks blocks of block_size tokens (all free).
+ * Errors: INVALID_ARG (null out, num_blocks < 0, block_size < 1). */
+pkv_status pkv_bm_create(int num_blocks, int block_size, pkv_block_manager** out);
+/* Frees the manager (null is ignored). */
+void pkv_bm_destroy(pkv_block_manager* bm);
+/* Starts sequence seq_id holding num_tokens tokens: ceil(num_tokens / block_size) fresh blocks.
+ * Errors: INVALID_ARG (null, negative count, id already live), OUT_OF_BLOCKS. */
+pkv_status pkv_bm_add_sequence(pkv_block_manager* bm, int64_t seq_id, int64_t num_tokens);
+/* Starts sequence child sharing every block of parent (each block's count + 1), same length.
+ * Errors: INVALID_ARG (null, unknown parent, child already live). */
+pkv_status pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t child);
+/* Appends num_new_tokens tokens to seq_id, allocating the blocks they need. If the first new token
+ * goes into a partially filled last block that is shared, that block is copied first: cow_pair
+ * (2 int32, required) receives {source, destination} for pkv_copy_blocks, the sequence's last
+ * entry becomes the destination and the source's count drops by 1; otherwise {-1, -1}.
+ * Errors: INVALID_ARG (null, negative count, unknown id), OUT_OF_BLOCKS. */
+pkv_status pkv_bm_append(pkv_block_manager* bm, int64_t seq_id, int64_t num_new_tokens, int32_t* cow_pair);
+/* Ends seq_id: each of its blocks' counts drops by 1; blocks reaching 0 return to the free stack.
+ * Errors: INVALID_ARG (null, unknown id). */
+pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id);
+/* Reads one sequence: *num_tokens, *num_blocks, and (when blocks is not null) its block ids into
+ * blocks[0 .. *num_blocks). Errors: INVALID_ARG (null outputs, unknown id, capacity too small). */
+pkv_status pkv_bm_sequence(const pkv_block_manager* bm, int64_t seq_id, int64_t* num_tokens, int32_t* blocks,
+                           int capacity, int* num_blocks);
+/* Writes the block tables of num_seqs sequences as int32 rows of max_blocks_per_seq entries
+ * (host memory, caller-owned), unused entries -1. Errors: INVALID_ARG (unknown id, row too short). */
+pkv_status pkv_bm_block_tables(const pkv_block_manager* bm, const int64_t* seq_ids, int num_seqs, int32_t* tables,
+                               int max_blocks_per_seq);
+/* Reads one block's reference count. Errors: INVALID_ARG (null, id outside the pool). */
+pkv_status pkv_bm_refcount(const pkv_block_manager* bm, int32_t block, int32_t* count);
+/* Fills *stats. Errors: INVALID_ARG (null). */
+pkv_status pkv_bm_stats(const pkv_block_manager* bm, pkv_pool_stats* stats);
+/*
+ * One scheduling step of a {request_id: num_tokens} batch, all on the host: appends
+ * num_new_tokens[r] tokens to live sequence seq_ids[r] for every r (ids distinct), then writes the
+ * step's attention inputs into caller-owned host arrays: block_tables [num_seqs, max_blocks_per_seq]
+ * (-1 padded), context_lens [num_seqs] (lengths after the append), query_start_loc [num_seqs + 1]
+ * (prefix sum of num_new_tokens), and the copy-on-write pairs the appends need into
+ * cow_pairs [num_seqs, 2] with their count in *num_cow_pairs (at most one per sequence, in batch
+ * order). The pairs must be copied (pkv_copy_blocks) before this step's K/V is written.
+ * Errors: INVALID_ARG (null, unknown or repeated id, negative count, row too short, a length over
+ * INT32_MAX), OUT_OF_BLOCKS (checked for the whole batch first; nothing changes).
+ */
+pkv_status pkv_bm_step(pkv_block_manager* bm, const int64_t* seq_ids, const int32_t* num_new_tokens, int num_seqs,
+                       int32_t* block_tables, int max_blocks_per_seq, int32_t* context_lens,
+                       int32_t* query_start_loc, int32_t* cow_pairs, int* num_cow_pairs);
 
 /*
  * Kernel timing (no counterpart on the pages; a measurement aid). Between pkv_profile_start and

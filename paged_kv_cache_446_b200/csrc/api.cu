@@ -307,6 +307,7 @@ const char* pkv_status_string(pkv_status s) {
         case PKV_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
         case PKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case PKV_ERR_DEVICE_RANGE: return "device index out of range";
+        case PKV_ERR_OUT_OF_BLOCKS: return "out of free blocks";
     }
     return "unknown status";
 }

@@ -22,7 +22,9 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 PKV_OK = 0
 STATUS = {0: "PKV_OK", 1: "PKV_ERR_INVALID_ARG", 2: "PKV_ERR_UNSUPPORTED", 3: "PKV_ERR_CUDA",
-          4: "PKV_ERR_WORKSPACE_TOO_SMALL", 5: "PKV_ERR_DEVICE_TIMEOUT", 6: "PKV_ERR_DEVICE_RANGE"}
+          4: "PKV_ERR_WORKSPACE_TOO_SMALL", 5: "PKV_ERR_DEVICE_TIMEOUT", 6: "PKV_ERR_DEVICE_RANGE",
+          7: "PKV_ERR_OUT_OF_BLOCKS"}
+PKV_ERR_OUT_OF_BLOCKS = 7
 DTYPE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 DTYPE_NAME = {"f32": 0, "f16": 1, "bf16": 2}
 
@@ -284,3 +286,101 @@ def profile_stop() -> dict:
     out = {k: (ms[i], cnt[i]) for i, k in enumerate(KERNEL_KINDS)}
     out["dropped"] = dropped.value
     return out
+
+
+# ---- host block manager ------------------------------------------------------------------------
+
+class BmStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "num_blocks", "free_blocks", "used_blocks", "shared_blocks", "num_sequences", "logical_tokens",
+        "stored_tokens", "wasted_slots", "cow_copies")]
+
+
+_BM = ctypes.c_void_p
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_bm_create = _sig("pkv_bm_create", _I, [_I, _I, ctypes.POINTER(_BM)])
+_bm_destroy = _sig("pkv_bm_destroy", None, [_BM])
+_bm_add = _sig("pkv_bm_add_sequence", _I, [_BM, _I64, _I64])
+_bm_fork = _sig("pkv_bm_fork", _I, [_BM, _I64, _I64])
+_bm_append = _sig("pkv_bm_append", _I, [_BM, _I64, _I64, _I32P])
+_bm_free = _sig("pkv_bm_free", _I, [_BM, _I64])
+_bm_sequence = _sig("pkv_bm_sequence", _I, [_BM, _I64, ctypes.POINTER(_I64), _P, _I, ctypes.POINTER(_I)])
+_bm_tables = _sig("pkv_bm_block_tables", _I, [_BM, _P, _I, _P, _I])
+_bm_refcount = _sig("pkv_bm_refcount", _I, [_BM, ctypes.c_int32, _I32P])
+_bm_stats = _sig("pkv_bm_stats", _I, [_BM, ctypes.POINTER(BmStats)])
+_bm_step = _sig("pkv_bm_step", _I, [_BM, _P, _P, _I, _P, _I, _P, _P, _P, ctypes.POINTER(_I)])
+
+
+class BlockManager:
+    """Allocation state of one block pool (pkv_bm_* in include/pkv.h): on-demand blocks,
+    reference-counted sharing between forked sequences and copy-on-write of shared last blocks."""
+
+    def __init__(self, num_blocks: int, block_size: int = 16):
+        h = _BM()
+        _check(_bm_create(int(num_blocks), int(block_size), ctypes.byref(h)), "pkv_bm_create")
+        self._h = h
+        self.num_blocks = int(num_blocks)
+        self.block_size = int(block_size)
+
+    def __del__(self, _destroy=_bm_destroy):
+        if getattr(self, "_h", None):
+            _destroy(self._h)
+            self._h = None
+
+    def add(self, seq_id: int, num_tokens: int) -> None:
+        _check(_bm_add(self._h, int(seq_id), int(num_tokens)), "pkv_bm_add_sequence")
+
+    def fork(self, parent: int, child: int) -> None:
+        _check(_bm_fork(self._h, int(parent), int(child)), "pkv_bm_fork")
+
+    def append(self, seq_id: int, num_tokens: int) -> tuple[int, int] | None:
+        """Returns the (src, dst) copy the append needs, or None."""
+        pair = (ctypes.c_int32 * 2)()
+        _check(_bm_append(self._h, int(seq_id), int(num_tokens), pair), "pkv_bm_append")
+        return None if pair[0] < 0 else (pair[0], pair[1])
+
+    def free(self, seq_id: int) -> None:
+        _check(_bm_free(self._h, int(seq_id)), "pkv_bm_free")
+
+    def sequence(self, seq_id: int) -> tuple[int, list]:
+        """(tokens, block ids) of one sequence."""
+        tokens = _I64(0)
+        nb = _I(0)
+        _check(_bm_sequence(self._h, int(seq_id), ctypes.byref(tokens), None, 0, ctypes.byref(nb)), "pkv_bm_sequence")
+        blocks = np.empty(max(nb.value, 1), np.int32)
+        _check(_bm_sequence(self._h, int(seq_id), ctypes.byref(tokens), _np_ptr(blocks), blocks.shape[0],
+                            ctypes.byref(nb)), "pkv_bm_sequence")
+        return tokens.value, blocks[:nb.value].tolist()
+
+    def block_tables(self, seq_ids, max_blocks_per_seq: int) -> np.ndarray:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        out = np.empty((ids.shape[0], int(max_blocks_per_seq)), np.int32)
+        _check(_bm_tables(self._h, _np_ptr(ids), ids.shape[0], _np_ptr(out), int(max_blocks_per_seq)),
+               "pkv_bm_block_tables")
+        return out
+
+    def refcount(self, block: int) -> int:
+        c = ctypes.c_int32(0)
+        _check(_bm_refcount(self._h, int(block), ctypes.byref(c)), "pkv_bm_refcount")
+        return c.value
+
+    def stats(self) -> dict:
+        st = BmStats()
+        _check(_bm_stats(self._h, ctypes.byref(st)), "pkv_bm_stats")
+        return {n: getattr(st, n) for n, _ in BmStats._fields_}
+
+    def step(self, batch: dict, max_blocks_per_seq: int):
+        """Appends batch {seq_id: num_new_tokens} (dict order) and returns the step's host inputs:
+        (block_tables int32 [R, max_blocks_per_seq], context_lens int32 [R], query_start_loc int32 [R+1],
+        copy pairs int32 [P, 2])."""
+        ids = np.fromiter(batch.keys(), np.int64, len(batch))
+        n = np.fromiter(batch.values(), np.int32, len(batch))
+        R = ids.shape[0]
+        tables = np.empty((R, int(max_blocks_per_seq)), np.int32)
+        ctx = np.empty(R, np.int32)
+        qsl = np.empty(R + 1, np.int32)
+        pairs = np.empty((max(R, 1), 2), np.int32)
+        npairs = _I(0)
+        _check(_bm_step(self._h, _np_ptr(ids), _np_ptr(n), R, _np_ptr(tables), int(max_blocks_per_seq), _np_ptr(ctx),
+                        _np_ptr(qsl), _np_ptr(pairs), ctypes.byref(npairs)), "pkv_bm_step")
+        return tables, ctx, qsl, pairs[:npairs.value].copy()

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_function(pkv):
 
 
 def test_status_strings(pkv):
-    for code in range(7):
+    for code in range(8):
         assert pkv._lib.pkv_status_string(code)
     assert "sm_100a" in pkv.version()
 
