@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5", "c6"])
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -53,7 +53,13 @@ def parse():
                     help="time only the prefill or decode requests of the workload")
     ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling subsets)")
     ap.add_argument("--heads-per-item", type=int, default=0, help="query heads per CUDA-core work item")
+    ap.add_argument("--rows-per-item", type=int, default=0, help="query rows of a request per CUDA-core work item")
+    ap.add_argument("--tc-min-rows", type=int, default=0, help="fewest rows a request needs for the tcgen05 tiles")
+    ap.add_argument("--cuda-core-only", action="store_true", help="serve every row on CUDA cores")
     return ap.parse_args()
+
+
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def peaks():
@@ -63,6 +69,17 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense 16-bit tensor-core peak (TFLOP/s) for a kernel timed alone: the measured burst figure."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def recorded_traffic(kernel: str, workload: str):
@@ -118,16 +135,16 @@ def decode_seq_tokens(wl) -> int:
     return int(ctx[n == 1].sum())
 
 
-def decode_kernel_bytes(wl) -> int:
-    """Algorithmic bytes of the CUDA-core kernel per launch: K+V of every decode row's (request, KV
-    head) context, plus its q rows read and output rows written."""
-    ctx = workload_desc(wl)
-    n = np.asarray(list(wl.batch.values()))
+def kernel_work(plan, wl) -> dict:
+    """Algorithmic work per launch from the plan: the CUDA-core kernel reads K+V of its requests'
+    contexts once per (request, KV head) plus its q rows and writes its output rows; the tcgen05
+    tiles likewise for theirs, and compute 4*D flops per (row, head, attended key)."""
     eb = 4 if wl.dtype == "f32" else 2
-    dec = n == 1
-    kv = int(ctx[dec].sum()) * wl.num_kv_heads * 2 * wl.head_dim * eb
-    qo = int(dec.sum()) * wl.num_q_heads * wl.head_dim * eb * 2
-    return kv + qo
+    row_bytes = wl.num_q_heads * wl.head_dim * eb * 2
+    core_rows = plan.num_q_tokens - plan.num_prefill_rows
+    return {"decode": {"bytes": int(plan.core_kv_bytes) + core_rows * row_bytes},
+            "prefill_tc": {"bytes": int(plan.tile_kv_bytes) + plan.num_prefill_rows * row_bytes,
+                           "flops": int(plan.tile_flops)}}
 
 
 class ClockSampler:
@@ -296,6 +313,12 @@ def main():
     opts = {"split_blocks": args.split_blocks} if args.split_blocks else {}
     if args.heads_per_item:
         opts["heads_per_item"] = args.heads_per_item
+    if args.rows_per_item:
+        opts["rows_per_item"] = args.rows_per_item
+    if args.tc_min_rows:
+        opts["tc_min_rows"] = args.tc_min_rows
+    if args.cuda_core_only:
+        opts["cuda_core_only"] = True
     step = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,
                               wl.num_kv_heads, wl.head_dim, dt, dev, write_batch=wl.write_batch or None,
                               copy_pairs=wl.copy_pairs, **opts)
@@ -390,16 +413,29 @@ def main():
         return
     peak, peak_kind = peaks()
     value = whole_job_gbs(kv_bytes(wl), world, ms_per_step)
-    dec_ms, dec_n = prof["decode"]
+    # Roofline of the kernel that takes the most time per step.
+    work = kernel_work(step.plan.plan, wl)
+    names = {"decode": "decode_kernel (CUDA-core split-K)", "prefill_tc": "prefill_tc_kernel (tcgen05 tiles)"}
+    timed = {k: prof[k] for k in work if prof[k][1]}
     roof = None
-    if dec_n:
-        dec_avg_ms = dec_ms / dec_n
-        achieved = decode_kernel_bytes(wl) / (dec_avg_ms * 1e-3) / 1e9
-        traffic = recorded_traffic("decode_kernel", wl.name)
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": traffic, "algorithmic_bytes": decode_kernel_bytes(wl),
-                "kernel": "decode_kernel (CUDA-core split-K)", "kernel_ms": dec_avg_ms,
-                "peak_source": f"{peak_kind} hbm_gbs (burst copy)"}
+    if timed:
+        k = max(timed, key=lambda x: timed[x][0])
+        avg_ms = timed[k][0] / timed[k][1]
+        w = work[k]
+        tc_peak, tc_kind = tensor_peak()
+        t_hbm = w["bytes"] / (peak * 1e9)
+        t_tc = w.get("flops", 0) / (tc_peak * 1e12)
+        if t_tc > t_hbm:
+            achieved = w["flops"] / (avg_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": achieved / tc_peak, "traffic": recorded_traffic(k + "_kernel", wl.name),
+                    "algorithmic_flops": w["flops"], "peak_source": f"{tc_kind} bf16_tflops (burst cuBLAS)"}
+        else:
+            achieved = w["bytes"] / (avg_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": recorded_traffic(k + "_kernel", wl.name), "algorithmic_bytes": w["bytes"],
+                    "peak_source": f"{peak_kind} hbm_gbs (burst copy)"}
+        roof.update(kernel=names[k], kernel_ms=avg_ms)
     launches = sum(v[1] for k, v in prof.items() if k != "dropped")
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -410,7 +446,8 @@ def main():
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
                    "num_blocks": wl.num_blocks, "kv_bytes_per_step_per_gpu": kv_bytes(wl),
                    "l2": "inputs larger than L2 (KV pool read per step >> 126 MB); no flush",
-                   "parallelism": f"replicas x{world} (independent requests per GPU)"},
+                   "parallelism": f"replicas x{world} (independent requests per GPU)",
+                   "plan_options": opts},
         "frac_of_hbm_peak": value / world / peak,
         "decode_seq_tokens_per_s": world * decode_seq_tokens(wl) / (ms_per_step * 1e-3),
         "decode_steps_per_s": 1e3 / ms_per_step,

@@ -117,6 +117,11 @@ typedef struct pkv_plan_options {
     int32_t heads_per_item;    /* query heads of one group served by one CUDA-core work item
                                   (1..8); 0 = min(Hq/Hkv, 8). Larger groups are split into items
                                   that read the same K/V blocks */
+    int32_t rows_per_item;     /* consecutive query rows of one request served by one CUDA-core
+                                  item, capped so rows x heads <= 8; 0 = as many as fit. Such an
+                                  item streams each K/V block once for all its (row, head) pairs */
+    int32_t tc_min_rows;       /* requests with at least this many rows (>= 2; 0 = 2) go to the
+                                  tcgen05 tiles where the shape allows; fewer rows, CUDA cores */
 } pkv_plan_options;
 
 /*
@@ -128,14 +133,14 @@ typedef struct pkv_plan {
     int32_t num_reqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim, dtype;
     int32_t num_decode_rows;     /* rows served by the CUDA-core split-K kernel */
     int32_t num_prefill_rows;    /* rows served by the tcgen05 tile kernel */
-    int32_t num_items;           /* CUDA-core work items (row, kv head, block chunk) */
+    int32_t num_items;           /* CUDA-core work items (rows, kv head, heads, block chunk) */
     int32_t num_tiles;           /* tcgen05 tiles (request, kv head, 128 packed rows) */
-    int32_t num_merge_rows;      /* (row, kv head) pairs merged from several chunks */
+    int32_t num_merge_rows;      /* chunked CUDA-core items' (rows, heads) sets merged from partials */
     int32_t num_partials;        /* chunk partial results in the workspace */
     int32_t split_blocks;        /* chunk length in blocks used for this batch */
     int32_t max_blocks;          /* longest context in blocks */
     int32_t heads_per_item;      /* query heads per CUDA-core work item */
-    int32_t reserved;
+    int32_t rows_per_item;       /* most consecutive rows any CUDA-core item serves (0: no items) */
     int64_t off_items, off_tiles, off_merge, off_part_o, off_part_ml; /* byte offsets into workspace */
     int64_t meta_bytes;          /* bytes uploaded by pkv_attention_plan (work lists) */
     int64_t ws_bytes;            /* total workspace bytes this plan needs */
@@ -143,6 +148,9 @@ typedef struct pkv_plan {
                                     2*D*elem per (kv head, key), counted once per (request, kv head)
                                     for decode rows and once per request for prefill rows */
     int64_t attn_flops;          /* 4*D per (query row, query head, attended key) */
+    int64_t core_kv_bytes;       /* part of kv_bytes read by the CUDA-core kernel */
+    int64_t tile_kv_bytes;       /* part of kv_bytes read by the tcgen05 tiles */
+    int64_t tile_flops;          /* part of attn_flops computed by the tcgen05 tiles */
 } pkv_plan;
 
 /*
@@ -258,8 +266,8 @@ pkv_status pkv_selftest_exp2(const float* x, float* y, int n, pkv_stream_t strea
 
 /*
  * Host block manager (host memory only; no CUDA call). Owns the allocation state of one block pool:
- * which physical blocks are free, each sequence's ordered block list and token count, and a
- * reference count per block.
+ * which physical blocks are free, each sequence's ordered block list and token count, a reference
+ * count per block and, optionally, a cache of full blocks keyed by the token prefix they end.
  *   - 一文搞懂vLLM：为啥它能让一张GPU扛住几十倍用户？, "PagedAttention：核心思路": a sequence gets blocks
  *     on demand (a new one only once its last block is full; any free block will do) and returns all
  *     of them to the pool when it finishes.
@@ -268,18 +276,32 @@ pkv_status pkv_selftest_exp2(const float* x, float* y, int n, pkv_stream_t strea
  *   - same page, "还不止是分页：Copy-on-Write 和内存共享": forked sequences share blocks under a
  *     reference count; before a sequence writes into a shared block, the block is copied and the
  *     writer's table points at the copy (copy-on-write); the original is left as it was.
- * Policy (not fixed by the pages, stated so results are reproducible): free blocks form a stack; a
- * new pool hands out ids 0, 1, 2, ... in order, and a block whose count drops to 0 is pushed on
- * top, so the most recently released block is reused first. A sequence's blocks are released last
- * to first. Only the last block of a sequence can be partially filled, so only it can need a copy.
+ *   - 一文搞懂vLLM：为啥它能让一张GPU扛住几十倍用户？, "PagedAttention 是怎么共享内存的": requests that
+ *     begin with the same prefix store its blocks once and each table points at them;
+ *     blog.mckayzhao.com/?p=56, "进阶特性：让推理再快一点" (Prefix Caching), and vLLM 简介
+ *     (docs.freetools.me), "自动前缀缓存": prefix caching is hash based: when the beginning of a new
+ *     request matches blocks computed before, those KV blocks are reused instead of recomputed.
+ * Policy (not fixed by the pages, stated so results are reproducible): free blocks form a queue. A
+ * new pool hands out ids 0, 1, 2, ... in order; a block whose count drops to 0 joins the back, and
+ * allocation takes the front, so the least recently released block is reused first. A sequence's
+ * blocks are released last to first (its later blocks leave the cache before its prefix). Only the
+ * last block of a sequence can be partially filled, so only it can need a copy.
+ * Prefix cache (managers created with PKV_BM_PREFIX_CACHE): every block of a token-tracked sequence
+ * that becomes full is registered under a chain hash of all tokens up to its end (SplitMix64 mixing
+ * of the previous block's key and the block's token ids). A released registered block stays
+ * reusable, with its contents, until allocation takes it from the front of the queue (eviction).
+ * A lookup accepts a block only if its recorded token ids and the identity of the block before it
+ * match, so a hit is exact, not merely hash-equal.
  * Every call either succeeds completely or changes nothing. A manager is not thread-safe: callers
  * serialise calls on one manager. Sequence ids are arbitrary int64 keys.
  */
 typedef struct pkv_block_manager pkv_block_manager; /* opaque */
 
+#define PKV_BM_PREFIX_CACHE 1 /* pkv_bm_create_ex flag: keep a prefix cache of full blocks */
+
 typedef struct pkv_pool_stats {
     int64_t num_blocks;     /* pool size */
-    int64_t free_blocks;    /* blocks with reference count 0 */
+    int64_t free_blocks;    /* blocks with reference count 0 (cached ones included) */
     int64_t used_blocks;    /* num_blocks - free_blocks */
     int64_t shared_blocks;  /* blocks with reference count > 1 */
     int64_t num_sequences;  /* live sequences */
@@ -287,26 +309,47 @@ typedef struct pkv_pool_stats {
     int64_t stored_tokens;  /* filled slots of used blocks (a shared slot counts once) */
     int64_t wasted_slots;   /* used_blocks * block_size - stored_tokens: reserved but unfilled */
     int64_t cow_copies;     /* copy-on-write copies requested since creation */
+    int64_t cached_blocks;  /* blocks a prefix lookup can currently return (held or free) */
+    int64_t cache_queries;  /* full prompt blocks looked up since creation */
+    int64_t cache_hits;     /* of those, blocks reused from the cache */
 } pkv_pool_stats;
 
-/* Creates a manager for a pool of num_blocks blocks of block_size tokens (all free).
- * Errors: INVALID_ARG (null out, num_blocks < 0, block_size < 1). */
+/* Creates a manager for a pool of num_blocks blocks of block_size tokens (all free), without a
+ * prefix cache. Errors: INVALID_ARG (null out, num_blocks < 0, block_size < 1). */
 pkv_status pkv_bm_create(int num_blocks, int block_size, pkv_block_manager** out);
+/* Same, with flags (0 or PKV_BM_PREFIX_CACHE). Errors: as above, or unknown flag bits. */
+pkv_status pkv_bm_create_ex(int num_blocks, int block_size, int flags, pkv_block_manager** out);
 /* Frees the manager (null is ignored). */
 void pkv_bm_destroy(pkv_block_manager* bm);
 /* Starts sequence seq_id holding num_tokens tokens: ceil(num_tokens / block_size) fresh blocks.
+ * Its token ids are unknown, so none of its blocks enters the prefix cache.
  * Errors: INVALID_ARG (null, negative count, id already live), OUT_OF_BLOCKS. */
 pkv_status pkv_bm_add_sequence(pkv_block_manager* bm, int64_t seq_id, int64_t num_tokens);
-/* Starts sequence child sharing every block of parent (each block's count + 1), same length.
- * Errors: INVALID_ARG (null, unknown parent, child already live). */
+/* Starts token-tracked sequence seq_id from the longest cached prefix of its prompt tokens[0, n)
+ * (host int32 token ids): the sequence holds the hit blocks (each block's count + 1) and
+ * *num_cached_tokens = hits * block_size of them. At most (n - 1) / block_size blocks are taken
+ * from the cache, so at least one prompt token is always left to compute. The caller appends the
+ * remaining tokens[*num_cached_tokens, n) with pkv_bm_append_tokens or pkv_bm_step; their K/V must
+ * be computed and written, the cached ones must not. Without a prefix cache nothing hits.
+ * Errors: INVALID_ARG (null, n < 0, id already live). Takes no free block for itself. */
+pkv_status pkv_bm_add_cached_prefix(pkv_block_manager* bm, int64_t seq_id, const int32_t* tokens, int64_t n,
+                                    int64_t* num_cached_tokens);
+/* Starts sequence child sharing every block of parent (each block's count + 1), same length and
+ * token ids. Errors: INVALID_ARG (null, unknown parent, child already live). */
 pkv_status pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t child);
 /* Appends num_new_tokens tokens to seq_id, allocating the blocks they need. If the first new token
  * goes into a partially filled last block that is shared, that block is copied first: cow_pair
  * (2 int32, required) receives {source, destination} for pkv_copy_blocks, the sequence's last
  * entry becomes the destination and the source's count drops by 1; otherwise {-1, -1}.
- * Errors: INVALID_ARG (null, negative count, unknown id), OUT_OF_BLOCKS. */
+ * The token ids are not given: a token-tracked sequence stops being tracked (its later blocks
+ * are not cached). Errors: INVALID_ARG (null, negative count, unknown id), OUT_OF_BLOCKS. */
 pkv_status pkv_bm_append(pkv_block_manager* bm, int64_t seq_id, int64_t num_new_tokens, int32_t* cow_pair);
-/* Ends seq_id: each of its blocks' counts drops by 1; blocks reaching 0 return to the free stack.
+/* Same, with the new tokens' ids (host int32 [num_new_tokens]); on a prefix-caching manager each
+ * block of a token-tracked sequence that becomes full is registered in the cache. */
+pkv_status pkv_bm_append_tokens(pkv_block_manager* bm, int64_t seq_id, const int32_t* tokens,
+                                int64_t num_new_tokens, int32_t* cow_pair);
+/* Ends seq_id: each of its blocks' counts drops by 1, last block first; blocks reaching 0 join the
+ * back of the free queue (a registered block keeps its cache entry until it is taken again).
  * Errors: INVALID_ARG (null, unknown id). */
 pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id);
 /* Reads one sequence: *num_tokens, *num_blocks, and (when blocks is not null) its block ids into
@@ -329,12 +372,15 @@ pkv_status pkv_bm_stats(const pkv_block_manager* bm, pkv_pool_stats* stats);
  * (prefix sum of num_new_tokens), and the copy-on-write pairs the appends need into
  * cow_pairs [num_seqs, 2] with their count in *num_cow_pairs (at most one per sequence, in batch
  * order). The pairs must be copied (pkv_copy_blocks) before this step's K/V is written.
+ * new_tokens (nullable) holds the new tokens' ids, concatenated in batch order
+ * (query_start_loc[num_seqs] entries) as pkv_bm_append_tokens takes them; when null, every
+ * token-tracked member stops being tracked, as with pkv_bm_append.
  * Errors: INVALID_ARG (null, unknown or repeated id, negative count, row too short, a length over
  * INT32_MAX), OUT_OF_BLOCKS (checked for the whole batch first; nothing changes).
  */
 pkv_status pkv_bm_step(pkv_block_manager* bm, const int64_t* seq_ids, const int32_t* num_new_tokens, int num_seqs,
-                       int32_t* block_tables, int max_blocks_per_seq, int32_t* context_lens,
-                       int32_t* query_start_loc, int32_t* cow_pairs, int* num_cow_pairs);
+                       const int32_t* new_tokens, int32_t* block_tables, int max_blocks_per_seq,
+                       int32_t* context_lens, int32_t* query_start_loc, int32_t* cow_pairs, int* num_cow_pairs);
 
 /*
  * Kernel timing (no counterpart on the pages; a measurement aid). Between pkv_profile_start and

@@ -79,7 +79,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
                       const pkv_plan_options* opts, int num_sms, PlanLists* L, pkv_plan* plan) {
     if (!qsl || (R > 0 && !ctx) || !plan) return fail(PKV_ERR_INVALID_ARG, "null planner argument");
     if (R < 0) return fail(PKV_ERR_INVALID_ARG, "num_reqs < 0");
-    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Hkv > 32767)
         return fail(PKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)", Hq, Hkv);
     if (D != 64 && D != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", D);
     if (!dtype_ok(dt)) return fail(PKV_ERR_INVALID_ARG, "bad dtype %d", (int)dt);
@@ -94,23 +94,33 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     pkv_plan_options o{};
     if (opts) o = *opts;
     const bool tc_ok = !o.cuda_core_only && prefill_tc_supported((int)dt, D, G);
+    const int tc_min = o.tc_min_rows > 2 ? o.tc_min_rows : 2;
     const int eb = elem_bytes(dt);
+    const int hpi = (o.heads_per_item > 0 && o.heads_per_item <= kMaxGroupPerItem) ? o.heads_per_item
+                                                                                  : std::min(G, kMaxGroupPerItem);
+    // Rows per CUDA-core item: as many consecutive rows of a request as fit 8 (row, head) slots.
+    const int rows_cap = kMaxGroupPerItem / hpi;
+    const int rpi = o.rows_per_item > 0 ? std::min(o.rows_per_item, rows_cap) : rows_cap;
 
-    struct CoreRow { int row, req, limit; };
+    struct CoreRow { int row, req, limit, nrows; };  // nrows consecutive rows; the first sees keys < limit
     static thread_local std::vector<CoreRow> core_rows;
     core_rows.clear();
     core_rows.reserve(R > 0 ? (size_t)qsl[R] : 0);
-    int64_t kv_bytes = 0, flops = 0;
+    int64_t kv_bytes = 0, flops = 0, tile_kv = 0, tile_flops = 0;
     int decode_rows = 0, prefill_rows = 0, max_blocks = 0;
     for (int r = 0; r < R; ++r) {
         const int n = qsl[r + 1] - qsl[r];
         if (n == 0) continue;
         const int P = ctx[r] - n;
         max_blocks = std::max<int>(max_blocks, (int)ceil_div(ctx[r], kBlockSize));
-        kv_bytes += (int64_t)ctx[r] * Hkv * 2 * D * eb;
+        const int64_t req_kv = (int64_t)ctx[r] * Hkv * 2 * D * eb;
         // keys attended: sum_j (P + j + 1)
-        flops += 4LL * D * Hq * ((int64_t)n * P + (int64_t)n * (n + 1) / 2);
-        if (n > 1 && tc_ok) {
+        const int64_t req_flops = 4LL * D * Hq * ((int64_t)n * P + (int64_t)n * (n + 1) / 2);
+        kv_bytes += req_kv;
+        flops += req_flops;
+        if (n > 1 && tc_ok && n >= tc_min) {
+            tile_kv += req_kv;
+            tile_flops += req_flops;
             prefill_rows += n;
             const int tt = tile_tokens(G);
             for (int h = 0; h < Hkv; ++h)
@@ -121,15 +131,13 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
                 }
         } else {
             if (n == 1) ++decode_rows;
-            for (int j = 0; j < n; ++j) core_rows.push_back(CoreRow{qsl[r] + j, r, P + j + 1});
+            for (int j = 0; j < n; j += rpi) core_rows.push_back(CoreRow{qsl[r] + j, r, P + j + 1, std::min(rpi, n - j)});
         }
     }
-    const int hpi = (o.heads_per_item > 0 && o.heads_per_item <= kMaxGroupPerItem) ? o.heads_per_item
-                                                                                  : std::min(G, kMaxGroupPerItem);
     // Chunk length: enough items for ~4 per resident warp, but never below 8 blocks.
     const int groups = (int)ceil_div(G, hpi);
     int64_t total_blocks = 0;
-    for (const CoreRow& c : core_rows) total_blocks += ceil_div(c.limit, kBlockSize) * Hkv * groups;
+    for (const CoreRow& c : core_rows) total_blocks += ceil_div(c.limit + c.nrows - 1, kBlockSize) * Hkv * groups;
     int chunk;
     if (o.no_split) chunk = 1 << 30;
     else if (o.split_blocks > 0) chunk = o.split_blocks;
@@ -143,7 +151,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     size_t n_items = 0, n_merge = 0;
     int max_len = 0;
     for (const CoreRow& c : core_rows) {
-        const int nb = (int)ceil_div(c.limit, kBlockSize);
+        const int nb = (int)ceil_div(c.limit + c.nrows - 1, kBlockSize);
         const int pieces = (int)ceil_div(nb, chunk);
         n_items += (size_t)pieces * Hkv * groups;
         if (pieces > 1) n_merge += (size_t)Hkv * groups;
@@ -152,7 +160,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     std::vector<size_t>& start = L->start;
     start.assign((size_t)max_len + 2, 0);
     for (const CoreRow& c : core_rows) {
-        const int nb = (int)ceil_div(c.limit, kBlockSize);
+        const int nb = (int)ceil_div(c.limit + c.nrows - 1, kBlockSize);
         const int pieces = (int)ceil_div(nb, chunk);
         const size_t per = (size_t)Hkv * groups;
         start[std::min(nb, chunk)] += per * (pieces > 1 ? pieces - 1 : 1);
@@ -172,7 +180,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     size_t mi = 0;
     int partials = 0;
     for (const CoreRow& c : core_rows) {
-        const int nb = (int)ceil_div(c.limit, kBlockSize);
+        const int nb = (int)ceil_div(c.limit + c.nrows - 1, kBlockSize);
         const int pieces = (int)ceil_div(nb, chunk);
         for (int h = 0; h < Hkv; ++h)
             for (int g0 = 0; g0 < G; g0 += hpi) {
@@ -180,11 +188,13 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
                 if (pieces > 1) {
                     first = partials;
                     partials += pieces;
-                    merges[mi++] = MergeRow{c.row, h * G + g0, std::min(hpi, G - g0), first, pieces, {0, 0, 0}};
+                    const int nh = std::min(hpi, G - g0);
+                    merges[mi++] = MergeRow{c.row, h * G + g0, nh * c.nrows, first, pieces, nh, {0, 0}};
                 }
                 for (int p = 0; p < pieces; ++p) {
                     const int b0 = p * chunk, b1 = std::min(nb, b0 + chunk);
-                    items[pos[b1 - b0]++] = DecodeItem{c.row, c.req, h, g0, b0, b1, c.limit, pieces > 1 ? first + p : -1};
+                    items[pos[b1 - b0]++] = DecodeItem{c.row, c.req, (int16_t)h, (int16_t)c.nrows, g0, b0, b1, c.limit,
+                                                       pieces > 1 ? first + p : -1};
                 }
             }
     }
@@ -218,6 +228,9 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->split_blocks = chunk;
     plan->max_blocks = max_blocks;
     plan->heads_per_item = hpi;
+    int max_rows = 0;
+    for (const CoreRow& c : core_rows) max_rows = std::max(max_rows, c.nrows);
+    plan->rows_per_item = max_rows;
     int64_t off = 256;  // first 256 bytes reserved
     plan->off_items = off;
     off = align256(off + (int64_t)L->items.size() * sizeof(DecodeItem));
@@ -233,6 +246,9 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->ws_bytes = off;
     plan->kv_bytes = kv_bytes;
     plan->attn_flops = flops;
+    plan->core_kv_bytes = kv_bytes - tile_kv;
+    plan->tile_kv_bytes = tile_kv;
+    plan->tile_flops = tile_flops;
     return PKV_OK;
 }
 
@@ -478,7 +494,9 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         a.part_ml = reinterpret_cast<float*>(ws + plan->off_part_ml);
         a.err = err; a.num_items = plan->num_items; a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks; a.num_q_heads = plan->num_q_heads; a.num_kv_heads = plan->num_kv_heads;
-        a.group = G; a.heads_per_item = plan->heads_per_item; a.scale_log2 = scale_log2;
+        a.group = G; a.heads_per_item = plan->heads_per_item;
+        a.slots_per_item = plan->heads_per_item * std::max(plan->rows_per_item, 1);
+        a.scale_log2 = scale_log2;
         ProfileScope prof(PKV_KERNEL_DECODE, s);
         cudaError_t e = launch_decode(plan->dtype, plan->head_dim, a, sms, s);
         if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -491,7 +509,7 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         m.part_ml = reinterpret_cast<const float*>(ws + plan->off_part_ml);
         m.num_rows = plan->num_merge_rows;
         m.num_q_heads = plan->num_q_heads;
-        m.heads_per_entry = plan->heads_per_item;
+        m.slots_per_entry = plan->heads_per_item * std::max(plan->rows_per_item, 1);
         ProfileScope prof(PKV_KERNEL_MERGE, s);
         cudaError_t e = launch_merge(plan->dtype, plan->head_dim, m, s);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");

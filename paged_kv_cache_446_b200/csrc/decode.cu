@@ -3,11 +3,15 @@
 //
 // What it computes follows blog.mckayzhao.com/?p=56, "PagedAttention：操作系统课本里翻出来的灵感":
 // each KV block of a request is found through its block table and K and V are read block by block;
-// the result equals attention over contiguous storage. Rows of any length are served (decode rows
-// and, one row at a time with a causal limit, prefill rows that the tcgen05 path does not take).
+// the result equals attention over contiguous storage. Rows of any length are served: decode rows,
+// and the rows of multi-token requests that the tcgen05 path does not take -- a speculative verify
+// step, where a request submits its k draft tokens plus one (一文搞懂vLLM：为啥它能让一张GPU扛住几十倍用户？,
+// "V1 架构：推倒重来的勇气": the step is a {request_id: num_tokens} dictionary), or rows of fp32 /
+// other shapes -- each row with its causal limit.
 //
 // Design (B200): every warp is an independent persistent worker. It walks a static round-robin
-// share of the planner's work items (row, KV head, up to 8 query heads, block range) and streams
+// share of the planner's work items (consecutive rows of a request x up to 8 query heads of a KV
+// head -- at most 8 (row, head) slots that share every K/V block -- and a block range) and streams
 // each (block, KV head) K and V chunk -- a contiguous 16*D run in the pool -- with one
 // cp.async.bulk (TMA engine, no tensor map) into a private ring of shared-memory stages,
 // completion tracked by an mbarrier per stage. The ring runs ahead across item boundaries, so
@@ -66,7 +70,10 @@ __device__ __forceinline__ DecodeItem load_item(const DecodeItem* items, int i) 
     const int4* p = reinterpret_cast<const int4*>(items + i);
     const int4 a = __ldg(p), b = __ldg(p + 1);
     DecodeItem it;
-    it.row = a.x; it.req = a.y; it.kv_head = a.z; it.head0 = a.w;
+    it.row = a.x; it.req = a.y;
+    it.kv_head = (int16_t)(a.z & 0xffff);                   // low half of the third word
+    it.num_rows = (int16_t)((unsigned)a.z >> 16);           // high half
+    it.head0 = a.w;
     it.blk_begin = b.x; it.blk_end = b.y; it.limit = b.z; it.partial = b.w;
     return it;
 }
@@ -121,14 +128,19 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
             unsigned char* st = wbase + stage * C::STAGE;
             const bool first = (p_blk == pi.blk_begin);
             const int nh = min(a.heads_per_item, a.group - pi.head0);
-            const uint32_t qbytes = first ? (uint32_t)(nh * C::ROW) : 0u;
+            const uint32_t qrow = (uint32_t)(nh * C::ROW);  // one row's heads, contiguous in q
+            const uint32_t qbytes = first ? qrow * (uint32_t)pi.num_rows : 0u;
             mbar_arrive_expect_tx(&bars[stage], 2u * C::BLK + qbytes);
             const size_t off = ((size_t)id * a.num_kv_heads + pi.kv_head) * head_stride;
             bulk_g2s(st, kp + off, C::BLK, &bars[stage]);
             bulk_g2s(st + C::BLK, vp + off, C::BLK, &bars[stage]);
             if (first) {
-                const size_t qoff = ((size_t)pi.row * a.num_q_heads + (size_t)pi.kv_head * a.group + pi.head0) * C::ROW;
-                bulk_g2s(st + 2 * C::BLK, qp + qoff, qbytes, &bars[stage]);
+                // The item's (row, head) slots land contiguously: slot j * nh + h at (j * nh + h) * ROW.
+                for (int j = 0; j < pi.num_rows; ++j) {
+                    const size_t qoff =
+                        ((size_t)(pi.row + j) * a.num_q_heads + (size_t)pi.kv_head * a.group + pi.head0) * C::ROW;
+                    bulk_g2s(st + 2 * C::BLK + j * qrow, qp + qoff, qrow, &bars[stage]);
+                }
             }
         }
         ++issued;
@@ -174,9 +186,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
     const int gm = M / C::PASSES;              // head-slot permutation
     const int im = M % C::PASSES;              // pass permutation
 
-    float2 q2[GP][C::E2];                      // q (scaled, log2 domain), head slots permuted by gm
-    float2 acc2[GP][C::E2];                    // output accumulator, logical head order
+    float2 q2[GP][C::E2];                      // q (scaled, log2 domain), slots permuted by gm
+    float2 acc2[GP][C::E2];                    // output accumulator, logical slot order
     float m_own = -INFINITY, l_own = 0.f;
+    int own_limit = 0;                         // keys visible to the slot this lane owns
 
     while (true) {
         const int stage = consumed % C::STAGES;
@@ -192,12 +205,14 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
         const unsigned char* Ks = st;
         const unsigned char* Vs = st + C::BLK;
         const int nh = min(a.heads_per_item, a.group - ci.head0);
+        const int ns = nh * ci.num_rows;          // (row, head) slots of the item
 
         if (c_blk == ci.blk_begin) {
+            own_limit = ci.limit + (g_own < ns ? g_own / nh : 0);
 #pragma unroll
             for (int gs = 0; gs < GP; ++gs) {
                 const int g = gs ^ gm;
-                if (g < nh) {
+                if (g < ns) {
                     float f[C::EPC];
                     Chunk<T>::unpack(lds128(st + 2 * C::BLK + g * C::ROW + chunk * 16), f);
 #pragma unroll
@@ -212,7 +227,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
             m_own = -INFINITY;
             l_own = 0.f;
         }
-        const int valid = min(kBlockSize, ci.limit - c_blk * kBlockSize);
+        // Keys of this block visible to the item's last row (V rows past it are zeroed) and to the
+        // slot this lane owns (its scores past it are masked).
+        const int valid = min(kBlockSize, ci.limit + ci.num_rows - 1 - c_blk * kBlockSize);
+        const int valid_own = own_limit - c_blk * kBlockSize;
 
         // ---- QK: partial dots of this lane's chunk for every (head slot, pass slot) ----
         float dots[C::NV];
@@ -245,7 +263,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
 #pragma unroll
         for (int k = 0; k < C::NOWN; ++k) {
             const int t = (i_own0 + k) * C::TPP + sub;
-            if (t >= valid) dots[k] = -INFINITY;
+            if (t >= valid_own) dots[k] = -INFINITY;
             mb = fmaxf(mb, dots[k]);
         }
 #pragma unroll
@@ -254,12 +272,15 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
 #pragma unroll
         for (int o = C::CPR; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(FULL_MASK, mb, o));
         const float m_new = fmaxf(m_own, mb);
-        const float alpha = fast_exp2(m_own - m_new);
+        // A slot can see no key of a chunk that starts past its row's limit (rows of one item have
+        // different limits): with m_new = -inf, subtract 0 so that alpha and p come out 0, not NaN.
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = fast_exp2(m_own - m_use);
         float ps = 0.f;
         float* prow = p_s + (g_own * C::TPP + sub) * C::PASSES;
 #pragma unroll
         for (int k = 0; k < C::NOWN; ++k) {
-            const float p = fast_exp2(dots[k] - m_new);
+            const float p = fast_exp2(dots[k] - m_use);
             ps += p;
             prow[i_own0 + k] = p;
         }
@@ -335,8 +356,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
             if (sub == 0) {
 #pragma unroll
                 for (int g = 0; g < GP; ++g) {
-                    if (g < nh) {
-                        const size_t qh = (size_t)ci.row * a.num_q_heads + (size_t)ci.kv_head * a.group + ci.head0 + g;
+                    if (g < ns) {
+                        const int jr = g / nh;
+                        const size_t qh = (size_t)(ci.row + jr) * a.num_q_heads + (size_t)ci.kv_head * a.group +
+                                          ci.head0 + (g - jr * nh);
                         if (ci.partial < 0) {
                             const float inv = 1.f / ml_s[2 * g + 1];
                             float o[C::EPC];
@@ -373,18 +396,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
     }
 }
 
-// One warp per (merge row, head): out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
+// One warp per (merge row, slot): out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
     constexpr int PER = D / 32;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    const int entry = gw / a.heads_per_entry;
-    const int g = gw % a.heads_per_entry;
+    const int entry = gw / a.slots_per_entry;
+    const int g = gw % a.slots_per_entry;
     griddep_wait();
     if (entry >= a.num_rows) return;
     const MergeRow mr = a.rows[entry];
-    if (g >= mr.num_heads) return;
+    if (g >= mr.num_slots) return;
     float M = -INFINITY;
     for (int i = 0; i < mr.count; ++i)
         M = fmaxf(M, a.part_ml[((size_t)(mr.first_partial + i) * kMaxGroupPerItem + g) * 2]);
@@ -401,7 +424,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
         for (int e = 0; e < PER; ++e) o[e] = fmaf(w, po[e], o[e]);
     }
     const float inv = 1.f / L;
-    T* out = static_cast<T*>(a.out) + ((size_t)mr.row * a.num_q_heads + mr.q_head0 + g) * D + lane * PER;
+    const int jr = g / mr.heads_per_row;
+    T* out = static_cast<T*>(a.out) +
+             ((size_t)(mr.row + jr) * a.num_q_heads + mr.q_head0 + (g - jr * mr.heads_per_row)) * D + lane * PER;
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
         if constexpr (sizeof(T) == 4) out[e] = o[e] * inv;
@@ -456,7 +481,7 @@ cudaError_t launch_decode_s(const DecodeArgs& a, int num_sms, cudaStream_t s) {
 
 template <typename T, int D>
 cudaError_t launch_decode_g(const DecodeArgs& a, int num_sms, cudaStream_t s) {
-    const int g = a.heads_per_item;
+    const int g = a.slots_per_item;
     if (g <= 1) return launch_decode_s<T, D, 1>(a, num_sms, s);
     if (g <= 2) return launch_decode_s<T, D, 2>(a, num_sms, s);
     if (g <= 4) return launch_decode_s<T, D, 4>(a, num_sms, s);
@@ -471,7 +496,7 @@ cudaError_t launch_decode_d(int head_dim, const DecodeArgs& a, int num_sms, cuda
 
 template <typename T>
 cudaError_t launch_merge_d(int head_dim, const MergeArgs& a, cudaStream_t s) {
-    const long long warps = (long long)a.num_rows * a.heads_per_entry;
+    const long long warps = (long long)a.num_rows * a.slots_per_entry;
     const int grid = (int)((warps * 32 + 127) / 128);
     if (grid < 1) return cudaSuccess;
     if (head_dim == 64) return launch_pdl(merge_kernel<T, 64>, dim3(grid), dim3(128), 0, s, a);

@@ -16,17 +16,20 @@ struct DeviceError {
     long long detail;
 };
 
-// One unit of CUDA-core work: a query row, a KV head, up to 8 query heads of its group and a
-// contiguous range of the row's KV blocks.
+// One unit of CUDA-core work: num_rows consecutive query rows of one request, a KV head, up to 8
+// query heads of its group and a contiguous range of the request's KV blocks. The item's
+// (row, head) pairs -- num_rows x heads, at most 8 -- share every K/V block it streams; row
+// row + j sees keys at positions < limit + j.
 struct DecodeItem {
-    int32_t row;        // query row (index into q/out)
+    int32_t row;        // first query row (index into q/out)
     int32_t req;        // request (row of the block table)
-    int32_t kv_head;
+    int16_t kv_head;
+    int16_t num_rows;   // consecutive query rows served (>= 1)
     int32_t head0;      // first query head of the group served here (offset inside the group)
     int32_t blk_begin;  // KV block range [blk_begin, blk_end) of the request
     int32_t blk_end;
-    int32_t limit;      // the row sees keys at positions < limit
-    int32_t partial;    // partial-result slot, or -1 when the item covers the whole row
+    int32_t limit;      // the first row sees keys at positions < limit
+    int32_t partial;    // partial-result slot, or -1 when the item covers whole rows
 };
 static_assert(sizeof(DecodeItem) == 32, "DecodeItem layout");
 
@@ -39,14 +42,16 @@ struct PrefillTile {
 };
 static_assert(sizeof(PrefillTile) == 16, "PrefillTile layout");
 
-// A (row, query-head range) whose chunks the log-sum-exp merge combines.
+// The (row, head) slots of one chunked item whose partials the log-sum-exp merge combines:
+// slot s is query row row + s / heads_per_row, query head q_head0 + s % heads_per_row.
 struct MergeRow {
     int32_t row;
     int32_t q_head0;       // first query head
-    int32_t num_heads;     // heads in this entry (<= 8)
+    int32_t num_slots;     // (row, head) slots in this entry (<= 8)
     int32_t first_partial; // partial slots first_partial .. first_partial + count - 1
     int32_t count;
-    int32_t pad[3];
+    int32_t heads_per_row;
+    int32_t pad[2];
 };
 static_assert(sizeof(MergeRow) == 32, "MergeRow layout");
 
@@ -67,6 +72,7 @@ struct DecodeArgs {
     int num_kv_heads;
     int group;           // Hq / Hkv
     int heads_per_item;  // query heads one item serves (<= 8)
+    int slots_per_item;  // largest num_rows x heads of any item (<= 8): selects the kernel variant
     float scale_log2;    // scale * log2(e)
 };
 
@@ -77,7 +83,7 @@ struct MergeArgs {
     const float* part_ml;
     int num_rows;
     int num_q_heads;
-    int heads_per_entry;  // heads per merge row (the plan's heads per item): warps launched per row
+    int slots_per_entry;  // largest num_slots of any merge row: warps launched per row
 };
 
 struct PrefillArgs {

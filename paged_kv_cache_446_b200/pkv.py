@@ -37,16 +37,17 @@ _SZ = ctypes.c_size_t
 
 class PlanOptions(ctypes.Structure):
     _fields_ = [("split_blocks", ctypes.c_int32), ("no_split", ctypes.c_int32),
-                ("cuda_core_only", ctypes.c_int32), ("num_sms", ctypes.c_int32), ("heads_per_item", ctypes.c_int32)]
+                ("cuda_core_only", ctypes.c_int32), ("num_sms", ctypes.c_int32), ("heads_per_item", ctypes.c_int32),
+                ("rows_per_item", ctypes.c_int32), ("tc_min_rows", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):
     _fields_ = [("magic", ctypes.c_uint32)] + [(n, ctypes.c_int32) for n in (
         "num_reqs", "num_q_tokens", "num_q_heads", "num_kv_heads", "head_dim", "dtype", "num_decode_rows",
         "num_prefill_rows", "num_items", "num_tiles", "num_merge_rows", "num_partials", "split_blocks",
-        "max_blocks", "heads_per_item", "reserved")] + [(n, ctypes.c_int64) for n in (
+        "max_blocks", "heads_per_item", "rows_per_item")] + [(n, ctypes.c_int64) for n in (
         "off_items", "off_tiles", "off_merge", "off_part_o", "off_part_ml", "meta_bytes", "ws_bytes", "kv_bytes",
-        "attn_flops")]
+        "attn_flops", "core_kv_bytes", "tile_kv_bytes", "tile_flops")]
 
 
 def _sig(name, restype, argtypes):
@@ -116,9 +117,10 @@ def _dtype_code(t: torch.Tensor) -> int:
     return DTYPE[t.dtype]
 
 
-def _opts(split_blocks=0, no_split=False, cuda_core_only=False, num_sms=0, heads_per_item=0) -> PlanOptions:
+def _opts(split_blocks=0, no_split=False, cuda_core_only=False, num_sms=0, heads_per_item=0, rows_per_item=0,
+          tc_min_rows=0) -> PlanOptions:
     return PlanOptions(int(split_blocks), int(bool(no_split)), int(bool(cuda_core_only)), int(num_sms),
-                       int(heads_per_item))
+                       int(heads_per_item), int(rows_per_item), int(tc_min_rows))
 
 
 # ---- a13: mixed-batch flattening -------------------------------------------------------------
@@ -293,12 +295,14 @@ def profile_stop() -> dict:
 class BmStats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "num_blocks", "free_blocks", "used_blocks", "shared_blocks", "num_sequences", "logical_tokens",
-        "stored_tokens", "wasted_slots", "cow_copies")]
+        "stored_tokens", "wasted_slots", "cow_copies", "cached_blocks", "cache_queries", "cache_hits")]
 
 
 _BM = ctypes.c_void_p
 _I32P = ctypes.POINTER(ctypes.c_int32)
-_bm_create = _sig("pkv_bm_create", _I, [_I, _I, ctypes.POINTER(_BM)])
+_bm_create = _sig("pkv_bm_create_ex", _I, [_I, _I, _I, ctypes.POINTER(_BM)])
+_bm_add_cached = _sig("pkv_bm_add_cached_prefix", _I, [_BM, _I64, _P, _I64, ctypes.POINTER(_I64)])
+_bm_append_tokens = _sig("pkv_bm_append_tokens", _I, [_BM, _I64, _P, _I64, _I32P])
 _bm_destroy = _sig("pkv_bm_destroy", None, [_BM])
 _bm_add = _sig("pkv_bm_add_sequence", _I, [_BM, _I64, _I64])
 _bm_fork = _sig("pkv_bm_fork", _I, [_BM, _I64, _I64])
@@ -308,16 +312,19 @@ _bm_sequence = _sig("pkv_bm_sequence", _I, [_BM, _I64, ctypes.POINTER(_I64), _P,
 _bm_tables = _sig("pkv_bm_block_tables", _I, [_BM, _P, _I, _P, _I])
 _bm_refcount = _sig("pkv_bm_refcount", _I, [_BM, ctypes.c_int32, _I32P])
 _bm_stats = _sig("pkv_bm_stats", _I, [_BM, ctypes.POINTER(BmStats)])
-_bm_step = _sig("pkv_bm_step", _I, [_BM, _P, _P, _I, _P, _I, _P, _P, _P, ctypes.POINTER(_I)])
+_bm_step = _sig("pkv_bm_step", _I, [_BM, _P, _P, _I, _P, _P, _I, _P, _P, _P, ctypes.POINTER(_I)])
+PKV_BM_PREFIX_CACHE = 1
 
 
 class BlockManager:
     """Allocation state of one block pool (pkv_bm_* in include/pkv.h): on-demand blocks,
-    reference-counted sharing between forked sequences and copy-on-write of shared last blocks."""
+    reference-counted sharing between forked sequences, copy-on-write of shared last blocks and,
+    with prefix_cache=True, reuse of cached full blocks for prompts that begin alike."""
 
-    def __init__(self, num_blocks: int, block_size: int = 16):
+    def __init__(self, num_blocks: int, block_size: int = 16, prefix_cache: bool = False):
         h = _BM()
-        _check(_bm_create(int(num_blocks), int(block_size), ctypes.byref(h)), "pkv_bm_create")
+        _check(_bm_create(int(num_blocks), int(block_size), PKV_BM_PREFIX_CACHE if prefix_cache else 0,
+                          ctypes.byref(h)), "pkv_bm_create_ex")
         self._h = h
         self.num_blocks = int(num_blocks)
         self.block_size = int(block_size)
@@ -333,10 +340,25 @@ class BlockManager:
     def fork(self, parent: int, child: int) -> None:
         _check(_bm_fork(self._h, int(parent), int(child)), "pkv_bm_fork")
 
-    def append(self, seq_id: int, num_tokens: int) -> tuple[int, int] | None:
-        """Returns the (src, dst) copy the append needs, or None."""
+    def add_cached_prefix(self, seq_id: int, tokens) -> int:
+        """Starts a token-tracked sequence from the longest cached prefix of `tokens`; returns how
+        many leading tokens are cached (the rest are appended, with their ids, by the caller)."""
+        ids = np.ascontiguousarray(tokens, dtype=np.int32)
+        cached = _I64(0)
+        _check(_bm_add_cached(self._h, int(seq_id), _np_ptr(ids), ids.shape[0], ctypes.byref(cached)),
+               "pkv_bm_add_cached_prefix")
+        return cached.value
+
+    def append(self, seq_id: int, num_tokens: int, tokens=None) -> tuple[int, int] | None:
+        """Returns the (src, dst) copy the append needs, or None. `tokens`: the new tokens' ids."""
         pair = (ctypes.c_int32 * 2)()
-        _check(_bm_append(self._h, int(seq_id), int(num_tokens), pair), "pkv_bm_append")
+        if tokens is None:
+            _check(_bm_append(self._h, int(seq_id), int(num_tokens), pair), "pkv_bm_append")
+        else:
+            ids = np.ascontiguousarray(tokens, dtype=np.int32)
+            if ids.shape[0] != int(num_tokens):
+                raise ValueError("len(tokens) != num_tokens")
+            _check(_bm_append_tokens(self._h, int(seq_id), _np_ptr(ids), int(num_tokens), pair), "pkv_bm_append_tokens")
         return None if pair[0] < 0 else (pair[0], pair[1])
 
     def free(self, seq_id: int) -> None:
@@ -369,18 +391,24 @@ class BlockManager:
         _check(_bm_stats(self._h, ctypes.byref(st)), "pkv_bm_stats")
         return {n: getattr(st, n) for n, _ in BmStats._fields_}
 
-    def step(self, batch: dict, max_blocks_per_seq: int):
+    def step(self, batch: dict, max_blocks_per_seq: int, new_tokens=None):
         """Appends batch {seq_id: num_new_tokens} (dict order) and returns the step's host inputs:
         (block_tables int32 [R, max_blocks_per_seq], context_lens int32 [R], query_start_loc int32 [R+1],
-        copy pairs int32 [P, 2])."""
+        copy pairs int32 [P, 2]). new_tokens: the new tokens' ids concatenated in batch order."""
         ids = np.fromiter(batch.keys(), np.int64, len(batch))
         n = np.fromiter(batch.values(), np.int32, len(batch))
+        tok = None
+        if new_tokens is not None:
+            tok = np.ascontiguousarray(new_tokens, dtype=np.int32)
+            if tok.shape[0] != int(n.sum()):
+                raise ValueError("new_tokens must hold sum(batch.values()) ids")
         R = ids.shape[0]
         tables = np.empty((R, int(max_blocks_per_seq)), np.int32)
         ctx = np.empty(R, np.int32)
         qsl = np.empty(R + 1, np.int32)
         pairs = np.empty((max(R, 1), 2), np.int32)
         npairs = _I(0)
-        _check(_bm_step(self._h, _np_ptr(ids), _np_ptr(n), R, _np_ptr(tables), int(max_blocks_per_seq), _np_ptr(ctx),
-                        _np_ptr(qsl), _np_ptr(pairs), ctypes.byref(npairs)), "pkv_bm_step")
+        _check(_bm_step(self._h, _np_ptr(ids), _np_ptr(n), R, None if tok is None else _np_ptr(tok), _np_ptr(tables),
+                        int(max_blocks_per_seq), _np_ptr(ctx), _np_ptr(qsl), _np_ptr(pairs), ctypes.byref(npairs)),
+               "pkv_bm_step")
         return tables, ctx, qsl, pairs[:npairs.value].copy()

@@ -1,4 +1,4 @@
-"""Seeded synthetic workloads for the five measured configurations.
+"""Seeded synthetic workloads for the measured configurations.
 
 This module only draws inputs: request lengths, block-table contents (physical block ids taken from
 a seeded permutation of the pool), copy-on-write pairs and the random q/k/v values. It performs none
@@ -20,6 +20,9 @@ families the pages mention -- LLaMA-13B in blog.mckayzhao.com/?p=56 "æ•…äº‹è¦ä»
   c5  70B-shaped bf16 mixed batch: 4 chunked-prefill requests of 512 rows at prior context
       {0,4096,16384,32768} followed by 128 decode rows with context U[256,16384]; every scheduled
       token is appended before attention
+  c6  speculative verify, LLaMA-13B-shaped fp16: 32 requests each submitting k = 4 draft tokens plus
+      one as k+1 = 5 query rows ({request_id: 5}, ä¸€æ–‡æžæ‡‚vLLMï¼šä¸ºå•¥å®ƒèƒ½è®©ä¸€å¼ GPUæ‰›ä½å‡ åå€ç”¨æˆ·ï¼Ÿ,
+      "V1 æž¶æž„ï¼šæŽ¨å€’é‡æ¥çš„å‹‡æ°”"), prior context U[512,4096]; the 5 new K/V rows are appended first
 
 `small=True` keeps each configuration's dtype, heads, head_dim and row mix but shrinks the number of
 requests and the lengths so the CPU oracle checks every output in seconds.
@@ -34,7 +37,7 @@ import torch
 
 BLOCK_SIZE = 16
 TORCH_DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
-CONFIGS = ("c1", "c2", "c3", "c4", "c5")
+CONFIGS = ("c1", "c2", "c3", "c4", "c5", "c6")
 
 
 @dataclass
@@ -109,7 +112,7 @@ def _tables_from_permutation(rng, lens_blocks: list[int], num_blocks: int) -> np
 
 def make(config: str, device: str | torch.device = "cpu", small: bool = False, seed: int | None = None,
          with_tensors: bool = True, part: str = "all", max_requests: int = 0) -> Workload:
-    """Build configuration `config` ("c1".."c5"); seed defaults to 1000 + the configuration number.
+    """Build configuration `config` ("c1".."c6"); seed defaults to 1000 + the configuration number.
 
     part="prefill" / "decode" keeps only the requests with more than one / exactly one row this
     step (their tables are relabelled onto a pool sized 1.2x their blocks, keeping the seeded
@@ -120,7 +123,7 @@ def make(config: str, device: str | torch.device = "cpu", small: bool = False, s
         raise ValueError(f"unknown configuration {config!r}")
     seed = 1000 + int(config[1]) if seed is None else int(seed)
     rng = np.random.default_rng(seed)
-    builder = {"c1": _c1, "c2": _c2, "c3": _c3, "c4": _c4, "c5": _c5}[config]
+    builder = {"c1": _c1, "c2": _c2, "c3": _c3, "c4": _c4, "c5": _c5, "c6": _c6}[config]
     wl = builder(rng, small)
     wl.seed = seed
     if part != "all" or max_requests > 0:
@@ -268,4 +271,20 @@ def _c5(rng, small):
                   prior_lens=(ctx - n).astype(np.int32), block_tables=bt, num_blocks=num_blocks,
                   write_batch=dict(batch), copy_pairs=np.zeros((0, 2), np.int32))
     wl.notes.update(prefill_priors=priors, chunk=chunk)
+    return wl
+
+
+def _c6(rng, small):
+    R, lo, hi, rows = (6, 17, 300, 5) if small else (32, 512, 4096, 5)
+    prior = rng.integers(lo, hi + 1, size=R).astype(np.int64)
+    ctx = prior + rows
+    need = [int(x) for x in _nblocks(ctx)]
+    num_blocks = int(math.ceil(1.2 * sum(need)))
+    bt = _tables_from_permutation(rng, need, num_blocks)
+    batch = {r: rows for r in range(R)}
+    wl = Workload(name="c6" + ("-small" if small else ""), dtype="f16", num_q_heads=40, num_kv_heads=40,
+                  head_dim=128, scale=float(np.float32(1.0 / math.sqrt(128))), batch=batch,
+                  prior_lens=prior.astype(np.int32), block_tables=bt, num_blocks=num_blocks,
+                  write_batch=dict(batch), copy_pairs=np.zeros((0, 2), np.int32))
+    wl.notes.update(draft_tokens=rows - 1)
     return wl

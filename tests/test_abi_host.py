@@ -103,12 +103,15 @@ def parse_meta(plan, meta):
 
 @pytest.mark.parametrize("seed", range(6))
 @pytest.mark.parametrize("opts", [{}, {"split_blocks": 1}, {"split_blocks": 3}, {"no_split": True},
-                                  {"cuda_core_only": True}, {"heads_per_item": 4}, {"heads_per_item": 3}])
+                                  {"cuda_core_only": True}, {"heads_per_item": 4}, {"heads_per_item": 3},
+                                  {"cuda_core_only": True, "split_blocks": 2}, {"tc_min_rows": 9},
+                                  {"cuda_core_only": True, "rows_per_item": 1},
+                                  {"cuda_core_only": True, "rows_per_item": 3, "heads_per_item": 2}])
 def test_planner_covers_every_block_once(pkv, seed, opts):
     """Every (row, query head, visible KV block) is covered by exactly one work item or tile."""
     rng = np.random.default_rng(seed)
     R = int(rng.integers(1, 12))
-    n = rng.choice([0, 1, 1, 1, 5, 37, 130], size=R)
+    n = rng.choice([0, 1, 1, 1, 2, 4, 5, 8, 37, 130], size=R)
     prior = rng.integers(0, 300, size=R)
     ctx = (prior + n).astype(np.int32)
     ctx[(n == 0) & (rng.random(R) < 0.5)] = 0
@@ -118,19 +121,31 @@ def test_planner_covers_every_block_once(pkv, seed, opts):
     plan, meta = pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, **opts)
     items, tiles, merges = parse_meta(plan, meta)
     G = Hq // Hkv
+    hpi = plan.heads_per_item
     cover = {}
-    for row, req, kvh, head0, b0, b1, limit, part in items:
-        assert qsl[req] <= row < qsl[req + 1]
+    max_rows = 0
+    for row, req, packed, head0, b0, b1, limit, part in items:
+        kvh, nrows = packed & 0xFFFF, packed >> 16
+        assert 1 <= nrows and nrows * min(hpi, G - head0) <= 8
+        max_rows = max(max_rows, nrows)
+        nreq = qsl[req + 1] - qsl[req]
+        assert qsl[req] <= row and row + nrows <= qsl[req + 1]
         j = row - qsl[req]
-        assert limit == ctx[req] - (qsl[req + 1] - qsl[req]) + j + 1
-        assert 0 <= b0 < b1 <= -(-limit // 16)
-        for h in range(head0, min(G, head0 + plan.heads_per_item)):
-            for b in range(b0, b1):
-                key = (row, kvh * G + h, b)
-                cover[key] = cover.get(key, 0) + 1
+        assert limit == ctx[req] - nreq + j + 1
+        assert 0 <= b0 < b1 <= -(-(limit + nrows - 1) // 16)
+        for jr in range(nrows):
+            visible = -(-(limit + jr) // 16)
+            for h in range(head0, min(G, head0 + hpi)):
+                for b in range(b0, min(b1, visible)):
+                    key = (row + jr, kvh * G + h, b)
+                    cover[key] = cover.get(key, 0) + 1
+    assert plan.rows_per_item == max_rows
+    if "rows_per_item" in opts:
+        assert max_rows <= opts["rows_per_item"]
     tile_rows = 2 * (128 // G)      # two 128-row MMA tiles per CTA
     for req, kvh, tok0, _ in tiles:
         nreq = qsl[req + 1] - qsl[req]
+        assert nreq >= max(2, opts.get("tc_min_rows", 2))
         for j in range(tok0, min(nreq, tok0 + tile_rows)):
             limit = ctx[req] - nreq + j + 1
             for h in range(G):
@@ -148,14 +163,16 @@ def test_planner_covers_every_block_once(pkv, seed, opts):
     assert cover == expect
     # Partials: every partial slot belongs to exactly one merge row, and chunked items point into it.
     owners = {}
-    for row, qh0, nh, first, count, *_ in merges:
+    for row, qh0, nslots, first, count, hpr, *_ in merges:
         for p in range(first, first + count):
             assert p not in owners
-            owners[p] = (row, qh0, nh)
+            owners[p] = (row, qh0, nslots, hpr)
     assert len(owners) == plan.num_partials
-    for row, req, kvh, head0, b0, b1, limit, part in items:
+    for row, req, packed, head0, b0, b1, limit, part in items:
+        kvh, nrows = packed & 0xFFFF, packed >> 16
         if part >= 0:
-            assert owners[part] == (row, kvh * G + head0, min(plan.heads_per_item, G - head0))
+            nh = min(hpi, G - head0)
+            assert owners[part] == (row, kvh * G + head0, nh * nrows, nh)
     if opts.get("no_split"):
         assert plan.num_merge_rows == 0
 

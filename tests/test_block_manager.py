@@ -10,7 +10,8 @@ import pytest
 
 from oracle.block_pool import OutOfBlocks
 from paged_kv_cache_446_b200 import build as pkv_build
-from pool_harness import ContentCheck, OracleAdapter, ProductAdapter, random_script, run_script
+from pool_harness import (ContentCheck, OracleAdapter, PrefixContentCheck, ProductAdapter, random_cache_script,
+                          random_script, run_cache_script, run_script)
 
 
 @pytest.fixture(scope="module")
@@ -35,9 +36,9 @@ def block_mapping(prod, orac, live):
 class Lockstep:
     """Applies each op to product and oracle; both must succeed or both run out of blocks."""
 
-    def __init__(self, num_blocks):
-        self.p = ProductAdapter(num_blocks)
-        self.o = OracleAdapter(num_blocks)
+    def __init__(self, num_blocks, prefix_cache=False):
+        self.p = ProductAdapter(num_blocks, prefix_cache=prefix_cache)
+        self.o = OracleAdapter(num_blocks, prefix_cache=prefix_cache)
         self.last = None
 
     def _both(self, name, *a):
@@ -59,11 +60,14 @@ class Lockstep:
     def fork(self, p, c):
         return self._both("fork", p, c)
 
-    def append(self, s, n):
-        return self._both("append", s, n)
+    def append(self, s, n, tokens=None):
+        return self._both("append", s, n, tokens)
 
-    def step(self, batch):
-        return self._both("step", batch)
+    def step(self, batch, tokens=None):
+        return self._both("step", batch, tokens)
+
+    def prompt(self, s, tokens):
+        return self._both("prompt", s, tokens)
 
     def free(self, s):
         return self._both("free", s)
@@ -116,19 +120,19 @@ def test_contents_read_back(pkv, seed):
 
 
 def test_documented_allocation_order(pkv):
-    """A new pool hands out 0, 1, 2, ...; released blocks are reused most recent first; a sequence
-    releases its blocks last to first."""
-    m = pkv.BlockManager(8)
+    """A new pool hands out 0, 1, 2, ...; released blocks join the back of the free queue, so the
+    least recently released block is reused first; a sequence releases its blocks last to first."""
+    m = pkv.BlockManager(6)
     m.add(1, 40)
     assert m.sequence(1) == (40, [0, 1, 2])
     m.add(2, 1)
     assert m.sequence(2) == (1, [3])
-    m.free(1)                                # pushes 2, 1, 0: block 0 is on top
-    m.add(3, 17)
-    assert m.sequence(3) == (17, [0, 1])
-    m.free(2)
+    m.free(1)                                # queue: 4 5 2 1 0
+    m.add(3, 40)
+    assert m.sequence(3) == (40, [4, 5, 2])
+    m.free(2)                                # queue: 1 0 3
     assert m.append(3, 16) is None
-    assert m.sequence(3) == (33, [0, 1, 3])
+    assert m.sequence(3) == (56, [4, 5, 2, 1])
 
 
 def test_errors_change_nothing(pkv):
@@ -167,7 +171,7 @@ def test_errors_change_nothing(pkv):
     qsl = np.empty(3, np.int32)
     pairs = np.empty((2, 2), np.int32)
     cnt = ctypes.c_int(0)
-    assert pkv._bm_step(m._h, pkv._np_ptr(ids), pkv._np_ptr(n), 2, pkv._np_ptr(tables), 8, pkv._np_ptr(ctx),
+    assert pkv._bm_step(m._h, pkv._np_ptr(ids), pkv._np_ptr(n), 2, None, pkv._np_ptr(tables), 8, pkv._np_ptr(ctx),
                         pkv._np_ptr(qsl), pkv._np_ptr(pairs), ctypes.byref(cnt)) == 1
     assert (m.sequence(1), m.sequence(2), m.stats()) == snap
     with pytest.raises(pkv.PkvError):
@@ -235,3 +239,64 @@ def test_waste_statistics_on_workload_mixes(pkv):
         assert st["stored_tokens"] == int(lens.sum())
         assert st["wasted_slots"] <= 15 * len(lens)
         assert st["wasted_slots"] / (16 * st["used_blocks"]) < 0.04
+
+
+@pytest.mark.parametrize("seed,num_blocks", [(30, 24), (31, 40), (32, 64), (33, 200)])
+def test_prefix_cache_matches_oracle(pkv, seed, num_blocks):
+    """Prefix-caching managers follow the same documented allocation order as the oracle's plain
+    model, so block ids, cached-token counts, copies, tables and statistics must be identical."""
+    ls = Lockstep(num_blocks, prefix_cache=True)
+    live = set()
+
+    def after(i, op, res):
+        kind = op[0]
+        if res[0] == "ok":
+            if kind == "prompt":
+                live.add(op[1])
+            elif kind == "fork":
+                live.add(op[2])
+            elif kind == "free":
+                live.discard(op[1])
+        for s in live:
+            assert ls.p.table(s) == ls.o.table(s) and ls.p.length(s) == ls.o.length(s)
+        for b in range(num_blocks):
+            assert ls.p.holders(b) == ls.o.holders(b)
+        assert ls.p.stats() == ls.o.stats()
+        if res[0] == "ok" and kind in ("prompt", "append", "step"):
+            _, rp, ro = ls.last
+            assert rp == ro
+
+    outcomes = run_cache_script(ls, random_cache_script(seed, num_ops=250), after)
+    st = ls.p.stats()
+    assert st["cache_hits"] > 0
+    if num_blocks <= 40:
+        assert "out_of_blocks" in {r[0] for r in outcomes}
+
+
+@pytest.mark.parametrize("seed", [40, 41])
+def test_prefix_cache_contents_read_back(pkv, seed):
+    mgr = ProductAdapter(48, prefix_cache=True)
+    cc = PrefixContentCheck(mgr, 48)
+    run_cache_script(cc, random_cache_script(seed, num_ops=300), lambda i, op, res: cc.check())
+    assert cc.cached_tokens > 0
+
+
+def test_prefix_cache_api(pkv):
+    m = pkv.BlockManager(32, prefix_cache=True)
+    system = list(range(50, 150))
+    assert m.add_cached_prefix(1, system + [1]) == 0       # one lookup, a miss
+    m.append(1, 101, system + [1])
+    assert m.add_cached_prefix(2, system + [2, 3]) == 96
+    tables, ctx, qsl, pairs = m.step({2: 6}, 8, system[96:] + [2, 3])
+    assert ctx.tolist() == [102] and qsl.tolist() == [0, 6]
+    assert tables[0, :6].tolist() == m.sequence(1)[1][:6]
+    st = m.stats()
+    assert st["cache_hits"] == 6 and st["cache_queries"] == 7 and st["cached_blocks"] == 6
+    # Without a prefix cache nothing is looked up; without ids, appends stop tracking.
+    n = pkv.BlockManager(8)
+    assert n.add_cached_prefix(1, list(range(40))) == 0
+    assert n.sequence(1) == (0, [])
+    with pytest.raises(ValueError):
+        m.append(2, 2, [1])
+    with pytest.raises(pkv.PkvError):
+        m.add_cached_prefix(2, [1, 2])                         # id already live

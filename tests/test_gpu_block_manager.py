@@ -108,3 +108,71 @@ def test_manager_driven_serving_run(dtype_name, Hq, Hkv):
     st = mgr.stats()
     assert steps == 7 and copies >= 9 and st["cow_copies"] == copies
     assert st["wasted_slots"] < 16 * st["used_blocks"]
+
+
+@pytest.mark.parametrize("dtype_name,Hq,Hkv", [("f16", 32, 8), ("bf16", 64, 8)])
+def test_prefix_cached_serving_run(dtype_name, Hq, Hkv):
+    """Requests that share system prompts, with a prefix-caching manager: a new request computes
+    only the prompt tokens past its cached blocks (its rows attend the cached blocks written by
+    earlier requests), next to decode rows of running requests; finished conversations come back
+    with a new message. Each step is compared with the oracle (outputs and whole pools)."""
+    from paged_kv_cache_446_b200 import pkv
+    from paged_kv_cache_446_b200 import workloads as W
+    from paged_kv_cache_446_b200.step import PagedAttentionStep
+
+    dev = torch.device("cuda:0")
+    dtype = W.TORCH_DTYPES[dtype_name]
+    D, NB, width = 128, 96, 24
+    scale = float(np.float32(1.0 / math.sqrt(D)))
+    gen = torch.Generator().manual_seed(9)
+    rng = np.random.default_rng(9)
+    mgr = pkv.BlockManager(NB, prefix_cache=True)
+    k_pool = _rand((NB, Hkv, 16, D), dtype, gen).to(dev)
+    v_pool = _rand((NB, Hkv, 16, D), dtype, gen).to(dev)
+    h = {"k_pool": storage(k_pool), "v_pool": storage(v_pool)}
+    systems = [list(range(1000, 1000 + 70)), list(range(2000, 2000 + 33))]
+    ids, live, finished = {}, [], []
+    cached_total = 0
+    for step_no in range(8):
+        batch, toks = {}, []
+        for s in live:                                   # decode rows of running requests
+            t = [int(rng.integers(0, 30000))]
+            batch[s] = 1
+            toks += t
+            ids[s] += t
+        for k in range(2):                               # two new requests per step
+            s = 100 * step_no + k
+            if finished and rng.random() < 0.5:
+                prompt = finished.pop(0) + [int(x) for x in rng.integers(0, 30000, size=9)]
+            else:
+                prompt = systems[int(rng.integers(2))] + [int(x) for x in rng.integers(0, 30000, size=int(rng.integers(1, 20)))]
+            cached = mgr.add_cached_prefix(s, prompt)
+            cached_total += cached
+            batch[s] = len(prompt) - cached
+            toks += prompt[cached:]
+            ids[s] = list(prompt)
+            live.append(s)
+        tables, ctx, qsl, pairs = mgr.step(batch, width, toks)
+        counts = np.asarray(list(batch.values()), np.int64)
+        prior = (ctx - counts).astype(np.int32)
+        T = int(qsl[-1])
+        q = _rand((T, Hq, D), dtype, gen)
+        k_new = _rand((T, Hkv, D), dtype, gen)
+        v_new = _rand((T, Hkv, D), dtype, gen)
+        wl = SimpleNamespace(copy_pairs=pairs, write_batch=dict(batch), batch=batch, prior_lens=prior,
+                             block_tables=tables, scale=scale, dtype=dtype_name)
+        h.update(q=storage(q), k_new=storage(k_new), v_new=storage(v_new))
+        ref = oracle_step(wl, h)
+        step = PagedAttentionStep(batch, prior, tables, NB, Hq, Hkv, D, dtype, dev, write_batch=dict(batch),
+                                  copy_pairs=pairs)
+        out = step.run(q.to(dev), k_pool, v_pool, scale, k_new.to(dev), v_new.to(dev))
+        torch.cuda.synchronize()
+        assert pkv.device_error() == (0, -1)
+        err = max_err(out, ref)
+        assert err <= TOL[dtype_name], f"step {step_no}: max |err| {err}"
+        assert np.array_equal(storage(k_pool), h["k_pool"]) and np.array_equal(storage(v_pool), h["v_pool"])
+        while len(live) > 4:                             # the oldest requests finish
+            s = live.pop(0)
+            finished.append(ids.pop(s))
+            mgr.free(s)
+    assert cached_total > 0 and mgr.stats()["cache_hits"] > 0

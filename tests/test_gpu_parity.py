@@ -245,3 +245,31 @@ def test_heads_per_item(dev, hpi):
     same result."""
     wl = W.make("c5", device=dev, small=True)
     run_and_compare(wl, dev, heads_per_item=hpi, cuda_core_only=True)
+
+
+# Speculative verify steps: each request submits k draft tokens plus one as k+1 query rows.
+VERIFY_CASES = [
+    ("f16", 40, 40, 128, [(700, 5), (33, 5), (1500, 5), (15, 2)]),   # G = 1: 5 rows per item
+    ("bf16", 32, 8, 128, [(900, 4), (63, 3), (2000, 8), (5, 1)]),    # G = 4: 2 rows per item
+    ("f16", 16, 8, 128, [(31, 4), (32, 4), (47, 8), (400, 6)]),      # G = 2: 4 rows per item
+    ("bf16", 64, 8, 128, [(1200, 4), (16, 2)]),                      # G = 8: 1 row per item
+    ("f32", 8, 8, 128, [(300, 8), (17, 7), (0, 3)]),                 # fp32 (CUDA cores only)
+    ("f16", 16, 16, 64, [(250, 6), (9, 5)]),                         # head_dim 64
+]
+
+
+@pytest.mark.parametrize("opts", [{"tc_min_rows": 9}, {"tc_min_rows": 9, "split_blocks": 1},
+                                  {"tc_min_rows": 9, "split_blocks": 3}, {"cuda_core_only": True, "rows_per_item": 1},
+                                  {}], ids=["rows", "rows-split1", "rows-split3", "one-row", "default"])
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,specs", VERIFY_CASES)
+def test_verify_rows(dev, dtype, Hq, Hkv, D, specs, opts):
+    """Multi-token rows served by CUDA-core items that pack consecutive rows of a request (each
+    with its own causal limit) -- chunked so that some chunks lie wholly past the earlier rows'
+    limits -- one row per item, or the default routing, all against the oracle."""
+    wl = custom(dev, dtype, Hq, Hkv, D, specs, seed=21)
+    _, step = run_and_compare(wl, dev, **opts)
+    p = step.plan.plan
+    G = Hq // Hkv
+    if opts.get("tc_min_rows") and p.num_items:
+        assert p.rows_per_item == min(max(n for _, n in specs), max(1, 8 // min(G, 8)))
+

@@ -157,3 +157,119 @@ def test_out_of_blocks_changes_nothing():
     with pytest.raises(OutOfBlocks):
         mgr.step({0: 30})
     assert (mgr.table(0), mgr.stats()) == before
+
+
+# ---- prefix cache -------------------------------------------------------------------------------
+from oracle.block_pool import CACHE_MUTANTS  # noqa: E402
+from pool_harness import PrefixContentCheck, random_cache_script, run_cache_script  # noqa: E402
+
+
+def pin_prefix_cache_contents(mutant=None):
+    """Random serving scripts (shared system prompts, continued conversations, decode appends,
+    forks, frees, small pools that evict): every live sequence reads, at every position, the K/V
+    of its own prefix -- so every reused block held exactly the prefix it was reused for -- and
+    every count equals its holders. The cache must also have been used."""
+    hits = 0
+    for seed, num_blocks in [(0, 30), (1, 48), (2, 120), (3, 20)]:
+        mgr = OracleAdapter(num_blocks, 16, mutant, prefix_cache=True)
+        cc = PrefixContentCheck(mgr, num_blocks)
+
+        def after(i, op, res):
+            cc.check()
+            holders_match_tables(mgr, cc.ids)
+
+        run_cache_script(cc, random_cache_script(seed), after)
+        hits += cc.cached_tokens
+    assert hits > 0
+
+
+def pin_shared_system_prompt(mutant=None):
+    """Requests that begin with the same system prompt keep one copy of its blocks and every
+    table points at it (一文搞懂vLLM, "PagedAttention 是怎么共享内存的")."""
+    mgr = OracleAdapter(32, 16, mutant, prefix_cache=True)
+    cc = PrefixContentCheck(mgr, 32)
+    system = list(range(100, 200))                      # 100 tokens: 6 full blocks + 4
+    assert cc.prompt("A", system + [1, 2, 3]) == 0
+    assert cc.prompt("B", system + [7, 8]) == 96        # the 6 full blocks of the shared prefix
+    a, b = mgr.table("A"), mgr.table("B")
+    assert a[:6] == b[:6] and a[6] != b[6]
+    assert all(mgr.holders(x) == 2 for x in a[:6])
+    cc.check()
+
+
+def pin_multi_turn(mutant=None):
+    """In a multi-turn conversation only the newest message needs computing: every full block of
+    the history hits the cache, even after the earlier turn finished (blog.mckayzhao.com/?p=56,
+    "进阶特性：让推理再快一点"; vLLM 简介, "自动前缀缓存")."""
+    mgr = OracleAdapter(64, 16, mutant, prefix_cache=True)
+    cc = PrefixContentCheck(mgr, 64)
+    turn1 = list(range(1000, 1070))                     # 70-token first prompt
+    cc.prompt(1, turn1)
+    answer = list(range(2000, 2041))                    # 41 tokens generated one by one
+    for t in answer:
+        cc.append(1, 1, [t])
+    history = turn1 + answer                            # 111 tokens: 6 full blocks + 15
+    cc.free(1)
+    cached = cc.prompt(2, history + list(range(3000, 3012)))
+    assert cached == 16 * (len(history) // 16) == 96
+    cc.check()
+
+
+def pin_last_token_computed(mutant=None):
+    """A prompt wholly in the cache still computes its last token (its block is not reused)."""
+    mgr = OracleAdapter(16, 16, mutant, prefix_cache=True)
+    cc = PrefixContentCheck(mgr, 16)
+    ids = list(range(32))
+    cc.prompt("x", ids)
+    assert cc.prompt("y", ids) == 16
+    cc.check()
+
+
+def pin_cached_blocks_survive_until_taken(mutant=None):
+    """A finished request's blocks stay reusable until the pool needs them; blocks are taken
+    least recently released first and a request releases its last block first, so a longer
+    prompt loses its tail before its beginning."""
+    mgr = OracleAdapter(8, 16, mutant, prefix_cache=True)
+    cc = PrefixContentCheck(mgr, 8)
+    ids = list(range(64))                               # 4 full blocks
+    cc.prompt("a", ids + [999])                         # blocks 0-4
+    cc.free("a")                                        # free: 5 6 7 4 3 2 1 0
+    assert cc.prompt("b", ids + [5]) == 64              # reuses 0-3, takes 5
+    cc.free("b")                                        # free: 6 7 4 5 3 2 1 0
+    cc.prompt("filler", list(range(500, 565)))          # takes 6 7 4 5 3: the 4th prompt block goes
+    cc.free("filler")
+    assert cc.prompt("c", ids + [6]) == 48              # the first three prompt blocks survived
+    cc.check()
+
+
+def pin_whole_prefix_must_match(mutant=None):
+    """A block's K/V depend on every token before it, so a block is reused only for the same whole
+    prefix: equal tokens after a different beginning are computed again."""
+    mgr = OracleAdapter(16, 16, mutant, prefix_cache=True)
+    cc = PrefixContentCheck(mgr, 16)
+    x, y, z, w = (list(range(k, k + 16)) for k in (0, 100, 200, 300))
+    cc.prompt("a", x + w + [1])                         # caches x, then x+w
+    cc.prompt("b", z + y + [2])                         # caches z, then z+y
+    assert cc.prompt("c", x + y + [3]) == 16            # x hits; y's cached block follows z, not x
+    assert cc.prompt("d", x + y + [4]) == 32            # c has cached x+y by now
+    cc.check()
+
+
+CACHE_PINS = [pin_prefix_cache_contents, pin_shared_system_prompt, pin_multi_turn, pin_last_token_computed,
+              pin_cached_blocks_survive_until_taken, pin_whole_prefix_must_match]
+
+
+@pytest.mark.parametrize("pin", CACHE_PINS, ids=lambda p: p.__name__)
+def test_prefix_cache_pin(pin):
+    pin()
+
+
+@pytest.mark.parametrize("mutant", CACHE_MUTANTS)
+def test_prefix_cache_mutant_is_caught(mutant):
+    failed = []
+    for pin in CACHE_PINS:
+        try:
+            pin(mutant=mutant)
+        except Exception as e:  # an assertion or a model error both count as caught
+            failed.append((pin.__name__, type(e).__name__))
+    assert failed, f"no pin catches mutant {mutant}"
