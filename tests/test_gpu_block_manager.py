@@ -176,3 +176,69 @@ def test_prefix_cached_serving_run(dtype_name, Hq, Hkv):
             finished.append(ids.pop(s))
             mgr.free(s)
     assert cached_total > 0 and mgr.stats()["cache_hits"] > 0
+
+
+@pytest.mark.parametrize("dtype_name,Hq,Hkv", [("f16", 32, 8), ("bf16", 16, 16)])
+def test_beam_search_run(dtype_name, Hq, Hkv):
+    """Beam search over a paged cache (blog.mckayzhao.com/?p=56, "还不止是分页：Copy-on-Write 和内存
+    共享"): each step every beam forks candidates, the best (here: seeded random) keep going and the
+    rest are freed, so beams share ever deeper trees of blocks; a candidate writing into a shared
+    partial block gets a copy. Each step's decode rows and pools are compared with the oracle."""
+    from paged_kv_cache_446_b200 import pkv
+    from paged_kv_cache_446_b200 import workloads as W
+    from paged_kv_cache_446_b200.step import PagedAttentionStep
+
+    dev = torch.device("cuda:0")
+    dtype = W.TORCH_DTYPES[dtype_name]
+    D, NB, width, beams, fan = 128, 128, 16, 4, 3
+    scale = float(np.float32(1.0 / math.sqrt(D)))
+    gen = torch.Generator().manual_seed(13)
+    rng = np.random.default_rng(13)
+    mgr = pkv.BlockManager(NB)
+    k_pool = _rand((NB, Hkv, 16, D), dtype, gen).to(dev)
+    v_pool = _rand((NB, Hkv, 16, D), dtype, gen).to(dev)
+    h = {"k_pool": storage(k_pool), "v_pool": storage(v_pool)}
+    mgr.add(0, 0)
+    live, next_id, copies = [0], 1, 0
+    first = True
+    for step_no in range(12):
+        if first:
+            batch = {0: 45}                      # the prompt
+            first = False
+        else:
+            cands = []
+            for b in live:                       # every beam proposes `fan` continuations
+                for _ in range(fan):
+                    mgr.fork(b, next_id)
+                    cands.append(next_id)
+                    next_id += 1
+            for b in live:
+                mgr.free(b)
+            keep = sorted(rng.choice(len(cands), size=min(beams, len(cands)), replace=False).tolist())
+            for i, c in enumerate(cands):
+                if i not in keep:
+                    mgr.free(c)
+            live = [cands[i] for i in keep]
+            batch = {b: 1 for b in live}
+        tables, ctx, qsl, pairs = mgr.step(batch, width)
+        counts = np.asarray(list(batch.values()), np.int64)
+        prior = (ctx - counts).astype(np.int32)
+        T = int(qsl[-1])
+        q = _rand((T, Hq, D), dtype, gen)
+        k_new = _rand((T, Hkv, D), dtype, gen)
+        v_new = _rand((T, Hkv, D), dtype, gen)
+        wl = SimpleNamespace(copy_pairs=pairs, write_batch=dict(batch), batch=batch, prior_lens=prior,
+                             block_tables=tables, scale=scale, dtype=dtype_name)
+        h.update(q=storage(q), k_new=storage(k_new), v_new=storage(v_new))
+        ref = oracle_step(wl, h)
+        step = PagedAttentionStep(batch, prior, tables, NB, Hq, Hkv, D, dtype, dev, write_batch=dict(batch),
+                                  copy_pairs=pairs)
+        out = step.run(q.to(dev), k_pool, v_pool, scale, k_new.to(dev), v_new.to(dev))
+        torch.cuda.synchronize()
+        assert pkv.device_error() == (0, -1)
+        err = max_err(out, ref)
+        assert err <= TOL[dtype_name], f"step {step_no}: max |err| {err}"
+        assert np.array_equal(storage(k_pool), h["k_pool"]) and np.array_equal(storage(v_pool), h["v_pool"])
+        copies += len(pairs)
+    st = mgr.stats()
+    assert copies > 0 and st["shared_blocks"] > 0 and st["num_sequences"] == beams
