@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--rows-per-item", type=int, default=0, help="query rows of a request per CUDA-core work item")
     ap.add_argument("--tc-min-rows", type=int, default=0, help="fewest rows a request needs for the tcgen05 tiles")
     ap.add_argument("--cuda-core-only", action="store_true", help="serve every row on CUDA cores")
+    ap.add_argument("--decode-kernel", type=int, default=0, choices=[0, 1, 2],
+                    help="kernel for CUDA-core rows: 0 planner's choice, 1 FMA, 2 warp MMA")
     return ap.parse_args()
 
 
@@ -319,6 +321,8 @@ def main():
         opts["tc_min_rows"] = args.tc_min_rows
     if args.cuda_core_only:
         opts["cuda_core_only"] = True
+    if args.decode_kernel:
+        opts["decode_kernel"] = args.decode_kernel
     step = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,
                               wl.num_kv_heads, wl.head_dim, dt, dev, write_batch=wl.write_batch or None,
                               copy_pairs=wl.copy_pairs, **opts)
@@ -415,12 +419,15 @@ def main():
     value = whole_job_gbs(kv_bytes(wl), world, ms_per_step)
     # Roofline of the kernel that takes the most time per step.
     work = kernel_work(step.plan.plan, wl)
-    names = {"decode": "decode_kernel (CUDA-core split-K)", "prefill_tc": "prefill_tc_kernel (tcgen05 tiles)"}
+    names = {"decode": ("decode_mma_kernel (warp-MMA split-K)" if step.plan.plan.decode_kernel == 2
+                        else "decode_kernel (CUDA-core split-K)"),
+             "prefill_tc": "prefill_tc_kernel (tcgen05 tiles)"}
     timed = {k: prof[k] for k in work if prof[k][1]}
     roof = None
     if timed:
         k = max(timed, key=lambda x: timed[x][0])
         avg_ms = timed[k][0] / timed[k][1]
+        kname = "decode_mma_kernel" if (k == "decode" and step.plan.plan.decode_kernel == 2) else k + "_kernel"
         w = work[k]
         tc_peak, tc_kind = tensor_peak()
         t_hbm = w["bytes"] / (peak * 1e9)
@@ -428,12 +435,12 @@ def main():
         if t_tc > t_hbm:
             achieved = w["flops"] / (avg_ms * 1e-3) / 1e12
             roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                    "frac": achieved / tc_peak, "traffic": recorded_traffic(k + "_kernel", wl.name),
+                    "frac": achieved / tc_peak, "traffic": recorded_traffic(kname, wl.name),
                     "algorithmic_flops": w["flops"], "peak_source": f"{tc_kind} bf16_tflops (burst cuBLAS)"}
         else:
             achieved = w["bytes"] / (avg_ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": recorded_traffic(k + "_kernel", wl.name), "algorithmic_bytes": w["bytes"],
+                    "traffic": recorded_traffic(kname, wl.name), "algorithmic_bytes": w["bytes"],
                     "peak_source": f"{peak_kind} hbm_gbs (burst copy)"}
         roof.update(kernel=names[k], kernel_ms=avg_ms)
     launches = sum(v[1] for k, v in prof.items() if k != "dropped")

@@ -122,6 +122,9 @@ typedef struct pkv_plan_options {
                                   item streams each K/V block once for all its (row, head) pairs */
     int32_t tc_min_rows;       /* requests with at least this many rows (>= 2; 0 = 2) go to the
                                   tcgen05 tiles where the shape allows; fewer rows, CUDA cores */
+    int32_t decode_kernel;     /* kernel for the rows not on tcgen05 tiles: 0 = chosen by the
+                                  planner, 1 = FMA kernel (items of <= 8 (row, head) slots),
+                                  2 = warp-MMA kernel (<= 16 slots; f16/bf16, head_dim 128) */
 } pkv_plan_options;
 
 /*
@@ -141,6 +144,8 @@ typedef struct pkv_plan {
     int32_t max_blocks;          /* longest context in blocks */
     int32_t heads_per_item;      /* query heads per CUDA-core work item */
     int32_t rows_per_item;       /* most consecutive rows any CUDA-core item serves (0: no items) */
+    int32_t decode_kernel;       /* 1 FMA kernel, 2 warp-MMA kernel, 0 no CUDA-core items */
+    int32_t part_stride;         /* (row, head) slots per partial-result entry */
     int64_t off_items, off_tiles, off_merge, off_part_o, off_part_ml; /* byte offsets into workspace */
     int64_t meta_bytes;          /* bytes uploaded by pkv_attention_plan (work lists) */
     int64_t ws_bytes;            /* total workspace bytes this plan needs */

@@ -96,10 +96,23 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     const bool tc_ok = !o.cuda_core_only && prefill_tc_supported((int)dt, D, G);
     const int tc_min = o.tc_min_rows > 2 ? o.tc_min_rows : 2;
     const int eb = elem_bytes(dt);
-    const int hpi = (o.heads_per_item > 0 && o.heads_per_item <= kMaxGroupPerItem) ? o.heads_per_item
-                                                                                  : std::min(G, kMaxGroupPerItem);
-    // Rows per CUDA-core item: as many consecutive rows of a request as fit 8 (row, head) slots.
-    const int rows_cap = kMaxGroupPerItem / hpi;
+    if (o.decode_kernel < 0 || o.decode_kernel > 2) return fail(PKV_ERR_INVALID_ARG, "decode_kernel %d", o.decode_kernel);
+    const bool mma_ok = decode_mma_supported((int)dt, D);
+    if (o.decode_kernel == 2 && !mma_ok)
+        return fail(PKV_ERR_UNSUPPORTED, "the MMA decode kernel needs f16/bf16 and head_dim 128");
+    // CUDA-core rows: decode rows, and multi-row requests the tcgen05 tiles do not take.
+    bool multi_core = false;
+    for (int r = 0; r < R; ++r) {
+        const int n = qsl[r + 1] - qsl[r];
+        if (n > 1 && !(tc_ok && n >= tc_min)) multi_core = true;
+    }
+    // Kernel for the CUDA-core rows: warp-level MMAs over 16 (row, head) slots where items hold
+    // 8 or more slots (a large query group, or several rows of a request); FMAs otherwise.
+    const int kind = o.decode_kernel ? o.decode_kernel : ((mma_ok && (G >= 8 || multi_core)) ? 2 : 1);
+    const int slot_cap = kind == 2 ? kMmaSlots : kMaxGroupPerItem;
+    const int hpi = (o.heads_per_item > 0 && o.heads_per_item <= slot_cap) ? o.heads_per_item : std::min(G, slot_cap);
+    // Rows per CUDA-core item: as many consecutive rows of a request as fit the item's slots.
+    const int rows_cap = slot_cap / hpi;
     const int rpi = o.rows_per_item > 0 ? std::min(o.rows_per_item, rows_cap) : rows_cap;
 
     struct CoreRow { int row, req, limit, nrows; };  // nrows consecutive rows; the first sees keys < limit
@@ -231,6 +244,8 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     int max_rows = 0;
     for (const CoreRow& c : core_rows) max_rows = std::max(max_rows, c.nrows);
     plan->rows_per_item = max_rows;
+    plan->decode_kernel = L->items.empty() ? 0 : kind;
+    plan->part_stride = slot_cap;
     int64_t off = 256;  // first 256 bytes reserved
     plan->off_items = off;
     off = align256(off + (int64_t)L->items.size() * sizeof(DecodeItem));
@@ -240,9 +255,9 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     off = align256(off + (int64_t)L->merges.size() * sizeof(MergeRow));
     plan->meta_bytes = off;
     plan->off_part_o = off;
-    off = align256(off + (int64_t)L->num_partials * kMaxGroupPerItem * D * 4);
+    off = align256(off + (int64_t)L->num_partials * slot_cap * D * 4);
     plan->off_part_ml = off;
-    off = align256(off + (int64_t)L->num_partials * kMaxGroupPerItem * 2 * 4);
+    off = align256(off + (int64_t)L->num_partials * slot_cap * 2 * 4);
     plan->ws_bytes = off;
     plan->kv_bytes = kv_bytes;
     plan->attn_flops = flops;
@@ -496,9 +511,11 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         a.num_blocks = num_blocks; a.num_q_heads = plan->num_q_heads; a.num_kv_heads = plan->num_kv_heads;
         a.group = G; a.heads_per_item = plan->heads_per_item;
         a.slots_per_item = plan->heads_per_item * std::max(plan->rows_per_item, 1);
+        a.part_stride = plan->part_stride;
         a.scale_log2 = scale_log2;
         ProfileScope prof(PKV_KERNEL_DECODE, s);
-        cudaError_t e = launch_decode(plan->dtype, plan->head_dim, a, sms, s);
+        cudaError_t e = plan->decode_kernel == 2 ? launch_decode_mma(plan->dtype, a, sms, s)
+                                                 : launch_decode(plan->dtype, plan->head_dim, a, sms, s);
         if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     }
     if (plan->num_merge_rows > 0) {
@@ -510,6 +527,7 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         m.num_rows = plan->num_merge_rows;
         m.num_q_heads = plan->num_q_heads;
         m.slots_per_entry = plan->heads_per_item * std::max(plan->rows_per_item, 1);
+        m.part_stride = plan->part_stride;
         ProfileScope prof(PKV_KERNEL_MERGE, s);
         cudaError_t e = launch_merge(plan->dtype, plan->head_dim, m, s);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");

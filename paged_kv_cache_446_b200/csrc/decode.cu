@@ -371,13 +371,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
                             *reinterpret_cast<uint4*>(static_cast<unsigned char*>(a.out) + qh * C::ROW + chunk * 16) =
                                 Chunk<T>::pack(o);
                         } else {
-                            float* po = a.part_o + ((size_t)ci.partial * kMaxGroupPerItem + g) * D + chunk * C::EPC;
+                            float* po = a.part_o + ((size_t)ci.partial * a.part_stride + g) * D + chunk * C::EPC;
 #pragma unroll
                             for (int e = 0; e < C::E2; e += 2)
                                 *reinterpret_cast<float4*>(po + 2 * e) =
                                     make_float4(acc2[g][e].x, acc2[g][e].y, acc2[g][e + 1].x, acc2[g][e + 1].y);
                             if (chunk == 0) {
-                                float* pm = a.part_ml + ((size_t)ci.partial * kMaxGroupPerItem + g) * 2;
+                                float* pm = a.part_ml + ((size_t)ci.partial * a.part_stride + g) * 2;
                                 pm[0] = ml_s[2 * g];
                                 pm[1] = ml_s[2 * g + 1];
                             }
@@ -410,13 +410,13 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
     if (g >= mr.num_slots) return;
     float M = -INFINITY;
     for (int i = 0; i < mr.count; ++i)
-        M = fmaxf(M, a.part_ml[((size_t)(mr.first_partial + i) * kMaxGroupPerItem + g) * 2]);
+        M = fmaxf(M, a.part_ml[((size_t)(mr.first_partial + i) * a.part_stride + g) * 2]);
     float L = 0.f;
     float o[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) o[e] = 0.f;
     for (int i = 0; i < mr.count; ++i) {
-        const size_t p = (size_t)(mr.first_partial + i) * kMaxGroupPerItem + g;
+        const size_t p = (size_t)(mr.first_partial + i) * a.part_stride + g;
         const float w = fast_exp2(a.part_ml[p * 2] - M);
         L = fmaf(w, a.part_ml[p * 2 + 1], L);
         const float* po = a.part_o + p * D + lane * PER;

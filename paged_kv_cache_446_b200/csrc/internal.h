@@ -7,7 +7,8 @@
 namespace pkv {
 
 constexpr int kBlockSize = 16;      // tokens per KV block
-constexpr int kMaxGroupPerItem = 8; // query heads one CUDA-core work item serves (GQA packing)
+constexpr int kMaxGroupPerItem = 8; // (row, head) slots one FMA-kernel work item serves
+constexpr int kMmaSlots = 16;       // (row, head) slots one MMA-kernel work item serves
 
 // First device-side error and its detail (an index); zero when none happened.
 struct DeviceError {
@@ -62,8 +63,8 @@ struct DecodeArgs {
     const void* v_pool;
     const int32_t* block_tables;
     const DecodeItem* items;
-    float* part_o;       // [num_partials][8][D]
-    float* part_ml;      // [num_partials][8][2] (max in log2 units, sum)
+    float* part_o;       // [num_partials][part_stride][D]
+    float* part_ml;      // [num_partials][part_stride][2] (max in log2 units, sum)
     DeviceError* err;
     int num_items;
     int max_blocks_per_seq;
@@ -72,7 +73,8 @@ struct DecodeArgs {
     int num_kv_heads;
     int group;           // Hq / Hkv
     int heads_per_item;  // query heads one item serves (<= 8)
-    int slots_per_item;  // largest num_rows x heads of any item (<= 8): selects the kernel variant
+    int slots_per_item;  // largest num_rows x heads of any item: selects the kernel variant
+    int part_stride;     // slots per partial-result entry (8 for the FMA kernel, 16 for the MMA kernel)
     float scale_log2;    // scale * log2(e)
 };
 
@@ -84,6 +86,7 @@ struct MergeArgs {
     int num_rows;
     int num_q_heads;
     int slots_per_entry;  // largest num_slots of any merge row: warps launched per row
+    int part_stride;      // slots per partial-result entry
 };
 
 struct PrefillArgs {
@@ -109,6 +112,8 @@ struct PrefillArgs {
 // Launchers (return the launch error, if any).
 cudaError_t launch_decode(int dtype, int head_dim, const DecodeArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_merge(int dtype, int head_dim, const MergeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_mma(int dtype, const DecodeArgs& a, int num_sms, cudaStream_t s);
+bool decode_mma_supported(int dtype, int head_dim);
 cudaError_t launch_prefill_tc(int dtype, const PrefillArgs& a, int num_sms, cudaStream_t s);
 bool prefill_tc_supported(int dtype, int head_dim, int group);
 cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, const int32_t* qsl, const int32_t* ctx,

@@ -32,6 +32,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "tma_host.h"
 
 namespace pkv {
 namespace {
@@ -61,13 +62,6 @@ constexpr float kRescaleThreshold = 8.f;
 constexpr int kPolyPairs = 2;
 
 // ---- tcgen05 / TMA primitives ---------------------------------------------------------------
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
@@ -508,30 +502,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// ---- host side: tensor maps ------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static std::once_flag once;
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-bool encode(CUtensorMap* m, CUtensorMapDataType t, int rank, const void* base, const cuuint64_t* dims,
-            const cuuint64_t* strides, const cuuint32_t* box) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, t, rank, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename T, int POLY>
 cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     const CUtensorMapDataType dt =
@@ -545,8 +515,8 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     const cuuint64_t kdims[2] = {128, (cuuint64_t)rows};
     const cuuint64_t kstr[1] = {128 * 2};
     const cuuint32_t kbox[2] = {64, (cuuint32_t)kBlockSize};
-    if (!encode(&mq, dt, 3, a.q, qdims, qstr, qbox) || !encode(&mk, dt, 2, a.k_pool, kdims, kstr, kbox) ||
-        !encode(&mv, dt, 2, a.v_pool, kdims, kstr, kbox))
+    if (!encode_tiled(&mq, dt, 3, a.q, qdims, qstr, qbox) || !encode_tiled(&mk, dt, 2, a.k_pool, kdims, kstr, kbox) ||
+        !encode_tiled(&mv, dt, 2, a.v_pool, kdims, kstr, kbox))
         return cudaErrorInvalidValue;
     static int configured[64] = {0};
     int dev = 0;

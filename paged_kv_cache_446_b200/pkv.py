@@ -38,14 +38,14 @@ _SZ = ctypes.c_size_t
 class PlanOptions(ctypes.Structure):
     _fields_ = [("split_blocks", ctypes.c_int32), ("no_split", ctypes.c_int32),
                 ("cuda_core_only", ctypes.c_int32), ("num_sms", ctypes.c_int32), ("heads_per_item", ctypes.c_int32),
-                ("rows_per_item", ctypes.c_int32), ("tc_min_rows", ctypes.c_int32)]
+                ("rows_per_item", ctypes.c_int32), ("tc_min_rows", ctypes.c_int32), ("decode_kernel", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):
     _fields_ = [("magic", ctypes.c_uint32)] + [(n, ctypes.c_int32) for n in (
         "num_reqs", "num_q_tokens", "num_q_heads", "num_kv_heads", "head_dim", "dtype", "num_decode_rows",
         "num_prefill_rows", "num_items", "num_tiles", "num_merge_rows", "num_partials", "split_blocks",
-        "max_blocks", "heads_per_item", "rows_per_item")] + [(n, ctypes.c_int64) for n in (
+        "max_blocks", "heads_per_item", "rows_per_item", "decode_kernel", "part_stride")] + [(n, ctypes.c_int64) for n in (
         "off_items", "off_tiles", "off_merge", "off_part_o", "off_part_ml", "meta_bytes", "ws_bytes", "kv_bytes",
         "attn_flops", "core_kv_bytes", "tile_kv_bytes", "tile_flops")]
 
@@ -118,9 +118,9 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _opts(split_blocks=0, no_split=False, cuda_core_only=False, num_sms=0, heads_per_item=0, rows_per_item=0,
-          tc_min_rows=0) -> PlanOptions:
+          tc_min_rows=0, decode_kernel=0) -> PlanOptions:
     return PlanOptions(int(split_blocks), int(bool(no_split)), int(bool(cuda_core_only)), int(num_sms),
-                       int(heads_per_item), int(rows_per_item), int(tc_min_rows))
+                       int(heads_per_item), int(rows_per_item), int(tc_min_rows), int(decode_kernel))
 
 
 # ---- a13: mixed-batch flattening -------------------------------------------------------------

@@ -106,7 +106,9 @@ def parse_meta(plan, meta):
                                   {"cuda_core_only": True}, {"heads_per_item": 4}, {"heads_per_item": 3},
                                   {"cuda_core_only": True, "split_blocks": 2}, {"tc_min_rows": 9},
                                   {"cuda_core_only": True, "rows_per_item": 1},
-                                  {"cuda_core_only": True, "rows_per_item": 3, "heads_per_item": 2}])
+                                  {"cuda_core_only": True, "rows_per_item": 3, "heads_per_item": 2},
+                                  {"decode_kernel": 1}, {"decode_kernel": 2, "tc_min_rows": 9},
+                                  {"decode_kernel": 2, "heads_per_item": 16, "split_blocks": 2}])
 def test_planner_covers_every_block_once(pkv, seed, opts):
     """Every (row, query head, visible KV block) is covered by exactly one work item or tile."""
     rng = np.random.default_rng(seed)
@@ -118,7 +120,15 @@ def test_planner_covers_every_block_once(pkv, seed, opts):
     qsl = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
     Hq, Hkv = [(8, 8), (32, 8), (64, 8), (32, 2), (6, 3)][seed % 5]
     dtype = ["f16", "bf16", "f32"][seed % 3]
+    if opts.get("decode_kernel") == 2 and dtype == "f32":
+        with pytest.raises(pkv.PkvError):
+            pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, **opts)
+        return
     plan, meta = pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, **opts)
+    if plan.num_items:
+        assert plan.decode_kernel in (1, 2) and plan.part_stride == (16 if plan.decode_kernel == 2 else 8)
+        if "decode_kernel" in opts:
+            assert plan.decode_kernel == opts["decode_kernel"]
     items, tiles, merges = parse_meta(plan, meta)
     G = Hq // Hkv
     hpi = plan.heads_per_item
@@ -126,7 +136,7 @@ def test_planner_covers_every_block_once(pkv, seed, opts):
     max_rows = 0
     for row, req, packed, head0, b0, b1, limit, part in items:
         kvh, nrows = packed & 0xFFFF, packed >> 16
-        assert 1 <= nrows and nrows * min(hpi, G - head0) <= 8
+        assert 1 <= nrows and nrows * min(hpi, G - head0) <= plan.part_stride
         max_rows = max(max_rows, nrows)
         nreq = qsl[req + 1] - qsl[req]
         assert qsl[req] <= row and row + nrows <= qsl[req + 1]

@@ -271,5 +271,30 @@ def test_verify_rows(dev, dtype, Hq, Hkv, D, specs, opts):
     p = step.plan.plan
     G = Hq // Hkv
     if opts.get("tc_min_rows") and p.num_items:
-        assert p.rows_per_item == min(max(n for _, n in specs), max(1, 8 // min(G, 8)))
+        cap = p.part_stride
+        assert p.rows_per_item == min(max(n for _, n in specs), max(1, cap // min(G, cap)))
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("opts", [{}, {"split_blocks": 1}, {"split_blocks": 5}, {"no_split": True}],
+                         ids=["auto-split", "split1", "split5", "nosplit"])
+@pytest.mark.parametrize("config", ["c2", "c3", "c4", "c5", "c6"])
+def test_decode_kernels(dev, config, opts, kernel):
+    """The FMA and warp-MMA kernels for CUDA-core rows, forced, on each 16-bit configuration
+    (small), chunked in several ways, against the oracle."""
+    wl = W.make(config, device=dev, small=True)
+    _, step = run_and_compare(wl, dev, decode_kernel=kernel, tc_min_rows=9, **opts)
+    assert step.plan.plan.decode_kernel == kernel
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,specs", [
+    ("bf16", 64, 8, 128, [(16 * 2080 - 1, 1), (3, 1), (100, 16)]),    # long context; 16 rows
+    ("f16", 32, 2, 128, [(31, 1), (16, 1), (200, 2)]),                # group of 16: 16 slots per row
+    ("bf16", 96, 4, 128, [(70, 1), (5, 3)]),                          # group of 24: split over items
+    ("f16", 8, 8, 128, [(0, 1), (15, 1), (16, 1), (17, 9)]),          # tiny contexts, G = 1
+])
+def test_mma_kernel_edges(dev, dtype, Hq, Hkv, D, specs):
+    wl = custom(dev, dtype, Hq, Hkv, D, specs, seed=23)
+    _, step = run_and_compare(wl, dev, decode_kernel=2, tc_min_rows=64)
+    assert step.plan.plan.decode_kernel == 2
 
