@@ -120,8 +120,10 @@ typedef struct pkv_plan_options {
     int32_t rows_per_item;     /* consecutive query rows of one request served by one CUDA-core
                                   item, capped so rows x heads <= 8; 0 = as many as fit. Such an
                                   item streams each K/V block once for all its (row, head) pairs */
-    int32_t tc_min_rows;       /* requests with at least this many rows (>= 2; 0 = 2) go to the
-                                  tcgen05 tiles where the shape allows; fewer rows, CUDA cores */
+    int32_t tc_min_rows;       /* requests with at least this many rows (>= 2) go to the tcgen05
+                                  tiles where the shape allows; fewer rows, the CUDA-core kernel.
+                                  0 = rows x group > 16 with the MMA kernel (a request whose
+                                  (row, head) pairs fit one MMA item stays there), else 2 */
     int32_t decode_kernel;     /* kernel for the rows not on tcgen05 tiles: 0 = chosen by the
                                   planner, 1 = FMA kernel (items of <= 8 (row, head) slots),
                                   2 = warp-MMA kernel (<= 16 slots; f16/bf16, head_dim 128) */
@@ -145,7 +147,7 @@ typedef struct pkv_plan {
     int32_t heads_per_item;      /* query heads per CUDA-core work item */
     int32_t rows_per_item;       /* most consecutive rows any CUDA-core item serves (0: no items) */
     int32_t decode_kernel;       /* 1 FMA kernel, 2 warp-MMA kernel, 0 no CUDA-core items */
-    int32_t part_stride;         /* (row, head) slots per partial-result entry */
+    int32_t part_stride;         /* (row, head) slots per partial-result entry: the largest item's */
     int64_t off_items, off_tiles, off_merge, off_part_o, off_part_ml; /* byte offsets into workspace */
     int64_t meta_bytes;          /* bytes uploaded by pkv_attention_plan (work lists) */
     int64_t ws_bytes;            /* total workspace bytes this plan needs */

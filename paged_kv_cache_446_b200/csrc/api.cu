@@ -94,21 +94,19 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     pkv_plan_options o{};
     if (opts) o = *opts;
     const bool tc_ok = !o.cuda_core_only && prefill_tc_supported((int)dt, D, G);
-    const int tc_min = o.tc_min_rows > 2 ? o.tc_min_rows : 2;
     const int eb = elem_bytes(dt);
     if (o.decode_kernel < 0 || o.decode_kernel > 2) return fail(PKV_ERR_INVALID_ARG, "decode_kernel %d", o.decode_kernel);
     const bool mma_ok = decode_mma_supported((int)dt, D);
+    // Multi-row requests whose rows x heads fit one 16-slot MMA item stream each K/V block once
+    // there, as a tcgen05 tile would, and faster (measured on speculative verify steps); larger
+    // ones go to the tiles.
+    const int tc_min = o.tc_min_rows >= 2 ? o.tc_min_rows : (mma_ok && o.decode_kernel != 1 ? std::max(2, kMmaSlots / G + 1) : 2);
     if (o.decode_kernel == 2 && !mma_ok)
         return fail(PKV_ERR_UNSUPPORTED, "the MMA decode kernel needs f16/bf16 and head_dim 128");
-    // CUDA-core rows: decode rows, and multi-row requests the tcgen05 tiles do not take.
-    bool multi_core = false;
-    for (int r = 0; r < R; ++r) {
-        const int n = qsl[r + 1] - qsl[r];
-        if (n > 1 && !(tc_ok && n >= tc_min)) multi_core = true;
-    }
-    // Kernel for the CUDA-core rows: warp-level MMAs over 16 (row, head) slots where items hold
-    // 8 or more slots (a large query group, or several rows of a request); FMAs otherwise.
-    const int kind = o.decode_kernel ? o.decode_kernel : ((mma_ok && (G >= 8 || multi_core)) ? 2 : 1);
+    // Kernel for the CUDA-core rows: warp-level MMAs over 16 (row, head) slots wherever the type
+    // and head size allow (measured as fast or faster than the FMA kernel for groups of 1 to 8
+    // and for packed rows); the FMA kernel otherwise.
+    const int kind = o.decode_kernel ? o.decode_kernel : (mma_ok ? 2 : 1);
     const int slot_cap = kind == 2 ? kMmaSlots : kMaxGroupPerItem;
     const int hpi = (o.heads_per_item > 0 && o.heads_per_item <= slot_cap) ? o.heads_per_item : std::min(G, slot_cap);
     // Rows per CUDA-core item: as many consecutive rows of a request as fit the item's slots.
@@ -245,7 +243,9 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     for (const CoreRow& c : core_rows) max_rows = std::max(max_rows, c.nrows);
     plan->rows_per_item = max_rows;
     plan->decode_kernel = L->items.empty() ? 0 : kind;
-    plan->part_stride = slot_cap;
+    // Partial entries hold as many (row, head) slots as the largest item has.
+    const int part_stride = std::max(1, std::min(slot_cap, hpi * std::max(max_rows, 1)));
+    plan->part_stride = part_stride;
     int64_t off = 256;  // first 256 bytes reserved
     plan->off_items = off;
     off = align256(off + (int64_t)L->items.size() * sizeof(DecodeItem));
@@ -255,9 +255,9 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     off = align256(off + (int64_t)L->merges.size() * sizeof(MergeRow));
     plan->meta_bytes = off;
     plan->off_part_o = off;
-    off = align256(off + (int64_t)L->num_partials * slot_cap * D * 4);
+    off = align256(off + (int64_t)L->num_partials * part_stride * D * 4);
     plan->off_part_ml = off;
-    off = align256(off + (int64_t)L->num_partials * slot_cap * 2 * 4);
+    off = align256(off + (int64_t)L->num_partials * part_stride * 2 * 4);
     plan->ws_bytes = off;
     plan->kv_bytes = kv_bytes;
     plan->attn_flops = flops;

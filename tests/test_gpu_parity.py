@@ -224,7 +224,7 @@ PREFILL_CASES = [
 @pytest.mark.parametrize("dtype,Hq,Hkv,D,specs", PREFILL_CASES)
 def test_prefill_tiles_tcgen05(dev, dtype, Hq, Hkv, D, specs):
     wl = custom(dev, dtype, Hq, Hkv, D, specs, seed=11)
-    _, step = run_and_compare(wl, dev)
+    _, step = run_and_compare(wl, dev, tc_min_rows=2)
     assert step.plan.plan.num_tiles > 0, "expected the tcgen05 tile path"
 
 
@@ -232,7 +232,7 @@ def test_prefill_tiles_tcgen05(dev, dtype, Hq, Hkv, D, specs):
 def test_prefill_tiles_match_cuda_core_path(dev, dtype, Hq, Hkv, D, specs):
     """The tcgen05 tiles and the CUDA-core kernel agree on the same prefill rows."""
     wl = custom(dev, dtype, Hq, Hkv, D, specs, seed=12)
-    a = make_step(wl, dev).run(wl.q, wl.k_pool, wl.v_pool, wl.scale).clone()
+    a = make_step(wl, dev, tc_min_rows=2).run(wl.q, wl.k_pool, wl.v_pool, wl.scale).clone()
     b = make_step(wl, dev, cuda_core_only=True).run(wl.q, wl.k_pool, wl.v_pool, wl.scale)
     torch.cuda.synchronize()
     err = (a.double() - b.double()).abs().max().item()
