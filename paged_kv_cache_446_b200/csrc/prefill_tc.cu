@@ -59,7 +59,7 @@ constexpr uint32_t kTmemCols = 512;                  // S_A [0,128), S_B [128,25
 constexpr float kRescaleThreshold = 8.f;
 // Of each 32 exponentials of an unmasked key tile, 2 * POLY are computed by exp2_poly2 on the FMA
 // pipe (the kernel's template parameter; default kPolyPairs, PKV_PREFILL_POLY_PAIRS overrides it).
-constexpr int kPolyPairs = 2;
+constexpr int kPolyPairs = 0;  // measured: with three TMEM round trips per tile, MUFU alone is fastest
 
 // ---- tcgen05 / TMA primitives ---------------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
@@ -374,20 +374,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const bool full = kt * 128 + 128 <= all_visible;   // no masking anywhere in this key tile
-            // pass 1: row maximum of scale * s over the visible keys
-            float mx = -INFINITY;
+            float alpha = 1.f;
+            float2 ps2 = make_float2(0.f, 0.f);
             if (full && a.scale_log2 >= 0.f) {
-#pragma unroll
-                for (int c = 0; c < 4; c += 2) {
+                // Three TMEM round trips: keys 64..127 for the maximum; keys 0..63 for the maximum
+                // and, from the same registers, their P (columns 0..31, over S already read); keys
+                // 64..127 again for their P (columns 32..63).
+                float mx = -INFINITY;
+                {
                     float sv[64];
-                    tmem_ld32(ts + c * 32, sv);
-                    tmem_ld32(ts + c * 32 + 32, sv + 32);
+                    tmem_ld32(ts + 64, sv);
+                    tmem_ld32(ts + 96, sv + 32);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
                 }
+                float sv[64];
+                tmem_ld32(ts, sv);
+                tmem_ld32(ts + 32, sv + 32);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
                 mx *= a.scale_log2;
+                if (mx > m + kRescaleThreshold) {
+                    alpha = fast_exp2(m - mx);  // 0 on the first tile
+                    m = mx;
+                }
+                const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 1) {
+                        tmem_ld32(ts + 64, sv);
+                        tmem_ld32(ts + 96, sv + 32);
+                        tmem_wait_ld();
+                    }
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
+                        const float2 p = (i & 15) < POLY ? exp2_poly2(e) : make_float2(fast_exp2(e.x), fast_exp2(e.y));
+                        ps2 = __fadd2_rn(ps2, p);
+                        pk[i] = pack2<T>(p.x, p.y);
+                    }
+                    tmem_st32(ts + h * 32, pk);
+                }
             } else {
+                // pass 1: row maximum of scale * s over the visible keys
+                float mx = -INFINITY;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float sv[32];
@@ -395,44 +428,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
                     const int key0 = kt * 128 + c * 32;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, key0 + i < limit ? sv[i] * a.scale_log2 : -INFINITY);
+                    for (int i = 0; i < 32; ++i)
+                        mx = fmaxf(mx, (full || key0 + i < limit) ? sv[i] * a.scale_log2 : -INFINITY);
                 }
-            }
-            float alpha = 1.f;
-            if (mx > m + kRescaleThreshold) {
-                alpha = fast_exp2(m - mx);  // 0 on the first tile
-                m = mx;
-            }
-            // pass 2: p = 2^(s*scale - m), rounded to T, written over S as the A operand of PV.
-            // Chunk c's P goes to columns 16c.., which pass 2 has already read.
-            float2 ps2 = make_float2(0.f, 0.f);
-            const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
+                if (mx > m + kRescaleThreshold) {
+                    alpha = fast_exp2(m - mx);  // 0 on the first tile
+                    m = mx;
+                }
+                // pass 2: p = 2^(s*scale - m), rounded to T, written over S as the A operand of PV.
+                // Chunk c's P goes to columns 16c.., which pass 2 has already read.
+                const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float sv[32];
-                tmem_ld32(ts + c * 32, sv);
-                tmem_wait_ld();
-                uint32_t pk[16];
-                if (full) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
-                        const float2 p = i < POLY ? exp2_poly2(e) : make_float2(fast_exp2(e.x), fast_exp2(e.y));
-                        ps2 = __fadd2_rn(ps2, p);
-                        pk[i] = pack2<T>(p.x, p.y);
-                    }
-                } else {
+                for (int c = 0; c < 4; ++c) {
+                    float sv[32];
+                    tmem_ld32(ts + c * 32, sv);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
                     const int key0 = kt * 128 + c * 32;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
-                        const float p0 = key0 + 2 * i < limit ? fast_exp2(e.x) : 0.f;
-                        const float p1 = key0 + 2 * i + 1 < limit ? fast_exp2(e.y) : 0.f;
+                        const float p0 = (full || key0 + 2 * i < limit) ? fast_exp2(e.x) : 0.f;
+                        const float p1 = (full || key0 + 2 * i + 1 < limit) ? fast_exp2(e.y) : 0.f;
                         ps2 = __fadd2_rn(ps2, make_float2(p0, p1));
                         pk[i] = pack2<T>(p0, p1);
                     }
+                    tmem_st16(ts + c * 16, pk);
                 }
-                tmem_st16(ts + c * 16, pk);
             }
             const float ps = ps2.x + ps2.y;
             l = l * alpha + ps;
@@ -541,7 +563,7 @@ int poly_pairs() {
 template <typename T>
 cudaError_t launch_p(const PrefillArgs& a, cudaStream_t s) {
     switch (poly_pairs()) {
-        case 0: return launch_t<T, 0>(a, s);
+        case 2: return launch_t<T, 2>(a, s);
         case 4: return launch_t<T, 4>(a, s);
         default: return launch_t<T, kPolyPairs>(a, s);
     }
