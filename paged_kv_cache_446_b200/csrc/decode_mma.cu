@@ -94,6 +94,16 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
     }
 }
 
+// The two 16-bit values of a packed word as fp32 (low half first).
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+    if constexpr (std::is_same<T, __half>::value) {
+        return __half22float2(*reinterpret_cast<const __half2*>(&w));
+    } else {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+}
+
 // Two fp32 values rounded to the 16-bit type and packed, `lo` in the low half.
 template <typename T>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -279,8 +289,13 @@ __global__ void __launch_bounds__(kMmaWarps * 32)
             p[j][2] = fast_exp2(s[j][2] - mu1);
             p[j][3] = fast_exp2(s[j][3] - mu1);
         }
-        float rs0 = (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-        float rs1 = (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+        // P as the A operand of P V: rows g / g + 8, token columns 2c, 2c+1 (+8). The row sums
+        // add the weights as rounded, so that they match what P V accumulates.
+        const uint32_t pa[4] = {pack2<T>(p[0][0], p[0][1]), pack2<T>(p[0][2], p[0][3]), pack2<T>(p[1][0], p[1][1]),
+                                pack2<T>(p[1][2], p[1][3])};
+        const float2 r00 = unpack2<T>(pa[0]), r01 = unpack2<T>(pa[1]), r10 = unpack2<T>(pa[2]), r11 = unpack2<T>(pa[3]);
+        float rs0 = (r00.x + r00.y) + (r10.x + r10.y);
+        float rs1 = (r01.x + r01.y) + (r11.x + r11.y);
         rs0 += __shfl_xor_sync(FULL_MASK, rs0, 1);
         rs1 += __shfl_xor_sync(FULL_MASK, rs1, 1);
         rs0 += __shfl_xor_sync(FULL_MASK, rs0, 2);
@@ -296,9 +311,6 @@ __global__ void __launch_bounds__(kMmaWarps * 32)
                 o[j][3] *= al1;
             }
         }
-        // P as the A operand of P V: rows g / g + 8, token columns 2c, 2c+1 (+8).
-        const uint32_t pa[4] = {pack2<T>(p[0][0], p[0][1]), pack2<T>(p[0][2], p[0][3]), pack2<T>(p[1][0], p[1][1]),
-                                pack2<T>(p[1][2], p[1][3])};
 
         // ---- V rows past the last visible key may hold anything: zero them ----
         const int vis = ci.limit + ci.num_rows - 1 - c_blk * kBlockSize;

@@ -170,6 +170,26 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
         return *reinterpret_cast<const uint32_t*>(&h);
     }
 }
+// Inverse of pack2: the two 16-bit values of a packed word as fp32 (low half first).
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+    if constexpr (std::is_same<T, __half>::value) {
+        return __half22float2(*reinterpret_cast<const __half2*>(&w));
+    } else {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+}
+// What a pair of softmax weights adds to the row sum. PV uses the weights rounded to T; for fp16
+// the sum takes them as rounded too, so that the normalisation matches the numerator exactly (an
+// fp16 output of magnitude 4..8 has a rounding step of ~2e-3, which leaves no room for the
+// mismatch on rows dominated by one key). For bf16 the unrounded weights are summed: the
+// mismatch (at most 2^-9 relative) stays far inside bf16's own output rounding, and the unpack
+// costs about 5 % of the kernel.
+template <typename T>
+__device__ __forceinline__ float2 row_sum_term(float2 p, uint32_t packed) {
+    if constexpr (std::is_same<T, __half>::value) return unpack2<T>(packed);
+    else return p;
+}
 
 template <typename T, int POLY>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -377,44 +397,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             float alpha = 1.f;
             float2 ps2 = make_float2(0.f, 0.f);
             if (full && a.scale_log2 >= 0.f) {
-                // Three TMEM round trips: keys 64..127 for the maximum; keys 0..63 for the maximum
-                // and, from the same registers, their P (columns 0..31, over S already read); keys
-                // 64..127 again for their P (columns 32..63).
-                float mx = -INFINITY;
-                {
-                    float sv[64];
-                    tmem_ld32(ts + 64, sv);
-                    tmem_ld32(ts + 96, sv + 32);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
-                }
-                float sv[64];
-                tmem_ld32(ts, sv);
-                tmem_ld32(ts + 32, sv + 32);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
-                mx *= a.scale_log2;
-                if (mx > m + kRescaleThreshold) {
-                    alpha = fast_exp2(m - mx);  // 0 on the first tile
-                    m = mx;
-                }
-                const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
+                // Two TMEM round trips, one per half of the key tile: the half's maximum is taken in
+                // registers and P computed from the same registers against the row's reference m,
+                // raised first when the half exceeds it by more than the threshold. P of keys
+                // 64*h.. goes to columns 32*h.. (over S already read). If the second half raises m,
+                // the first half's P, already stored, is scaled down by the same factor.
+                const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
-                    if (h == 1) {
-                        tmem_ld32(ts + 64, sv);
-                        tmem_ld32(ts + 96, sv + 32);
+                    float sv[64];
+                    tmem_ld32(ts + h * 64, sv);
+                    tmem_ld32(ts + h * 64 + 32, sv + 32);
+                    tmem_wait_ld();
+                    float hm = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) hm = fmaxf(hm, sv[i]);
+                    hm *= a.scale_log2;
+                    const bool raise = hm > m + kRescaleThreshold;
+                    const float f = raise ? fast_exp2(m - hm) : 1.f;  // 0 while m is -inf
+                    // The TMEM accesses are warp-collective: the whole warp takes this branch when
+                    // any of its rows raised, each lane scaling its own row by its own factor.
+                    if (h == 1 && __any_sync(FULL_MASK, raise)) {
+                        tmem_wait_st();
+                        float pv[32];
+                        tmem_ld32(ts, pv);
                         tmem_wait_ld();
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float2 q = unpack2<T>(__float_as_uint(pv[i]));
+                            pk[i] = pack2<T>(q.x * f, q.y * f);
+                        }
+                        tmem_st32(ts, pk);
                     }
+                    if (raise) {
+                        ps2 = make_float2(ps2.x * f, ps2.y * f);
+                        alpha *= f;
+                        m = hm;
+                    }
+                    const float2 nm2 = make_float2(-m, -m);
                     uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
                         const float2 p = (i & 15) < POLY ? exp2_poly2(e) : make_float2(fast_exp2(e.x), fast_exp2(e.y));
-                        ps2 = __fadd2_rn(ps2, p);
                         pk[i] = pack2<T>(p.x, p.y);
+                        ps2 = __fadd2_rn(ps2, row_sum_term<T>(p, pk[i]));
                     }
                     tmem_st32(ts + h * 32, pk);
                 }
@@ -450,8 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
                         const float p0 = (full || key0 + 2 * i < limit) ? fast_exp2(e.x) : 0.f;
                         const float p1 = (full || key0 + 2 * i + 1 < limit) ? fast_exp2(e.y) : 0.f;
-                        ps2 = __fadd2_rn(ps2, make_float2(p0, p1));
                         pk[i] = pack2<T>(p0, p1);
+                        ps2 = __fadd2_rn(ps2, row_sum_term<T>(make_float2(p0, p1), pk[i]));
                     }
                     tmem_st16(ts + c * 16, pk);
                 }

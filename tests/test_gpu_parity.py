@@ -298,3 +298,20 @@ def test_mma_kernel_edges(dev, dtype, Hq, Hkv, D, specs):
     _, step = run_and_compare(wl, dev, decode_kernel=2, tc_min_rows=64)
     assert step.plan.plan.decode_kernel == 2
 
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_prefill_reference_raised_mid_tile(dev, dtype):
+    """Keys whose scores jump by far more than the rescale threshold inside a 128-key tile (its
+    second half) and from tile to tile, so the prefill softmax raises a row's reference after
+    part of the tile's P is stored and rescales O repeatedly."""
+    wl = custom(dev, dtype, 16, 8, 128, [(700, 40), (130, 9)], seed=31)
+    k = wl.k_pool
+    for r in range(len(wl.batch)):
+        ctx = int(wl.prior_lens[r]) + wl.batch[r]
+        for p in range(ctx):
+            f = 1.0 + (5.0 if p % 128 >= 64 else 0.0) + 1.5 * (p // 128)
+            blk = int(wl.block_tables[r, p // 16])
+            k[blk, :, p % 16, :] *= f
+    _, step = run_and_compare(wl, dev, tc_min_rows=2)
+    assert step.plan.plan.num_tiles > 0
