@@ -192,8 +192,9 @@ def plan_host(query_start_loc: np.ndarray, context_lens: np.ndarray, num_q_heads
 class AttentionPlan:
     """A planned batch: host plan, device workspace and device copies of the batch description.
 
-    The workspace is reused across plans; it grows (one more planner run) only when a batch needs
-    more than it holds.
+    The workspace is reused across plans and grows only when a batch needs more than it holds.
+    replan() uploads the new work lists and batch description on `stream`, ordered after the
+    kernels of the previous batch when those ran on the same stream.
     """
 
     def __init__(self, batch: dict, prior_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
@@ -201,35 +202,61 @@ class AttentionPlan:
         self.num_q_heads, self.num_kv_heads, self.head_dim, self.dtype = num_q_heads, num_kv_heads, head_dim, dtype
         self.device = torch.device(device)
         self.opts = _opts(**opts)
+        if self.opts.num_sms == 0:
+            self.opts.num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
         self.workspace = workspace
         self.plan = Plan()
+        self._meta = None       # pinned image of the work lists
+        self._staged = None     # pinned query_start_loc + context_lens
+        self._dev = None        # their device copy
+        self._uploaded = None   # event after the last upload from the pinned buffers
         self.replan(batch, prior_lens, stream=stream)
 
     def replan(self, batch: dict, prior_lens, stream=None) -> "AttentionPlan":
+        """Plans the batch on the host (pkv_attention_plan_host) into pinned memory and uploads the
+        work lists and the batch description with asynchronous copies on `stream`."""
         qsl, ctx = flatten_batch(batch, prior_lens)
         self.h_query_start_loc, self.h_context_lens = qsl, ctx
         self.num_q_tokens = int(qsl[-1])
-        code = _dtype_code(torch.empty(0, dtype=self.dtype))
-        st = _stream(stream)
-        for _ in range(2):
-            ws = self.workspace
-            status = _plan(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], self.num_q_heads, self.num_kv_heads,
-                           self.head_dim, code, ctypes.byref(self.opts), _ptr(ws) if ws is not None else None,
-                           ws.numel() if ws is not None else 0, ctypes.byref(self.plan), st)
-            if status == PKV_OK:
-                break
-            if status in (1, 4) and (ws is None or ws.numel() < self.plan.ws_bytes) and self.plan.ws_bytes > 0:
-                self.workspace = torch.empty(max(int(self.plan.ws_bytes), 256), dtype=torch.uint8, device=self.device)
-                continue
-            _check(status, "pkv_attention_plan")
-        _check(status, "pkv_attention_plan")
-        # One pinned staging buffer for both arrays keeps the upload asynchronous; torch's host
-        # allocator keeps it alive until the copy has run.
         R = ctx.shape[0]
-        staged = torch.from_numpy(np.concatenate([qsl, ctx])).pin_memory()
-        dev = staged.to(self.device, non_blocking=True)
-        self.query_start_loc = dev[:R + 1]
-        self.context_lens = dev[R + 1:]
+        code = _dtype_code(torch.empty(0, dtype=self.dtype))
+        if self._uploaded is not None:
+            self._uploaded.synchronize()          # the pinned buffers are free again
+        for _ in range(2):
+            cap = self._meta.numel() if self._meta is not None else 0
+            status = _plan_host(_np_ptr(qsl), _np_ptr(ctx), R, self.num_q_heads, self.num_kv_heads, self.head_dim, code,
+                                ctypes.byref(self.opts), self._meta.data_ptr() if cap else None, cap,
+                                ctypes.byref(self.plan))
+            if status == 4 or (status == PKV_OK and cap == 0):
+                self._meta = torch.empty(max(int(self.plan.meta_bytes) * 5 // 4, 4096), dtype=torch.uint8).pin_memory()
+                continue
+            break
+        _check(status, "pkv_attention_plan_host")
+        if self.workspace is None or self.workspace.numel() < self.plan.ws_bytes:
+            self.workspace = torch.empty(max(int(self.plan.ws_bytes), 256), dtype=torch.uint8, device=self.device)
+        n = 2 * R + 1
+        if self._staged is None or self._staged.numel() < n:
+            cap = max(n, 64)
+            self._staged = torch.empty(cap, dtype=torch.int32).pin_memory()
+            self._dev = torch.empty(cap, dtype=torch.int32, device=self.device)
+        host = self._staged.numpy()
+        host[:R + 1] = qsl
+        host[R + 1:n] = ctx
+        if isinstance(stream, torch.cuda.Stream):
+            s = stream
+        elif stream is None or _stream(stream) == torch.cuda.current_stream(self.device).cuda_stream:
+            s = torch.cuda.current_stream(self.device)
+        else:
+            s = torch.cuda.ExternalStream(_stream(stream))
+        mb = int(self.plan.meta_bytes)
+        with torch.cuda.stream(s):
+            self.workspace[:mb].copy_(self._meta[:mb], non_blocking=True)
+            self._dev[:n].copy_(self._staged[:n], non_blocking=True)
+            if self._uploaded is None:
+                self._uploaded = torch.cuda.Event()
+            self._uploaded.record(s)
+        self.query_start_loc = self._dev[:R + 1]
+        self.context_lens = self._dev[R + 1:n]
         return self
 
 
