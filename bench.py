@@ -137,6 +137,21 @@ def decode_seq_tokens(wl) -> int:
     return int(ctx[n == 1].sum())
 
 
+def pool_waste(wl) -> dict:
+    """Internal fragmentation of paging for the step's sequences (each holding its context after the
+    step), from the library's host block manager (pkv_bm_*): blocks reserved, slots reserved but
+    unfilled, and their fraction -- the quantity the pages put under 4 %. Sequences are counted
+    independently (blocks shared between them would be counted once per sharer)."""
+    from paged_kv_cache_446_b200 import pkv
+    _, ctx = pkv.flatten_batch(wl.batch, wl.prior_lens)
+    m = pkv.BlockManager(int(sum(-(-int(c) // 16) for c in ctx)) + 1)
+    for r, c in enumerate(ctx):
+        m.add(r, int(c))
+    st = m.stats()
+    return {"reserved_blocks": st["used_blocks"], "unfilled_slots": st["wasted_slots"],
+            "frac": st["wasted_slots"] / max(1, 16 * st["used_blocks"])}
+
+
 def kernel_work(plan, wl) -> dict:
     """Algorithmic work per launch from the plan: the CUDA-core kernel reads K+V of its requests'
     contexts once per (request, KV head) plus its q rows and writes its output rows; the tcgen05
@@ -210,14 +225,26 @@ def bus_id_of(dev) -> str | None:
         return None
 
 
-def run_oracle_sample(wl, h, target_seconds: float):
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_oracle_sample(wl, h, target_seconds: float, threads: int = 0, append: bool = True):
     """The oracle, as it stands, on the first m requests (all heads, all rows) of the step, with the
-    step's own KV append applied first. Returns dict(value_gbs, seconds, requests, cores, bytes)."""
+    step's own KV append applied first (unless append=False: already applied to h). Returns
+    dict(value_gbs, seconds, requests, cores, bytes). threads = 0: every host core."""
     import oracle
-    cores = os.cpu_count() or 1
+    cores = threads or os.cpu_count() or 1
     qsl, ctx = oracle.flatten_batch(wl.batch, wl.prior_lens)
     counts = np.asarray(list(wl.batch.values()), np.int64)
-    if wl.write_batch:
+    if wl.write_batch and append:
         wcounts = np.asarray([wl.write_batch.get(r, 0) for r in wl.batch.keys()], np.int64)
         wqsl, wctx = oracle.flatten_batch(dict(zip(wl.batch.keys(), wcounts)), ctx.astype(np.int64) - wcounts)
         if len(wl.copy_pairs):
@@ -331,10 +358,16 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         h = {k: storage(getattr(wl, k)) for k in ("q", "k_pool", "v_pool", "k_new", "v_new")}
         r = run_oracle_sample(wl, h, args.cpu_seconds)
-        del h
         cpu_baseline = {"value": r["value_gbs"], "unit": "GB/s", "cores": r["cores"], "kind": "oracle",
                         "sample": f"first {r['requests']} of {r['of']} requests of {wl.name} (all heads and rows, "
-                                  f"after the step's KV append) x{r['repeats']}, {r['seconds']:.1f} s"}
+                                  f"after the step's KV append) x{r['repeats']}, {r['seconds']:.1f} s",
+                        "cpu_model": cpu_model()}
+        if args.config in ("c1", "c2"):
+            r1 = run_oracle_sample(wl, h, args.cpu_seconds / 3, threads=1, append=False)
+            cpu_baseline["single_thread"] = {
+                "value": r1["value_gbs"], "unit": "GB/s", "cores": 1,
+                "sample": f"first {r1['requests']} of {r1['of']} requests x{r1['repeats']}, {r1['seconds']:.1f} s"}
+        del h
 
     def run_step():
         step.run(wl.q, wl.k_pool, wl.v_pool, wl.scale, wl.k_new, wl.v_new, out=out)
@@ -494,6 +527,8 @@ def main():
                    "parallelism": f"replicas x{world} (independent requests per GPU)",
                    "plan_options": opts},
         "frac_of_hbm_peak": value / world / peak,
+        "frac_of_8tbs_spec": value / world / 8000.0,
+        "kv_block_waste": pool_waste(wl),
         "decode_seq_tokens_per_s": world * decode_seq_tokens(wl) / (ms_per_step * 1e-3),
         "decode_steps_per_s": 1e3 / ms_per_step,
         "kernel_ms_per_step": {k: v[0] / max(1, args.steps) for k, v in prof.items() if k != "dropped"},

@@ -273,6 +273,17 @@ def paged_attention(plan: AttentionPlan, q: torch.Tensor, k_pool: torch.Tensor, 
     return out
 
 
+def attend(batch: dict, prior_lens, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+           block_tables: torch.Tensor, scale: float, out: torch.Tensor | None = None, stream=None,
+           **opts) -> torch.Tensor:
+    """One call for a {request_id: num_tokens} batch (dict order): builds query_start_loc and
+    context_lens from it and each request's prior context, plans on the host and runs
+    pkv_paged_attention. Callers that run many steps keep an AttentionPlan and replan it instead."""
+    plan = AttentionPlan(batch, prior_lens, q.shape[1], k_pool.shape[1], q.shape[2], q.dtype, q.device,
+                         stream=stream, **opts)
+    return paged_attention(plan, q, k_pool, v_pool, block_tables, scale, out=out, stream=stream)
+
+
 # ---- host validators and the device error word -----------------------------------------------
 
 def validate_tables(block_tables: np.ndarray, context_lens: np.ndarray, num_blocks: int) -> None:

@@ -315,3 +315,15 @@ def test_prefill_reference_raised_mid_tile(dev, dtype):
             k[blk, :, p % 16, :] *= f
     _, step = run_and_compare(wl, dev, tc_min_rows=2)
     assert step.plan.plan.num_tiles > 0
+
+
+def test_attend_one_call(dev):
+    """pkv.attend plans and runs a {request_id: num_tokens} batch in one call (no KV append)."""
+    from paged_kv_cache_446_b200 import pkv
+    wl = custom(dev, "bf16", 32, 8, 128, [(300, 1), (0, 40), (17, 5), (64, 1)], seed=41)
+    h = host_inputs(wl)
+    bt = torch.from_numpy(wl.block_tables).to(dev)
+    out = pkv.attend(wl.batch, wl.prior_lens, wl.q, wl.k_pool, wl.v_pool, bt, wl.scale)
+    torch.cuda.synchronize()
+    err = max_err(out, oracle_step(wl, h))
+    assert err <= TOL["bf16"], err
