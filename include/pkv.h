@@ -127,6 +127,15 @@ typedef struct pkv_plan_options {
     int32_t decode_kernel;     /* kernel for the rows not on tcgen05 tiles: 0 = chosen by the
                                   planner, 1 = FMA kernel (items of <= 8 (row, head) slots),
                                   2 = warp-MMA kernel (<= 16 slots; f16/bf16, head_dim 128) */
+    /* Shared prefixes (optional; read during the planning call only). A run of consecutive decode
+     * requests (one row each) whose tables start with the same >= min_shared_blocks physical
+     * blocks (each fully inside every member's context) reads those blocks once for all of them;
+     * each request's own blocks are read separately and the parts are merged by log-sum-exp. The
+     * pages' sharing of a common prefix (parallel samples, beam candidates, cached prompts):
+     * 一文搞懂vLLM：为啥它能让一张GPU扛住几十倍用户？, "PagedAttention 是怎么共享内存的". */
+    const int32_t* h_block_tables;   /* host copy of block_tables, or NULL (no sharing) */
+    int32_t block_table_stride;      /* its row length (max_blocks_per_seq) */
+    int32_t min_shared_blocks;       /* 0 = 4 */
 } pkv_plan_options;
 
 /*

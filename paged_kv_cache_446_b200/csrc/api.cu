@@ -55,6 +55,7 @@ struct PlanLists {
     std::vector<MergeRow> merges;
     std::vector<size_t> start;
     std::vector<int> req_keys;
+    std::vector<int> shared_first;
     int num_partials = 0;
     void reset() {
         items.clear();
@@ -113,7 +114,11 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     const int rows_cap = slot_cap / hpi;
     const int rpi = o.rows_per_item > 0 ? std::min(o.rows_per_item, rows_cap) : rows_cap;
 
-    struct CoreRow { int row, req, limit, nrows; };  // nrows consecutive rows; the first sees keys < limit
+    // CUDA-core work: nrows consecutive rows whose first sees keys < limit, over the blocks
+    // [bs, be). kind 0: ordinary rows (partials only when split into several chunks); kind 1: the
+    // shared-prefix blocks of a group of requests (rows j .. j+nrows-1 of the group, always
+    // partials); kind 2: one group member's own blocks (always merged with its group's partials).
+    struct CoreRow { int row, req, limit, nrows, bs, be, kind, group, j; };
     static thread_local std::vector<CoreRow> core_rows;
     core_rows.clear();
     core_rows.reserve(R > 0 ? (size_t)qsl[R] : 0);
@@ -142,13 +147,74 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
                 }
         } else {
             if (n == 1) ++decode_rows;
-            for (int j = 0; j < n; j += rpi) core_rows.push_back(CoreRow{qsl[r] + j, r, P + j + 1, std::min(rpi, n - j)});
+            for (int j = 0; j < n; j += rpi) {
+                const int nr = std::min(rpi, n - j);
+                core_rows.push_back(CoreRow{qsl[r] + j, r, P + j + 1, nr, 0, (int)ceil_div(P + j + nr, kBlockSize), 0, -1, 0});
+            }
         }
     }
+    // Shared prefixes (cascade): consecutive decode requests whose block tables begin with the
+    // same physical blocks (parallel samples, beam candidates, requests reusing a cached prompt)
+    // read those blocks once for all of them: one set of items over the shared blocks for all their
+    // rows, one per request over its own blocks, combined by the log-sum-exp merge. Needs the host
+    // copy of the tables.
+    struct Group { int r0, r1, k, first_core; };  // requests [r0, r1), k shared blocks
+    static thread_local std::vector<Group> grps;
+    grps.clear();
+    if (o.h_block_tables && o.block_table_stride > 0 && rpi >= 2) {  // an item must hold >= 2 rows
+        const int minb = o.min_shared_blocks > 0 ? o.min_shared_blocks : 4;
+        const int stride = o.block_table_stride;
+        auto decode_row = [&](int r) { return qsl[r + 1] - qsl[r] == 1; };
+        for (int r = 0; r < R;) {
+            if (!decode_row(r)) { ++r; continue; }
+            int k = std::min(ctx[r] / kBlockSize, stride);
+            int e = r + 1;
+            while (e < R && decode_row(e)) {
+                const int kk = std::min(k, ctx[e] / kBlockSize);
+                const int32_t* a = o.h_block_tables + (size_t)r * stride;
+                const int32_t* b = o.h_block_tables + (size_t)e * stride;
+                int cp = 0;
+                while (cp < kk && a[cp] == b[cp]) ++cp;
+                if (cp < minb) break;
+                k = cp;
+                ++e;
+            }
+            if (e - r >= 2 && k >= minb) {
+                grps.push_back(Group{r, e, k, 0});
+                r = e;
+            } else {
+                ++r;
+            }
+        }
+    }
+    if (!grps.empty()) {
+        // Group members' rows: their own blocks only. Then the groups' shared rows, first.
+        std::vector<int> member_group(R, -1);
+        for (int gi = 0; gi < (int)grps.size(); ++gi)
+            for (int r = grps[gi].r0; r < grps[gi].r1; ++r) member_group[r] = gi;
+        for (CoreRow& c : core_rows) {
+            const int gi = member_group[c.req];
+            if (gi < 0) continue;
+            c.kind = 2;
+            c.group = gi;
+            c.j = c.req - grps[gi].r0;
+            c.bs = grps[gi].k;
+        }
+        std::vector<CoreRow> shared;
+        for (int gi = 0; gi < (int)grps.size(); ++gi) {
+            Group& g = grps[gi];
+            g.first_core = (int)shared.size();
+            const int m = g.r1 - g.r0;
+            for (int j = 0; j < m; j += rpi)
+                shared.push_back(CoreRow{qsl[g.r0] + j, g.r0, g.k * kBlockSize, std::min(rpi, m - j), 0, g.k, 1, gi, j});
+        }
+        core_rows.insert(core_rows.begin(), shared.begin(), shared.end());
+    }
+
     // Chunk length: enough items for ~4 per resident warp, but never below 8 blocks.
     const int groups = (int)ceil_div(G, hpi);
     int64_t total_blocks = 0;
-    for (const CoreRow& c : core_rows) total_blocks += ceil_div(c.limit + c.nrows - 1, kBlockSize) * Hkv * groups;
+    for (const CoreRow& c : core_rows) total_blocks += (int64_t)(c.be - c.bs) * Hkv * groups;
     int chunk;
     if (o.no_split) chunk = 1 << 30;
     else if (o.split_blocks > 0) chunk = o.split_blocks;
@@ -156,26 +222,27 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
         const int64_t workers = (int64_t)std::max(num_sms, 1) * 8;
         chunk = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(total_blocks, workers * 4), 8), 1 << 20);
     }
+    auto pieces_of = [&](const CoreRow& c) { return (int)ceil_div(c.be - c.bs, chunk); };
+    auto with_partials = [&](const CoreRow& c, int pieces) { return c.kind != 0 || pieces > 1; };
     // Items are placed directly at their position in a stable order by length, longest first:
     // this balances the static round-robin over the persistent warps. Pass 1 counts the items of
     // each length from the row lengths alone; pass 2 writes every item to its slot.
     size_t n_items = 0, n_merge = 0;
     int max_len = 0;
     for (const CoreRow& c : core_rows) {
-        const int nb = (int)ceil_div(c.limit + c.nrows - 1, kBlockSize);
-        const int pieces = (int)ceil_div(nb, chunk);
+        const int pieces = pieces_of(c);
         n_items += (size_t)pieces * Hkv * groups;
-        if (pieces > 1) n_merge += (size_t)Hkv * groups;
-        max_len = std::max(max_len, std::min(nb, chunk));
+        if (c.kind == 2 || (c.kind == 0 && pieces > 1)) n_merge += (size_t)Hkv * groups;
+        max_len = std::max(max_len, std::min(c.be - c.bs, chunk));
     }
     std::vector<size_t>& start = L->start;
     start.assign((size_t)max_len + 2, 0);
     for (const CoreRow& c : core_rows) {
-        const int nb = (int)ceil_div(c.limit + c.nrows - 1, kBlockSize);
-        const int pieces = (int)ceil_div(nb, chunk);
+        const int pieces = pieces_of(c);
+        if (pieces == 0) continue;
         const size_t per = (size_t)Hkv * groups;
-        start[std::min(nb, chunk)] += per * (pieces > 1 ? pieces - 1 : 1);
-        if (pieces > 1) start[nb - (pieces - 1) * chunk] += per;
+        start[std::min(c.be - c.bs, chunk)] += per * (pieces > 1 ? pieces - 1 : 1);
+        if (pieces > 1) start[(c.be - c.bs) - (pieces - 1) * chunk] += per;
     }
     size_t acc = 0;
     for (int len = max_len; len >= 1; --len) {
@@ -190,22 +257,38 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     size_t* pos = start.data();
     size_t mi = 0;
     int partials = 0;
-    for (const CoreRow& c : core_rows) {
-        const int nb = (int)ceil_div(c.limit + c.nrows - 1, kBlockSize);
-        const int pieces = (int)ceil_div(nb, chunk);
+    // First partial entry of each (shared row, KV head, head group): members' merges point there.
+    std::vector<int>& shared_first = L->shared_first;
+    shared_first.clear();
+    for (int ci = 0; ci < (int)core_rows.size(); ++ci) {
+        const CoreRow& c = core_rows[ci];
+        const int pieces = pieces_of(c);
         for (int h = 0; h < Hkv; ++h)
             for (int g0 = 0; g0 < G; g0 += hpi) {
+                const int nh = std::min(hpi, G - g0);
                 int first = -1;
-                if (pieces > 1) {
+                if (with_partials(c, pieces)) {
                     first = partials;
                     partials += pieces;
-                    const int nh = std::min(hpi, G - g0);
-                    merges[mi++] = MergeRow{c.row, h * G + g0, nh * c.nrows, first, pieces, nh, {0, 0}};
+                }
+                if (c.kind == 1) {
+                    shared_first.push_back(first);
+                } else if (c.kind == 2 || pieces > 1) {
+                    int xf = -1, xc = 0, xs = 0;
+                    if (c.kind == 2) {
+                        const Group& g = grps[c.group];
+                        const CoreRow& sc = core_rows[g.first_core + c.j / rpi];
+                        xf = shared_first[((size_t)(g.first_core + c.j / rpi) * Hkv + h) * groups + g0 / hpi];
+                        xc = pieces_of(sc);
+                        xs = (c.j - sc.j) * nh;
+                    }
+                    merges[mi++] = MergeRow{c.row, h * G + g0, nh * c.nrows, first, first >= 0 ? pieces : 0, nh, xf, xc, xs,
+                                            {0, 0, 0}};
                 }
                 for (int p = 0; p < pieces; ++p) {
-                    const int b0 = p * chunk, b1 = std::min(nb, b0 + chunk);
+                    const int b0 = c.bs + p * chunk, b1 = std::min(c.be, b0 + chunk);
                     items[pos[b1 - b0]++] = DecodeItem{c.row, c.req, (int16_t)h, (int16_t)c.nrows, g0, b0, b1, c.limit,
-                                                       pieces > 1 ? first + p : -1};
+                                                       first >= 0 ? first + p : -1};
                 }
             }
     }

@@ -396,7 +396,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
     }
 }
 
-// One warp per (merge row, slot): out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
+// One warp per (merge row, slot): out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i over the row's
+// partials -- its own chunks and, for a request sharing its leading blocks with others, the shared
+// items' chunks. A chunk that saw no key of a slot has m = -inf and weight 0.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
     constexpr int PER = D / 32;
@@ -408,15 +410,19 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
     if (entry >= a.num_rows) return;
     const MergeRow mr = a.rows[entry];
     if (g >= mr.num_slots) return;
+    const int total = mr.count + (mr.extra_first >= 0 ? mr.extra_count : 0);
+    auto slot_of = [&](int i) -> size_t {
+        return i < mr.count ? (size_t)(mr.first_partial + i) * a.part_stride + g
+                            : (size_t)(mr.extra_first + i - mr.count) * a.part_stride + mr.extra_slot + g;
+    };
     float M = -INFINITY;
-    for (int i = 0; i < mr.count; ++i)
-        M = fmaxf(M, a.part_ml[((size_t)(mr.first_partial + i) * a.part_stride + g) * 2]);
+    for (int i = 0; i < total; ++i) M = fmaxf(M, a.part_ml[slot_of(i) * 2]);
     float L = 0.f;
     float o[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) o[e] = 0.f;
-    for (int i = 0; i < mr.count; ++i) {
-        const size_t p = (size_t)(mr.first_partial + i) * a.part_stride + g;
+    for (int i = 0; i < total; ++i) {
+        const size_t p = slot_of(i);
         const float w = fast_exp2(a.part_ml[p * 2] - M);
         L = fmaf(w, a.part_ml[p * 2 + 1], L);
         const float* po = a.part_o + p * D + lane * PER;

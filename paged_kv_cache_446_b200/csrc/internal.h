@@ -43,18 +43,24 @@ struct PrefillTile {
 };
 static_assert(sizeof(PrefillTile) == 16, "PrefillTile layout");
 
-// The (row, head) slots of one chunked item whose partials the log-sum-exp merge combines:
-// slot s is query row row + s / heads_per_row, query head q_head0 + s % heads_per_row.
+// The (row, head) slots of one item whose partials the log-sum-exp merge combines: slot s is
+// query row row + s / heads_per_row, query head q_head0 + s % heads_per_row. Its partials are the
+// entries first_partial .. first_partial + count - 1 (slot s of each) and, for a request whose
+// leading blocks are shared with others, the shared items' entries extra_first ..
+// extra_first + extra_count - 1 (slot extra_slot + s of each).
 struct MergeRow {
     int32_t row;
     int32_t q_head0;       // first query head
-    int32_t num_slots;     // (row, head) slots in this entry (<= 8)
-    int32_t first_partial; // partial slots first_partial .. first_partial + count - 1
+    int32_t num_slots;     // (row, head) slots in this entry (<= 16)
+    int32_t first_partial;
     int32_t count;
     int32_t heads_per_row;
-    int32_t pad[2];
+    int32_t extra_first;   // -1 when there are no shared partials
+    int32_t extra_count;
+    int32_t extra_slot;
+    int32_t pad[3];
 };
-static_assert(sizeof(MergeRow) == 32, "MergeRow layout");
+static_assert(sizeof(MergeRow) == 48, "MergeRow layout");
 
 struct DecodeArgs {
     const void* q;

@@ -38,7 +38,9 @@ _SZ = ctypes.c_size_t
 class PlanOptions(ctypes.Structure):
     _fields_ = [("split_blocks", ctypes.c_int32), ("no_split", ctypes.c_int32),
                 ("cuda_core_only", ctypes.c_int32), ("num_sms", ctypes.c_int32), ("heads_per_item", ctypes.c_int32),
-                ("rows_per_item", ctypes.c_int32), ("tc_min_rows", ctypes.c_int32), ("decode_kernel", ctypes.c_int32)]
+                ("rows_per_item", ctypes.c_int32), ("tc_min_rows", ctypes.c_int32), ("decode_kernel", ctypes.c_int32),
+                ("h_block_tables", ctypes.c_void_p), ("block_table_stride", ctypes.c_int32),
+                ("min_shared_blocks", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):
@@ -118,9 +120,17 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _opts(split_blocks=0, no_split=False, cuda_core_only=False, num_sms=0, heads_per_item=0, rows_per_item=0,
-          tc_min_rows=0, decode_kernel=0) -> PlanOptions:
-    return PlanOptions(int(split_blocks), int(bool(no_split)), int(bool(cuda_core_only)), int(num_sms),
-                       int(heads_per_item), int(rows_per_item), int(tc_min_rows), int(decode_kernel))
+          tc_min_rows=0, decode_kernel=0, shared_tables=None, min_shared_blocks=0) -> PlanOptions:
+    """Planner options. shared_tables: host int32 block tables [R, max_blocks] for shared-prefix
+    detection (the caller keeps the array alive while planning), or None."""
+    o = PlanOptions(int(split_blocks), int(bool(no_split)), int(bool(cuda_core_only)), int(num_sms),
+                    int(heads_per_item), int(rows_per_item), int(tc_min_rows), int(decode_kernel))
+    if shared_tables is not None:
+        assert shared_tables.dtype == np.int32 and shared_tables.flags["C_CONTIGUOUS"] and shared_tables.ndim == 2
+        o.h_block_tables = shared_tables.ctypes.data
+        o.block_table_stride = int(shared_tables.shape[1])
+    o.min_shared_blocks = int(min_shared_blocks)
+    return o
 
 
 # ---- a13: mixed-batch flattening -------------------------------------------------------------
@@ -177,6 +187,8 @@ def plan_host(query_start_loc: np.ndarray, context_lens: np.ndarray, num_q_heads
     qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
     ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
     plan = Plan()
+    if opts.get("shared_tables") is not None:
+        opts = dict(opts, shared_tables=np.ascontiguousarray(opts["shared_tables"], dtype=np.int32))
     o = _opts(**opts)
     _check(_plan_host(_np_ptr(qsl), _np_ptr(ctx), ctx.shape[0], num_q_heads, num_kv_heads, head_dim,
                       DTYPE_NAME[dtype], ctypes.byref(o), None, 0, ctypes.byref(plan)), "pkv_attention_plan_host")
@@ -201,7 +213,9 @@ class AttentionPlan:
                  dtype: torch.dtype, device, workspace: torch.Tensor | None = None, stream=None, **opts):
         self.num_q_heads, self.num_kv_heads, self.head_dim, self.dtype = num_q_heads, num_kv_heads, head_dim, dtype
         self.device = torch.device(device)
-        self.opts = _opts(**opts)
+        shared = opts.pop("shared_tables", None)
+        self._shared = None if shared is None else np.ascontiguousarray(shared, dtype=np.int32)
+        self.opts = _opts(shared_tables=self._shared, **opts)
         if self.opts.num_sms == 0:
             self.opts.num_sms = torch.cuda.get_device_properties(self.device).multi_processor_count
         self.workspace = workspace
@@ -212,9 +226,14 @@ class AttentionPlan:
         self._uploaded = None   # event after the last upload from the pinned buffers
         self.replan(batch, prior_lens, stream=stream)
 
-    def replan(self, batch: dict, prior_lens, stream=None) -> "AttentionPlan":
+    def replan(self, batch: dict, prior_lens, stream=None, shared_tables=None) -> "AttentionPlan":
         """Plans the batch on the host (pkv_attention_plan_host) into pinned memory and uploads the
-        work lists and the batch description with asynchronous copies on `stream`."""
+        work lists and the batch description with asynchronous copies on `stream`. shared_tables:
+        the batch's host block tables, when they changed (for shared-prefix detection)."""
+        if shared_tables is not None:
+            self._shared = np.ascontiguousarray(shared_tables, dtype=np.int32)
+            self.opts.h_block_tables = self._shared.ctypes.data
+            self.opts.block_table_stride = int(self._shared.shape[1])
         qsl, ctx = flatten_batch(batch, prior_lens)
         self.h_query_start_loc, self.h_context_lens = qsl, ctx
         self.num_q_tokens = int(qsl[-1])

@@ -25,6 +25,9 @@ class PagedAttentionStep:
         self.num_blocks = int(num_blocks)
         self.dtype = dtype
         self.block_tables = torch.from_numpy(np.ascontiguousarray(block_tables, dtype=np.int32)).to(self.device)
+        # The host tables let the planner read blocks shared by several requests once.
+        if plan_opts.pop("share_prefixes", True):
+            plan_opts.setdefault("shared_tables", np.ascontiguousarray(block_tables, dtype=np.int32))
         self.plan = pkv.AttentionPlan(batch, prior_lens, num_q_heads, num_kv_heads, head_dim, dtype, self.device,
                                       stream=stream, **plan_opts)
         # The write batch shares the requests and their context after the step; its rows are the

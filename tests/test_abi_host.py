@@ -97,64 +97,57 @@ def test_planner_rejects(pkv, bad):
 def parse_meta(plan, meta):
     items = np.frombuffer(meta[plan.off_items:plan.off_items + 32 * plan.num_items].tobytes(), np.int32)
     tiles = np.frombuffer(meta[plan.off_tiles:plan.off_tiles + 16 * plan.num_tiles].tobytes(), np.int32)
-    merges = np.frombuffer(meta[plan.off_merge:plan.off_merge + 32 * plan.num_merge_rows].tobytes(), np.int32)
-    return items.reshape(-1, 8), tiles.reshape(-1, 4), merges.reshape(-1, 8)
+    merges = np.frombuffer(meta[plan.off_merge:plan.off_merge + 48 * plan.num_merge_rows].tobytes(), np.int32)
+    return items.reshape(-1, 8), tiles.reshape(-1, 4), merges.reshape(-1, 12)
 
 
-@pytest.mark.parametrize("seed", range(6))
-@pytest.mark.parametrize("opts", [{}, {"split_blocks": 1}, {"split_blocks": 3}, {"no_split": True},
-                                  {"cuda_core_only": True}, {"heads_per_item": 4}, {"heads_per_item": 3},
-                                  {"cuda_core_only": True, "split_blocks": 2}, {"tc_min_rows": 9},
-                                  {"cuda_core_only": True, "rows_per_item": 1},
-                                  {"cuda_core_only": True, "rows_per_item": 3, "heads_per_item": 2},
-                                  {"decode_kernel": 1}, {"decode_kernel": 2, "tc_min_rows": 9},
-                                  {"decode_kernel": 2, "heads_per_item": 16, "split_blocks": 2}])
-def test_planner_covers_every_block_once(pkv, seed, opts):
-    """Every (row, query head, visible KV block) is covered by exactly one work item or tile."""
-    rng = np.random.default_rng(seed)
-    R = int(rng.integers(1, 12))
-    n = rng.choice([0, 1, 1, 1, 2, 4, 5, 8, 37, 130], size=R)
-    prior = rng.integers(0, 300, size=R)
-    ctx = (prior + n).astype(np.int32)
-    ctx[(n == 0) & (rng.random(R) < 0.5)] = 0
-    qsl = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
-    Hq, Hkv = [(8, 8), (32, 8), (64, 8), (32, 2), (6, 3)][seed % 5]
-    dtype = ["f16", "bf16", "f32"][seed % 3]
-    if opts.get("decode_kernel") == 2 and dtype == "f32":
-        with pytest.raises(pkv.PkvError):
-            pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, **opts)
-        return
-    plan, meta = pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, **opts)
-    if plan.num_items:
-        assert plan.decode_kernel in (1, 2) and 1 <= plan.part_stride <= (16 if plan.decode_kernel == 2 else 8)
-        if "decode_kernel" in opts:
-            assert plan.decode_kernel == opts["decode_kernel"]
+def check_plan(pkv, plan, meta, qsl, ctx, Hq, Hkv, opts, dtype, tables=None):
+    """Every (row, query head, visible KV block) is covered by exactly one work item or tile, each
+    item shows a row exactly the keys the row sees, and every partial result an item writes is read
+    by exactly one merge slot, for that same (row, head)."""
     items, tiles, merges = parse_meta(plan, meta)
+    R = len(ctx)
     G = Hq // Hkv
     hpi = plan.heads_per_item
-    cover = {}
+    req_of_row = np.repeat(np.arange(R), np.diff(qsl))
+
+    def true_limit(row):
+        r = req_of_row[row]
+        return r, int(ctx[r] - (qsl[r + 1] - qsl[r]) + (row - qsl[r]) + 1)
+
+    cover, written = {}, {}
     max_rows = 0
-    for row, req, packed, head0, b0, b1, limit, part in items:
+    for row0, req, packed, head0, b0, b1, limit, part in items:
         kvh, nrows = packed & 0xFFFF, packed >> 16
-        assert 1 <= nrows and nrows * min(hpi, G - head0) <= plan.part_stride <= 16
+        nh = min(hpi, G - head0)
+        assert 1 <= nrows and nrows * nh <= plan.part_stride <= 16
         max_rows = max(max_rows, nrows)
-        nreq = qsl[req + 1] - qsl[req]
-        assert qsl[req] <= row and row + nrows <= qsl[req + 1]
-        j = row - qsl[req]
-        assert limit == ctx[req] - nreq + j + 1
-        assert 0 <= b0 < b1 <= -(-(limit + nrows - 1) // 16)
+        assert 0 <= b0 < b1
         for jr in range(nrows):
-            visible = -(-(limit + jr) // 16)
-            for h in range(head0, min(G, head0 + hpi)):
-                for b in range(b0, min(b1, visible)):
-                    key = (row + jr, kvh * G + h, b)
+            row = row0 + jr
+            r, L = true_limit(row)
+            for b in range(b0, b1):
+                seen_by_kernel = min(max(limit + jr - 16 * b, 0), 16)
+                seen_by_row = min(max(L - 16 * b, 0), 16)
+                assert seen_by_kernel == seen_by_row, (row, b, limit, jr, L)
+                if seen_by_row == 0:
+                    continue
+                if tables is not None:
+                    assert tables[req, b] == tables[r, b], "item reads another request's block"
+                elif nrows > 1 or req != r:
+                    assert req == r
+                for h in range(head0, head0 + nh):
+                    key = (row, kvh * G + h, b)
                     cover[key] = cover.get(key, 0) + 1
+            if part >= 0:
+                for hh in range(nh):
+                    written[(part, jr * nh + hh)] = (row, kvh * G + head0 + hh)
     assert plan.rows_per_item == max_rows
     if "rows_per_item" in opts:
         assert max_rows <= opts["rows_per_item"]
-    tile_rows = 2 * (128 // G)      # two 128-row MMA tiles per CTA
     mma_ok = dtype != "f32" and opts.get("decode_kernel") != 1
     tc_min = opts.get("tc_min_rows") or (max(2, 16 // G + 1) if mma_ok else 2)
+    tile_rows = 2 * (128 // G)      # two 128-row MMA tiles per CTA
     for req, kvh, tok0, _ in tiles:
         nreq = qsl[req + 1] - qsl[req]
         assert nreq >= tc_min
@@ -173,20 +166,104 @@ def test_planner_covers_every_block_once(pkv, seed, opts):
                 for b in range(-(-limit // 16)):
                     expect[(qsl[r] + j, h, b)] = 1
     assert cover == expect
-    # Partials: every partial slot belongs to exactly one merge row, and chunked items point into it.
-    owners = {}
-    for row, qh0, nslots, first, count, hpr, *_ in merges:
-        for p in range(first, first + count):
-            assert p not in owners
-            owners[p] = (row, qh0, nslots, hpr)
-    assert len(owners) == plan.num_partials
-    for row, req, packed, head0, b0, b1, limit, part in items:
-        kvh, nrows = packed & 0xFFFF, packed >> 16
-        if part >= 0:
-            nh = min(hpi, G - head0)
-            assert owners[part] == (row, kvh * G + head0, nh * nrows, nh)
-    if opts.get("no_split"):
+    read = {}
+    for row, qh0, nslots, first, count, hpr, xf, xc, xs, *_ in merges:
+        for g in range(nslots):
+            target = (row + g // hpr, qh0 + g % hpr)
+            srcs = [(first + i, g) for i in range(count)] + ([(xf + i, xs + g) for i in range(xc)] if xf >= 0 else [])
+            assert srcs
+            for src in srcs:
+                assert src not in read
+                read[src] = target
+    assert read == written
+    if opts.get("no_split") and tables is None:
         assert plan.num_merge_rows == 0
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("opts", [{}, {"split_blocks": 1}, {"split_blocks": 3}, {"no_split": True},
+                                  {"cuda_core_only": True}, {"heads_per_item": 4}, {"heads_per_item": 3},
+                                  {"cuda_core_only": True, "split_blocks": 2}, {"tc_min_rows": 9},
+                                  {"cuda_core_only": True, "rows_per_item": 1},
+                                  {"cuda_core_only": True, "rows_per_item": 3, "heads_per_item": 2},
+                                  {"decode_kernel": 1}, {"decode_kernel": 2, "tc_min_rows": 9},
+                                  {"decode_kernel": 2, "heads_per_item": 16, "split_blocks": 2}])
+def test_planner_covers_every_block_once(pkv, seed, opts):
+    rng = np.random.default_rng(seed)
+    R = int(rng.integers(1, 12))
+    n = rng.choice([0, 1, 1, 1, 2, 4, 5, 8, 37, 130], size=R)
+    prior = rng.integers(0, 300, size=R)
+    ctx = (prior + n).astype(np.int32)
+    ctx[(n == 0) & (rng.random(R) < 0.5)] = 0
+    qsl = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    Hq, Hkv = [(8, 8), (32, 8), (64, 8), (32, 2), (6, 3)][seed % 5]
+    dtype = ["f16", "bf16", "f32"][seed % 3]
+    if opts.get("decode_kernel") == 2 and dtype == "f32":
+        with pytest.raises(pkv.PkvError):
+            pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, **opts)
+        return
+    plan, meta = pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, **opts)
+    if plan.num_items:
+        assert plan.decode_kernel in (1, 2) and 1 <= plan.part_stride <= (16 if plan.decode_kernel == 2 else 8)
+        if "decode_kernel" in opts:
+            assert plan.decode_kernel == opts["decode_kernel"]
+    check_plan(pkv, plan, meta, qsl, ctx, Hq, Hkv, opts, dtype)
+
+
+def shared_prefix_batch(rng, groups, lone):
+    """Decode requests in runs that share leading blocks (forks of a prompt), plus lone requests,
+    shuffled as whole runs; tables over a pool of distinct ids except for the shared blocks."""
+    runs = []
+    next_id = 0
+    for size, shared in groups:
+        ids = list(range(next_id, next_id + shared))
+        next_id += shared
+        run = []
+        for _ in range(size):
+            own = int(rng.integers(0, 40))
+            run.append((ids, own))
+        runs.append(run)
+    for _ in range(lone):
+        runs.append([([], int(rng.integers(1, 200)))])
+    order = rng.permutation(len(runs))
+    reqs = [req for i in order for req in runs[i]]
+    ctxs, rows = [], []
+    for ids, own in reqs:
+        c = 16 * len(ids) + own
+        c = max(c, 1)
+        nb = -(-c // 16)
+        row = list(ids) + list(range(next_id, next_id + nb - len(ids)))
+        next_id += nb - len(ids)
+        ctxs.append(c)
+        rows.append(row)
+    width = max(len(r) for r in rows)
+    tables = np.full((len(rows), width), -1, np.int32)
+    for i, row in enumerate(rows):
+        tables[i, :len(row)] = row
+    return np.array(ctxs, np.int32), tables
+
+
+@pytest.mark.parametrize("seed", range(5))
+@pytest.mark.parametrize("opts", [{}, {"split_blocks": 1}, {"split_blocks": 5}, {"no_split": True},
+                                  {"decode_kernel": 1}, {"heads_per_item": 2}, {"min_shared_blocks": 2}])
+def test_planner_shared_prefixes(pkv, seed, opts):
+    """Runs of decode requests that share leading blocks read them through shared items; coverage,
+    visibility, table consistency and merge wiring all hold."""
+    rng = np.random.default_rng(100 + seed)
+    ctx, tables = shared_prefix_batch(rng, [(8, 5), (3, 12), (2, 1), (5, 4)], lone=4)
+    R = len(ctx)
+    qsl = np.arange(R + 1, dtype=np.int32)
+    Hq, Hkv = [(32, 8), (64, 8), (8, 8), (32, 2), (6, 3)][seed % 5]
+    dtype = ["f16", "bf16", "f32"][seed % 3]
+    if opts.get("decode_kernel") == 2 and dtype == "f32":
+        return
+    plan, meta = pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, shared_tables=tables, **opts)
+    check_plan(pkv, plan, meta, qsl, ctx, Hq, Hkv, opts, dtype, tables=tables)
+    base, _ = pkv.plan_host(qsl, ctx, Hq, Hkv, 128, dtype, **opts)
+    items, _, _ = parse_meta(plan, meta)
+    if plan.heads_per_item * 2 <= (16 if plan.decode_kernel == 2 else 8):
+        assert max(it[2] >> 16 for it in items) > 1          # shared items pack several requests' rows
+    assert plan.kv_bytes == base.kv_bytes
 
 
 def test_workspace_size_matches_plan(pkv):

@@ -327,3 +327,26 @@ def test_attend_one_call(dev):
     torch.cuda.synchronize()
     err = max_err(out, oracle_step(wl, h))
     assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("opts", [{}, {"split_blocks": 1}, {"no_split": True}, {"share_prefixes": False}],
+                         ids=["auto", "split1", "nosplit", "no-sharing"])
+@pytest.mark.parametrize("dtype,Hq,Hkv", [("f16", 32, 8), ("bf16", 64, 8), ("bf16", 16, 16)])
+def test_shared_prefix_items(dev, dtype, Hq, Hkv, opts, kernel):
+    """Runs of decode requests sharing their leading blocks (one item set reads the shared blocks
+    for all of them, merged by log-sum-exp with each request's own blocks) against the oracle."""
+    from test_abi_host import shared_prefix_batch
+    rng = np.random.default_rng(61)
+    ctx, tables = shared_prefix_batch(rng, [(8, 5), (3, 12), (2, 1), (5, 4)], lone=4)
+    R = len(ctx)
+    NB = int(tables.max()) + 1
+    wl = W.Workload(name="shared", dtype=dtype, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=128,
+                    scale=float(np.float32(1 / math.sqrt(128))), batch={r: 1 for r in range(R)},
+                    prior_lens=(ctx - 1).astype(np.int32), block_tables=tables, num_blocks=NB,
+                    write_batch={}, copy_pairs=np.zeros((0, 2), np.int32), seed=61)
+    W._draw_tensors(wl, dev)
+    _, step = run_and_compare(wl, dev, decode_kernel=kernel, **opts)
+    slots = 16 if kernel == 2 else 8
+    if not opts and slots // min(Hq // Hkv, slots) >= 2:
+        assert step.plan.plan.rows_per_item > 1     # shared items pack several requests' rows
