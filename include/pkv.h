@@ -164,7 +164,8 @@ typedef struct pkv_plan {
                                     2*D*elem per (kv head, key), counted once per (request, kv head)
                                     for decode rows and once per request for prefill rows */
     int64_t attn_flops;          /* 4*D per (query row, query head, attended key) */
-    int64_t core_kv_bytes;       /* part of kv_bytes read by the CUDA-core kernel */
+    int64_t core_kv_bytes;       /* K+V bytes the CUDA-core kernel must read: its requests' contexts,
+                                    with a prefix shared by a run of requests counted once */
     int64_t tile_kv_bytes;       /* part of kv_bytes read by the tcgen05 tiles */
     int64_t tile_flops;          /* part of attn_flops computed by the tcgen05 tiles */
 } pkv_plan;

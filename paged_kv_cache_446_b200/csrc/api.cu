@@ -344,7 +344,10 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->ws_bytes = off;
     plan->kv_bytes = kv_bytes;
     plan->attn_flops = flops;
-    plan->core_kv_bytes = kv_bytes - tile_kv;
+    // K/V the CUDA-core kernel must read: a shared prefix once per group, not once per member.
+    int64_t shared_saved_tokens = 0;
+    for (const Group& g : grps) shared_saved_tokens += (int64_t)(g.r1 - g.r0 - 1) * g.k * kBlockSize;
+    plan->core_kv_bytes = kv_bytes - tile_kv - shared_saved_tokens * Hkv * 2 * D * eb;
     plan->tile_kv_bytes = tile_kv;
     plan->tile_flops = tile_flops;
     return PKV_OK;
