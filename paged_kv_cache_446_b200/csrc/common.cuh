@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
 #include <utility>
 
 #include "internal.h"
@@ -198,6 +199,44 @@ struct Chunk<__nv_bfloat16> {
 };
 
 __device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// Two fp32 values rounded (to nearest even) to a 16-bit type T and packed, `lo` in the low half.
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    if constexpr (std::is_same<T, __half>::value) {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+}
+// The two 16-bit values of a packed word as fp32 (low half first).
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+    if constexpr (std::is_same<T, __half>::value) {
+        return __half22float2(*reinterpret_cast<const __half2*>(&w));
+    } else {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+}
+
+// A CUDA-core work item, read with two 16-byte loads.
+__device__ __forceinline__ DecodeItem load_item(const DecodeItem* items, int i) {
+    const int4* p = reinterpret_cast<const int4*>(items + i);
+    const int4 a = __ldg(p), b = __ldg(p + 1);
+    DecodeItem it;
+    it.row = a.x;
+    it.req = a.y;
+    it.kv_head = (int16_t)(a.z & 0xffff);         // low half of the third word
+    it.num_rows = (int16_t)((unsigned)a.z >> 16); // high half
+    it.head0 = a.w;
+    it.blk_begin = b.x;
+    it.blk_end = b.y;
+    it.limit = b.z;
+    it.partial = b.w;
+    return it;
+}
 
 // ---- programmatic dependent launch -------------------------------------------------------------
 // Kernels are launched so that they may start while the previous kernel on the stream finishes;

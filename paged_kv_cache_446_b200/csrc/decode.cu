@@ -66,18 +66,6 @@ constexpr int kDecodeWarps = 2;  // independent warps per CTA
 template <int GP>
 constexpr int default_stages() { return GP >= 4 ? 2 : 3; }
 
-__device__ __forceinline__ DecodeItem load_item(const DecodeItem* items, int i) {
-    const int4* p = reinterpret_cast<const int4*>(items + i);
-    const int4 a = __ldg(p), b = __ldg(p + 1);
-    DecodeItem it;
-    it.row = a.x; it.req = a.y;
-    it.kv_head = (int16_t)(a.z & 0xffff);                   // low half of the third word
-    it.num_rows = (int16_t)((unsigned)a.z >> 16);           // high half
-    it.head0 = a.w;
-    it.blk_begin = b.x; it.blk_end = b.y; it.limit = b.z; it.partial = b.w;
-    return it;
-}
-
 template <typename T, int D, int GP, int NSTAGE>
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeArgs a) {
     using C = Dec<T, D, GP, NSTAGE>;

@@ -45,18 +45,6 @@ constexpr int kStage = kKV + kQ;               // 12 KiB, a multiple of the 1 Ki
 template <int NSTAGE>
 constexpr int smem_bytes() { return 1024 + kMmaWarps * NSTAGE * (kStage + 8); }
 
-__device__ __forceinline__ DecodeItem load_item_mma(const DecodeItem* items, int i) {
-    const int4* p = reinterpret_cast<const int4*>(items + i);
-    const int4 a = __ldg(p), b = __ldg(p + 1);
-    DecodeItem it;
-    it.row = a.x; it.req = a.y;
-    it.kv_head = (int16_t)(a.z & 0xffff);
-    it.num_rows = (int16_t)((unsigned)a.z >> 16);
-    it.head0 = a.w;
-    it.blk_begin = b.x; it.blk_end = b.y; it.limit = b.z; it.partial = b.w;
-    return it;
-}
-
 // Byte offset, inside a 16-row chunk stored as two 64-column halves with the 128-byte swizzle, of
 // the 16 bytes holding columns [8 * col8, 8 * col8 + 8) of row r (col8 in 0..15).
 __device__ __forceinline__ uint32_t sw_off(int r, int col8) {
@@ -94,28 +82,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
     }
 }
 
-// The two 16-bit values of a packed word as fp32 (low half first).
-template <typename T>
-__device__ __forceinline__ float2 unpack2(uint32_t w) {
-    if constexpr (std::is_same<T, __half>::value) {
-        return __half22float2(*reinterpret_cast<const __half2*>(&w));
-    } else {
-        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-    }
-}
-
-// Two fp32 values rounded to the 16-bit type and packed, `lo` in the low half.
-template <typename T>
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-    if constexpr (std::is_same<T, __half>::value) {
-        const __half2 h = __floats2half2_rn(lo, hi);
-        return *reinterpret_cast<const uint32_t*>(&h);
-    } else {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-        return *reinterpret_cast<const uint32_t*>(&h);
-    }
-}
-
 template <typename T, int NSTAGE>
 __global__ void __launch_bounds__(kMmaWarps * 32)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
@@ -141,7 +107,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32)
 
     // ---------------- producer (lane 0 issues; runs up to NSTAGE blocks ahead) ----------------
     int p_it = gw;
-    DecodeItem pi = load_item_mma(a.items, p_it);
+    DecodeItem pi = load_item(a.items, p_it);
     int p_blk = pi.blk_begin;
     int p_base = p_blk;
     int p_ids = (p_blk + lane < pi.blk_end) ? __ldg(a.block_tables + (size_t)pi.req * a.max_blocks_per_seq + p_blk + lane) : 0;
@@ -180,7 +146,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32)
         if (p_blk == pi.blk_end) {
             p_it += W;
             if (p_it < a.num_items) {
-                pi = load_item_mma(a.items, p_it);
+                pi = load_item(a.items, p_it);
                 p_blk = pi.blk_begin;
                 p_base = p_blk;
                 p_ids = (p_blk + lane < pi.blk_end)
@@ -199,7 +165,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32)
 
     // ---------------- consumer (the whole warp) ----------------
     int c_it = gw;
-    DecodeItem ci = load_item_mma(a.items, c_it);
+    DecodeItem ci = load_item(a.items, c_it);
     int c_blk = ci.blk_begin;
     uint32_t consumed = 0;
 
@@ -372,7 +338,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32)
             }
             c_it += W;
             if (c_it >= a.num_items) break;
-            ci = load_item_mma(a.items, c_it);
+            ci = load_item(a.items, c_it);
             c_blk = ci.blk_begin;
         } else {
             ++c_blk;

@@ -160,25 +160,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // Warp-uniform "all succeeded" for the lanes of one warp.
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(FULL_MASK, v); }
 
-template <typename T>
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-    if constexpr (std::is_same<T, __half>::value) {
-        const __half2 h = __floats2half2_rn(a, b);
-        return *reinterpret_cast<const uint32_t*>(&h);
-    } else {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-        return *reinterpret_cast<const uint32_t*>(&h);
-    }
-}
-// Inverse of pack2: the two 16-bit values of a packed word as fp32 (low half first).
-template <typename T>
-__device__ __forceinline__ float2 unpack2(uint32_t w) {
-    if constexpr (std::is_same<T, __half>::value) {
-        return __half22float2(*reinterpret_cast<const __half2*>(&w));
-    } else {
-        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-    }
-}
 // What a pair of softmax weights adds to the row sum. PV uses the weights rounded to T; for fp16
 // the sum takes them as rounded too, so that the normalisation matches the numerator exactly (an
 // fp16 output of magnitude 4..8 has a rounding step of ~2e-3, which leaves no room for the
