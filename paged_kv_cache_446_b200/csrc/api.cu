@@ -353,11 +353,18 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     return PKV_OK;
 }
 
+// The work-list image: each list at its offset, the header and the alignment gaps zeroed.
 void write_meta(const PlanLists& L, const pkv_plan& plan, unsigned char* meta) {
-    std::memset(meta, 0, (size_t)plan.meta_bytes);
+    const size_t end_items = plan.off_items + L.items.size() * sizeof(DecodeItem);
+    const size_t end_tiles = plan.off_tiles + L.tiles.size() * sizeof(PrefillTile);
+    const size_t end_merge = plan.off_merge + L.merges.size() * sizeof(MergeRow);
+    std::memset(meta, 0, (size_t)plan.off_items);
     if (!L.items.empty()) std::memcpy(meta + plan.off_items, L.items.data(), L.items.size() * sizeof(DecodeItem));
+    std::memset(meta + end_items, 0, (size_t)plan.off_tiles - end_items);
     if (!L.tiles.empty()) std::memcpy(meta + plan.off_tiles, L.tiles.data(), L.tiles.size() * sizeof(PrefillTile));
+    std::memset(meta + end_tiles, 0, (size_t)plan.off_merge - end_tiles);
     if (!L.merges.empty()) std::memcpy(meta + plan.off_merge, L.merges.data(), L.merges.size() * sizeof(MergeRow));
+    std::memset(meta + end_merge, 0, (size_t)plan.meta_bytes - end_merge);
 }
 
 // Per-thread kernel timing state (pkv_profile_start / pkv_profile_stop).

@@ -138,7 +138,7 @@ def _opts(split_blocks=0, no_split=False, cuda_core_only=False, num_sms=0, heads
 def flatten_batch(batch: dict, prior_lens) -> tuple[np.ndarray, np.ndarray]:
     """{request_id: num_tokens} (dict order) + each request's prior context ->
     (query_start_loc int32 [R+1], context_lens int32 [R]) on the host."""
-    counts = np.fromiter((int(v) for v in batch.values()), dtype=np.int64, count=len(batch))
+    counts = np.fromiter(batch.values(), dtype=np.int64, count=len(batch))
     qsl = np.zeros(len(batch) + 1, dtype=np.int64)
     np.cumsum(counts, out=qsl[1:])
     ctx = np.asarray(prior_lens, dtype=np.int64).reshape(-1) + counts
