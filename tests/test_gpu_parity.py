@@ -350,3 +350,48 @@ def test_shared_prefix_items(dev, dtype, Hq, Hkv, opts, kernel):
     slots = 16 if kernel == 2 else 8
     if not opts and slots // min(Hq // Hkv, slots) >= 2:
         assert step.plan.plan.rows_per_item > 1     # shared items pack several requests' rows
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_mixed_batches(dev, seed):
+    """Seeded random batches: decode, verify and prefill rows mixed, random group sizes, dtypes,
+    chunkings and kernels, requests with no rows, against the oracle."""
+    rng = np.random.default_rng(700 + seed)
+    dtype = ["f16", "bf16", "f32"][seed % 3]
+    Hkv = int(rng.choice([1, 2, 4, 8]))
+    G = int(rng.choice([1, 2, 3, 4, 8, 16]))
+    D = 64 if (dtype == "f32" and seed % 2) else 128
+    R = int(rng.integers(1, 10))
+    specs = []
+    for _ in range(R):
+        n = int(rng.choice([0, 1, 1, 1, 2, 5, 16, 70]))
+        prior = int(rng.integers(0 if n else 1, 700))
+        specs.append((prior, n))
+    if all(n == 0 for _, n in specs):
+        specs[0] = (specs[0][0], 1)
+    opts = {}
+    if rng.random() < 0.5:
+        opts["split_blocks"] = int(rng.choice([1, 2, 7]))
+    if rng.random() < 0.3:
+        opts["tc_min_rows"] = int(rng.choice([2, 9, 64]))
+    if dtype != "f32" and D == 128 and rng.random() < 0.3:
+        opts["decode_kernel"] = int(rng.choice([1, 2]))
+    wl = custom(dev, dtype, Hkv * G, Hkv, D, specs, seed=700 + seed)
+    run_and_compare(wl, dev, **opts)
+
+
+def test_pool_too_large_for_tensor_maps_is_refused(dev):
+    """A pool whose rows (blocks x KV heads x 16) do not fit a 32-bit tensor-map coordinate is
+    refused at launch with a CUDA status, before any kernel runs."""
+    import ctypes
+    from paged_kv_cache_446_b200 import pkv
+    wl = custom(dev, "bf16", 16, 8, 128, [(40, 1), (10, 1)], seed=71)
+    step = make_step(wl, dev)
+    p = step.plan
+    huge_nb = (1 << 31) // (8 * 16) + 1
+    status = pkv._attention(pkv._ptr(wl.q), pkv._ptr(wl.q), pkv._ptr(wl.k_pool), pkv._ptr(wl.v_pool),
+                            pkv._ptr(step.block_tables), step.block_tables.shape[1], pkv._ptr(p.context_lens),
+                            pkv._ptr(p.query_start_loc), huge_nb, ctypes.c_float(wl.scale), ctypes.byref(p.plan),
+                            pkv._ptr(p.workspace), p.workspace.numel(), pkv._stream(None))
+    torch.cuda.synchronize()
+    assert status == 3
