@@ -378,12 +378,13 @@ cudaError_t launch_mma_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     return launch_pdl(decode_mma_kernel<T, NSTAGE>, dim3(grid), dim3(kMmaWarps * 32), smem, s, a, mk, mv);
 }
 
-// Ring depth: 3 stages, or PKV_DECODE_MMA_STAGES (2..4) as a tuning override.
+// Ring depth: 2 stages (24 KiB per warp, so 4 CTAs = 8 warps fit an SM; measured best on every
+// configuration against 3 and 4), or PKV_DECODE_MMA_STAGES (2..4) as a tuning override.
 inline int mma_stages() {
     static const int v = [] {
         const char* e = getenv("PKV_DECODE_MMA_STAGES");
         const int x = e ? atoi(e) : 0;
-        return (x >= 2 && x <= 4) ? x : 3;
+        return (x >= 2 && x <= 4) ? x : 2;
     }();
     return v;
 }
@@ -391,9 +392,9 @@ inline int mma_stages() {
 template <typename T>
 cudaError_t launch_mma_s(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     switch (mma_stages()) {
-        case 2: return launch_mma_t<T, 2>(a, num_sms, s);
+        case 3: return launch_mma_t<T, 3>(a, num_sms, s);
         case 4: return launch_mma_t<T, 4>(a, num_sms, s);
-        default: return launch_mma_t<T, 3>(a, num_sms, s);
+        default: return launch_mma_t<T, 2>(a, num_sms, s);
     }
 }
 
