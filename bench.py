@@ -3,7 +3,7 @@
 
 One step = one pass of the whole path over one batch of synthetic input: copy-on-write block
 copies (when the workload has shared blocks), slot mapping, KV append, then paged attention over
-the mixed batch (CUDA-core split-K kernel, tcgen05 prefill tiles when present, log-sum-exp merge).
+the mixed batch (split-K decode kernel, tcgen05 prefill tiles when present, log-sum-exp merge).
 The default workload is the LLaMA-13B-shaped fp16 decode batch (64 rows, 40/40 heads, head_dim
 128, context U[128,2048], one appended token per row). Its KV pool is ~1.4 GB, larger than the
 126 MB L2, so no explicit L2 flush is used between steps.
@@ -52,12 +52,12 @@ def parse():
     ap.add_argument("--part", default="all", choices=["all", "prefill", "decode"],
                     help="time only the prefill or decode requests of the workload")
     ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling subsets)")
-    ap.add_argument("--heads-per-item", type=int, default=0, help="query heads per CUDA-core work item")
-    ap.add_argument("--rows-per-item", type=int, default=0, help="query rows of a request per CUDA-core work item")
+    ap.add_argument("--heads-per-item", type=int, default=0, help="query heads per split-K work item")
+    ap.add_argument("--rows-per-item", type=int, default=0, help="query rows of a request per split-K work item")
     ap.add_argument("--tc-min-rows", type=int, default=0, help="fewest rows a request needs for the tcgen05 tiles")
     ap.add_argument("--cuda-core-only", action="store_true", help="serve every row on CUDA cores")
     ap.add_argument("--decode-kernel", type=int, default=0, choices=[0, 1, 2],
-                    help="kernel for CUDA-core rows: 0 planner's choice, 1 FMA, 2 warp MMA")
+                    help="kernel for split-K rows: 0 planner's choice, 1 FMA, 2 warp MMA")
     return ap.parse_args()
 
 
@@ -153,7 +153,7 @@ def pool_waste(wl) -> dict:
 
 
 def kernel_work(plan, wl) -> dict:
-    """Algorithmic work per launch from the plan: the CUDA-core kernel reads K+V of its requests'
+    """Algorithmic work per launch from the plan: the split-K kernel reads K+V of its requests'
     contexts once per (request, KV head) plus its q rows and writes its output rows; the tcgen05
     tiles likewise for theirs, and compute 4*D flops per (row, head, attended key)."""
     eb = 4 if wl.dtype == "f32" else 2
@@ -491,7 +491,7 @@ def main():
     # Roofline of the kernel that takes the most time per step.
     work = kernel_work(step.plan.plan, wl)
     names = {"decode": ("decode_mma_kernel (warp-MMA split-K)" if step.plan.plan.decode_kernel == 2
-                        else "decode_kernel (CUDA-core split-K)"),
+                        else "decode_kernel (FMA split-K)"),
              "prefill_tc": "prefill_tc_kernel (tcgen05 tiles)"}
     timed = {k: prof[k] for k in work if prof[k][1]}
     roof = None

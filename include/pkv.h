@@ -111,17 +111,20 @@ typedef struct pkv_plan_options {
     int32_t split_blocks;      /* >0: decode/support rows are cut into chunks of this many blocks;
                                   0: chosen from the batch size and the SM count */
     int32_t no_split;          /* 1: every row is one chunk (no log-sum-exp merge) */
-    int32_t cuda_core_only;    /* 1: multi-row requests also go to the CUDA-core path (no tcgen05) */
+    int32_t cuda_core_only;    /* 1: no tcgen05 tiles; multi-row requests also go to the split-K
+                                  decode kernel (warp-MMA or FMA) */
     int32_t num_sms;           /* SM count the chunking targets; 0 = query the current device
                                   (pkv_attention_plan) or 148 (pkv_attention_plan_host) */
-    int32_t heads_per_item;    /* query heads of one group served by one CUDA-core work item
-                                  (1..8); 0 = min(Hq/Hkv, 8). Larger groups are split into items
+    int32_t heads_per_item;    /* query heads of one group served by one split-K work item (1..16
+                                  for the warp-MMA kernel, 1..8 for the FMA kernel); 0 = the group,
+                                  capped at that slot count. Larger groups are split into items
                                   that read the same K/V blocks */
-    int32_t rows_per_item;     /* consecutive query rows of one request served by one CUDA-core
-                                  item, capped so rows x heads <= 8; 0 = as many as fit. Such an
-                                  item streams each K/V block once for all its (row, head) pairs */
+    int32_t rows_per_item;     /* consecutive query rows of one request served by one split-K item,
+                                  capped so rows x heads fits the kernel's slots; 0 = as many as
+                                  fit. Such an item streams each K/V block once for all its
+                                  (row, head) pairs */
     int32_t tc_min_rows;       /* requests with at least this many rows (>= 2) go to the tcgen05
-                                  tiles where the shape allows; fewer rows, the CUDA-core kernel.
+                                  tiles where the shape allows; fewer rows, the split-K kernel.
                                   0 = rows x group > 16 with the MMA kernel (a request whose
                                   (row, head) pairs fit one MMA item stays there), else 2 */
     int32_t decode_kernel;     /* kernel for the rows not on tcgen05 tiles: 0 = chosen by the
@@ -145,17 +148,17 @@ typedef struct pkv_plan_options {
 typedef struct pkv_plan {
     uint32_t magic;              /* PKV_PLAN_MAGIC once filled */
     int32_t num_reqs, num_q_tokens, num_q_heads, num_kv_heads, head_dim, dtype;
-    int32_t num_decode_rows;     /* rows served by the CUDA-core split-K kernel */
+    int32_t num_decode_rows;     /* rows served by the split-K decode kernel */
     int32_t num_prefill_rows;    /* rows served by the tcgen05 tile kernel */
-    int32_t num_items;           /* CUDA-core work items (rows, kv head, heads, block chunk) */
+    int32_t num_items;           /* split-K work items (rows, kv head, heads, block chunk) */
     int32_t num_tiles;           /* tcgen05 tiles (request, kv head, 128 packed rows) */
-    int32_t num_merge_rows;      /* chunked CUDA-core items' (rows, heads) sets merged from partials */
+    int32_t num_merge_rows;      /* chunked split-K items' (rows, heads) sets merged from partials */
     int32_t num_partials;        /* chunk partial results in the workspace */
     int32_t split_blocks;        /* chunk length in blocks used for this batch */
     int32_t max_blocks;          /* longest context in blocks */
-    int32_t heads_per_item;      /* query heads per CUDA-core work item */
-    int32_t rows_per_item;       /* most consecutive rows any CUDA-core item serves (0: no items) */
-    int32_t decode_kernel;       /* 1 FMA kernel, 2 warp-MMA kernel, 0 no CUDA-core items */
+    int32_t heads_per_item;      /* query heads per split-K work item */
+    int32_t rows_per_item;       /* most consecutive rows any split-K item serves (0: no items) */
+    int32_t decode_kernel;       /* 1 FMA kernel, 2 warp-MMA kernel, 0 no split-K items */
     int32_t part_stride;         /* (row, head) slots per partial-result entry: the largest item's */
     int64_t off_items, off_tiles, off_merge, off_part_o, off_part_ml; /* byte offsets into workspace */
     int64_t meta_bytes;          /* bytes uploaded by pkv_attention_plan (work lists) */
@@ -164,7 +167,7 @@ typedef struct pkv_plan {
                                     2*D*elem per (kv head, key), counted once per (request, kv head)
                                     for decode rows and once per request for prefill rows */
     int64_t attn_flops;          /* 4*D per (query row, query head, attended key) */
-    int64_t core_kv_bytes;       /* K+V bytes the CUDA-core kernel must read: its requests' contexts,
+    int64_t core_kv_bytes;       /* K+V bytes the split-K kernel must read: its requests' contexts,
                                     with a prefix shared by a run of requests counted once */
     int64_t tile_kv_bytes;       /* part of kv_bytes read by the tcgen05 tiles */
     int64_t tile_flops;          /* part of attn_flops computed by the tcgen05 tiles */
@@ -183,14 +186,21 @@ pkv_status pkv_attention_workspace_size(const int32_t* h_query_start_loc, const 
  * pkv_attention_plan_host -- split the batch into work lists on the host, without any CUDA call.
  * Source for the batch: blog.mckayzhao.com/?p=56, "V1 架构：推倒重来的勇气" (one step = a dict
  * {request_id: num_tokens}; decode rows and chunked-prefill rows share the batch) and "进阶特性"
- * (chunked prefill). Rows with num_tokens == 1 become decode work; requests with more rows go to
- * the tcgen05 tile kernel when dtype is f16/bf16, head_dim is 128 and Hq/Hkv divides 128 (otherwise
- * to the CUDA-core kernel, one row at a time with its causal limit). Long rows are cut into
- * chunks whose partial results a log-sum-exp merge combines.
+ * (chunked prefill). Requests with fewer than tc_min_rows rows (by default: all whose rows x
+ * group fit one 16-slot warp-MMA item, so decode and short speculative-verify rows) become split-K
+ * work: items of up to 16 (row, head) slots (8 for the FMA kernel) of one request and KV head,
+ * consecutive rows packed together, each slot with its own causal limit. The warp-MMA kernel
+ * serves them when dtype is f16/bf16 and head_dim is 128, the FMA kernel otherwise. Requests with
+ * more rows go to the tcgen05 tile kernel when dtype is f16/bf16, head_dim is 128 and Hq/Hkv
+ * divides 128 (otherwise to the split-K kernel). Long contexts are cut into block chunks whose
+ * partial results a log-sum-exp merge combines. With opts->h_block_tables, runs of decode
+ * requests that start with the same physical blocks become one shared-prefix item set plus
+ * per-request suffix items, merged the same way.
  * h_meta (host, meta_capacity bytes) receives the image that pkv_attention_plan uploads to the
  * start of the workspace; pass NULL to only fill *plan.
  * Errors: INVALID_ARG (query_start_loc not starting at 0 or decreasing, context < num_tokens,
- * num_tokens > 0 with context 0, Hq % Hkv != 0), UNSUPPORTED (head_dim not 64/128, Hq/Hkv > 16),
+ * num_tokens > 0 with context 0, Hq % Hkv != 0, decode_kernel outside 0..2), UNSUPPORTED (head_dim
+ * not 64/128, decode_kernel 2 asked for where the warp-MMA kernel does not apply),
  * WORKSPACE_TOO_SMALL (meta_capacity below plan->meta_bytes).
  */
 pkv_status pkv_attention_plan_host(const int32_t* h_query_start_loc, const int32_t* h_context_lens, int num_reqs,
@@ -217,7 +227,8 @@ pkv_status pkv_attention_plan(const int32_t* h_query_start_loc, const int32_t* h
  *   out[row][h][:] = sum_t softmax_t(scale * q[row][h] . K_r[t]) V_r[t],  t = 0 .. ctx_r - n_r + j
  * with K_r[t] = k_pool[block_tables[r][t/16]][h / (Hq/Hkv)][t%16]. Softmax and accumulation in fp32;
  * the output is rounded to the element type. Launches, on `stream`: the tcgen05 prefill tile
- * kernel (if the plan has tiles), the CUDA-core split-K kernel (if it has items) and the
+ * kernel (if the plan has tiles), the split-K decode kernel the plan names (warp-MMA or FMA, if
+ * it has items) and the
  * log-sum-exp merge kernel (if it has merge rows). The plan and workspace must come from
  * pkv_attention_plan with the same batch; q/out shapes must match it.
  * Errors: INVALID_ARG (null pointers, plan magic/shape mismatch), WORKSPACE_TOO_SMALL, CUDA.
