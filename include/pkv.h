@@ -160,6 +160,7 @@ typedef struct pkv_plan {
     int32_t rows_per_item;       /* most consecutive rows any split-K item serves (0: no items) */
     int32_t decode_kernel;       /* 1 FMA kernel, 2 warp-MMA kernel, 0 no split-K items */
     int32_t part_stride;         /* (row, head) slots per partial-result entry: the largest item's */
+    int32_t merge_slots;         /* most (row, head) slots of any merge row (the merge grid's stride) */
     int64_t off_items, off_tiles, off_merge, off_part_o, off_part_ml; /* byte offsets into workspace */
     int64_t meta_bytes;          /* bytes uploaded by pkv_attention_plan (work lists) */
     int64_t ws_bytes;            /* total workspace bytes this plan needs */
@@ -218,6 +219,28 @@ pkv_status pkv_attention_plan(const int32_t* h_query_start_loc, const int32_t* h
                               int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
                               const pkv_plan_options* opts, void* d_workspace, size_t ws_bytes, pkv_plan* plan,
                               pkv_stream_t stream);
+
+/*
+ * pkv_attention_plan_async -- the per-step planning call of a serving loop: plans the batch on the
+ * host straight into caller-owned page-locked memory and enqueues its uploads on `stream`, so the
+ * host never waits for a copy:
+ *   h_meta[0, plan->meta_bytes)  -> d_workspace[0, plan->meta_bytes)   (the work lists)
+ *   h_desc[0, 2R + 1)            -> d_desc[0, 2R + 1)                  (R = num_reqs, int32)
+ * where h_desc receives query_start_loc (R + 1 entries) followed by context_lens (R entries), so
+ * d_desc and d_desc + R + 1 are the device query_start_loc and context_lens of the batch (pass
+ * h_desc = d_desc = NULL to skip that copy). h_meta and h_desc must be page-locked and stay
+ * untouched until the copies have run: record an event on `stream` after the call and wait for
+ * it before reusing them. The batch is the one pkv_attention_plan_host describes (same source).
+ * Errors: as pkv_attention_plan_host; WORKSPACE_TOO_SMALL when meta_capacity < plan->meta_bytes
+ * or ws_bytes < plan->ws_bytes -- nothing is enqueued and *plan holds the sizes needed, with its
+ * magic cleared so that it cannot be launched; INVALID_ARG when only one of h_desc / d_desc is
+ * NULL; CUDA.
+ */
+pkv_status pkv_attention_plan_async(const int32_t* h_query_start_loc, const int32_t* h_context_lens, int num_reqs,
+                                    int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
+                                    const pkv_plan_options* opts, void* h_meta, size_t meta_capacity,
+                                    void* d_workspace, size_t ws_bytes, int32_t* h_desc, int32_t* d_desc,
+                                    pkv_plan* plan, pkv_stream_t stream);
 
 /*
  * pkv_paged_attention -- attention for every row of a planned mixed batch.

@@ -57,6 +57,9 @@ struct PlanLists {
     std::vector<int> req_keys;
     std::vector<int> shared_first;
     int num_partials = 0;
+    size_t num_items = 0, num_merges = 0;
+    // Set when the planner wrote the whole image straight into the caller's buffer.
+    const unsigned char* direct = nullptr;
     void reset() {
         items.clear();
         tiles.clear();
@@ -64,6 +67,8 @@ struct PlanLists {
         start.clear();
         req_keys.clear();
         num_partials = 0;
+        num_items = num_merges = 0;
+        direct = nullptr;
     }
 };
 
@@ -76,8 +81,11 @@ PlanLists& thread_lists() {
 // Query rows per tcgen05 CTA: two 128-row MMA tiles, each (128 / G) consecutive query rows x G heads.
 int tile_tokens(int group) { return 2 * (128 / group); }
 
+// out_meta / out_cap: when given and large enough, the work lists are written straight into that
+// image (the layout write_meta produces), skipping the intermediate lists.
 pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int Hkv, int D, pkv_dtype dt,
-                      const pkv_plan_options* opts, int num_sms, PlanLists* L, pkv_plan* plan) {
+                      const pkv_plan_options* opts, int num_sms, PlanLists* L, pkv_plan* plan,
+                      unsigned char* out_meta = nullptr, size_t out_cap = 0) {
     if (!qsl || (R > 0 && !ctx) || !plan) return fail(PKV_ERR_INVALID_ARG, "null planner argument");
     if (R < 0) return fail(PKV_ERR_INVALID_ARG, "num_reqs < 0");
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Hkv > 32767)
@@ -250,10 +258,26 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
         start[len] = acc;
         acc += cnt;
     }
-    L->items.resize(n_items);
-    L->merges.resize(n_merge);
-    DecodeItem* items = L->items.data();
-    MergeRow* merges = L->merges.data();
+    // Image layout (header, items, tiles, merges; 256-byte aligned), known from the counts.
+    const int64_t off_items = 256;
+    const int64_t off_tiles = align256(off_items + (int64_t)n_items * sizeof(DecodeItem));
+    const int64_t off_merge = align256(off_tiles + (int64_t)L->tiles.size() * sizeof(PrefillTile));
+    const int64_t meta_bytes = align256(off_merge + (int64_t)n_merge * sizeof(MergeRow));
+    const bool direct = out_meta && out_cap >= (size_t)meta_bytes;
+    DecodeItem* items;
+    MergeRow* merges;
+    if (direct) {
+        items = reinterpret_cast<DecodeItem*>(out_meta + off_items);
+        merges = reinterpret_cast<MergeRow*>(out_meta + off_merge);
+    } else {
+        L->items.resize(n_items);
+        L->merges.resize(n_merge);
+        items = L->items.data();
+        merges = L->merges.data();
+    }
+    L->num_items = n_items;
+    L->num_merges = n_merge;
+    if (direct) L->direct = out_meta;
     size_t* pos = start.data();
     size_t mi = 0;
     int partials = 0;
@@ -315,9 +339,9 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->dtype = (int32_t)dt;
     plan->num_decode_rows = decode_rows;
     plan->num_prefill_rows = prefill_rows;
-    plan->num_items = (int32_t)L->items.size();
+    plan->num_items = (int32_t)n_items;
     plan->num_tiles = (int32_t)L->tiles.size();
-    plan->num_merge_rows = (int32_t)L->merges.size();
+    plan->num_merge_rows = (int32_t)n_merge;
     plan->num_partials = L->num_partials;
     plan->split_blocks = chunk;
     plan->max_blocks = max_blocks;
@@ -325,18 +349,18 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     int max_rows = 0;
     for (const CoreRow& c : core_rows) max_rows = std::max(max_rows, c.nrows);
     plan->rows_per_item = max_rows;
-    plan->decode_kernel = L->items.empty() ? 0 : kind;
+    plan->decode_kernel = n_items == 0 ? 0 : kind;
     // Partial entries hold as many (row, head) slots as the largest item has.
     const int part_stride = std::max(1, std::min(slot_cap, hpi * std::max(max_rows, 1)));
     plan->part_stride = part_stride;
-    int64_t off = 256;  // first 256 bytes reserved
-    plan->off_items = off;
-    off = align256(off + (int64_t)L->items.size() * sizeof(DecodeItem));
-    plan->off_tiles = off;
-    off = align256(off + (int64_t)L->tiles.size() * sizeof(PrefillTile));
-    plan->off_merge = off;
-    off = align256(off + (int64_t)L->merges.size() * sizeof(MergeRow));
-    plan->meta_bytes = off;
+    int merge_slots = 0;
+    for (size_t i = 0; i < n_merge; ++i) merge_slots = std::max(merge_slots, merges[i].num_slots);
+    plan->merge_slots = merge_slots;
+    plan->off_items = off_items;  // the first 256 bytes are reserved
+    plan->off_tiles = off_tiles;
+    plan->off_merge = off_merge;
+    plan->meta_bytes = meta_bytes;
+    int64_t off = meta_bytes;
     plan->off_part_o = off;
     off = align256(off + (int64_t)L->num_partials * part_stride * D * 4);
     plan->off_part_ml = off;
@@ -354,16 +378,23 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
 }
 
 // The work-list image: each list at its offset, the header and the alignment gaps zeroed.
+// Fills the image around the items and merges (header, gaps, tiles) -- and the items and merges
+// themselves unless the planner already wrote them in place.
 void write_meta(const PlanLists& L, const pkv_plan& plan, unsigned char* meta) {
-    const size_t end_items = plan.off_items + L.items.size() * sizeof(DecodeItem);
+    if (L.direct && L.direct != meta) {
+        std::memcpy(meta, L.direct, (size_t)plan.meta_bytes);
+        return;
+    }
+    const bool in_place = L.direct == meta;
+    const size_t end_items = plan.off_items + L.num_items * sizeof(DecodeItem);
     const size_t end_tiles = plan.off_tiles + L.tiles.size() * sizeof(PrefillTile);
-    const size_t end_merge = plan.off_merge + L.merges.size() * sizeof(MergeRow);
+    const size_t end_merge = plan.off_merge + L.num_merges * sizeof(MergeRow);
     std::memset(meta, 0, (size_t)plan.off_items);
-    if (!L.items.empty()) std::memcpy(meta + plan.off_items, L.items.data(), L.items.size() * sizeof(DecodeItem));
+    if (!in_place && L.num_items) std::memcpy(meta + plan.off_items, L.items.data(), L.num_items * sizeof(DecodeItem));
     std::memset(meta + end_items, 0, (size_t)plan.off_tiles - end_items);
     if (!L.tiles.empty()) std::memcpy(meta + plan.off_tiles, L.tiles.data(), L.tiles.size() * sizeof(PrefillTile));
     std::memset(meta + end_tiles, 0, (size_t)plan.off_merge - end_tiles);
-    if (!L.merges.empty()) std::memcpy(meta + plan.off_merge, L.merges.data(), L.merges.size() * sizeof(MergeRow));
+    if (!in_place && L.num_merges) std::memcpy(meta + plan.off_merge, L.merges.data(), L.num_merges * sizeof(MergeRow));
     std::memset(meta + end_merge, 0, (size_t)plan.meta_bytes - end_merge);
 }
 
@@ -522,7 +553,7 @@ pkv_status pkv_attention_plan_host(const int32_t* h_query_start_loc, const int32
     PlanLists& L = thread_lists();
     const int sms = (opts && opts->num_sms > 0) ? opts->num_sms : 148;
     pkv_status s = plan_lists(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim,
-                              dtype, opts, sms, &L, plan);
+                              dtype, opts, sms, &L, plan, static_cast<unsigned char*>(h_meta), h_meta ? meta_capacity : 0);
     if (s != PKV_OK) return s;
     if (h_meta) {
         if (meta_capacity < (size_t)plan->meta_bytes)
@@ -552,6 +583,39 @@ pkv_status pkv_attention_plan(const int32_t* h_query_start_loc, const int32_t* h
     write_meta(L, *plan, meta.data());
     // Pageable source: the call returns once the bytes are staged, so `meta` may be reused.
     cudaError_t e = cudaMemcpyAsync(d_workspace, meta.data(), meta.size(), cudaMemcpyHostToDevice, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        plan->magic = 0;
+        return cuda_fail(e, "plan upload");
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_attention_plan_async(const int32_t* h_query_start_loc, const int32_t* h_context_lens, int num_reqs,
+                                    int num_q_heads, int num_kv_heads, int head_dim, pkv_dtype dtype,
+                                    const pkv_plan_options* opts, void* h_meta, size_t meta_capacity,
+                                    void* d_workspace, size_t ws_bytes, int32_t* h_desc, int32_t* d_desc,
+                                    pkv_plan* plan, pkv_stream_t stream) {
+    if ((h_desc == nullptr) != (d_desc == nullptr))
+        return fail(PKV_ERR_INVALID_ARG, "h_desc and d_desc must both be given or both be NULL");
+    PlanLists& L = thread_lists();
+    const int sms = (opts && opts->num_sms > 0) ? opts->num_sms : current_sm_count();
+    pkv_status s = plan_lists(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim,
+                              dtype, opts, sms, &L, plan, static_cast<unsigned char*>(h_meta), h_meta ? meta_capacity : 0);
+    if (s != PKV_OK) return s;
+    if (!h_meta || !d_workspace || meta_capacity < (size_t)plan->meta_bytes || ws_bytes < (size_t)plan->ws_bytes) {
+        plan->magic = 0;
+        return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "work lists need %lld host / %lld device bytes (given %zu / %zu)",
+                    (long long)plan->meta_bytes, (long long)plan->ws_bytes, h_meta ? meta_capacity : 0,
+                    d_workspace ? ws_bytes : 0);
+    }
+    write_meta(L, *plan, static_cast<unsigned char*>(h_meta));
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(d_workspace, h_meta, (size_t)plan->meta_bytes, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess && h_desc && num_reqs >= 0) {
+        std::memcpy(h_desc, h_query_start_loc, sizeof(int32_t) * ((size_t)num_reqs + 1));
+        if (num_reqs > 0) std::memcpy(h_desc + num_reqs + 1, h_context_lens, sizeof(int32_t) * (size_t)num_reqs);
+        e = cudaMemcpyAsync(d_desc, h_desc, sizeof(int32_t) * (2 * (size_t)num_reqs + 1), cudaMemcpyHostToDevice, st);
+    }
     if (e != cudaSuccess) {
         plan->magic = 0;
         return cuda_fail(e, "plan upload");
@@ -619,7 +683,9 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         m.part_ml = reinterpret_cast<const float*>(ws + plan->off_part_ml);
         m.num_rows = plan->num_merge_rows;
         m.num_q_heads = plan->num_q_heads;
-        m.slots_per_entry = plan->heads_per_item * std::max(plan->rows_per_item, 1);
+        // One warp per (merge row, slot): the stride is the largest merge row, not the largest
+        // item (a shared-prefix item packs several requests' rows; each member's merge row is one).
+        m.slots_per_entry = std::max(plan->merge_slots, 1);
         m.part_stride = plan->part_stride;
         ProfileScope prof(PKV_KERNEL_MERGE, s);
         cudaError_t e = launch_merge(plan->dtype, plan->head_dim, m, s);

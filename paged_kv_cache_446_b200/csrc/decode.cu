@@ -387,9 +387,33 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const DecodeA
 // One warp per (merge row, slot): out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i over the row's
 // partials -- its own chunks and, for a request sharing its leading blocks with others, the shared
 // items' chunks. A chunk that saw no key of a slot has m = -inf and weight 0.
+// The kernel is a chain of dependent memory latencies, so it keeps that chain short: once the merge
+// row is read, the (m, l) pairs (one partial per lane) and the output columns of the first kPre
+// partials (each lane its D/32 columns) are loaded together; the weights then reach every lane by
+// shuffles. Further partials, if any, are read kPre at a time.
+template <int PER>
+struct MergeVec;
+template <>
+struct MergeVec<4> {
+    using type = float4;
+    __device__ static void fma(float w, const float4& v, float* o) {
+        o[0] = fmaf(w, v.x, o[0]); o[1] = fmaf(w, v.y, o[1]); o[2] = fmaf(w, v.z, o[2]); o[3] = fmaf(w, v.w, o[3]);
+    }
+};
+template <>
+struct MergeVec<2> {
+    using type = float2;
+    __device__ static void fma(float w, const float2& v, float* o) {
+        o[0] = fmaf(w, v.x, o[0]); o[1] = fmaf(w, v.y, o[1]);
+    }
+};
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
     constexpr int PER = D / 32;
+    constexpr int kPre = 4;
+    using V = MergeVec<PER>;
+    using VT = typename V::type;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     const int entry = gw / a.slots_per_entry;
@@ -403,29 +427,59 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
         return i < mr.count ? (size_t)(mr.first_partial + i) * a.part_stride + g
                             : (size_t)(mr.extra_first + i - mr.count) * a.part_stride + mr.extra_slot + g;
     };
-    float M = -INFINITY;
-    for (int i = 0; i < total; ++i) M = fmaxf(M, a.part_ml[slot_of(i) * 2]);
+    auto o_at = [&](int i) { return *reinterpret_cast<const VT*>(a.part_o + slot_of(i) * D + lane * PER); };
+    const float2* ml = reinterpret_cast<const float2*>(a.part_ml);
+    // Issued together: this lane's (m, l) and the first partials' output columns.
+    const float2 mine = lane < total ? ml[slot_of(lane)] : make_float2(-INFINITY, 0.f);
+    VT pre[kPre];
+#pragma unroll
+    for (int u = 0; u < kPre; ++u)
+        if (u < total) pre[u] = o_at(u);
+    // Row maximum over all partials (lanes hold the first 32; more are folded in by a loop).
+    float M = mine.x;
+    for (int i = lane + 32; i < total; i += 32) M = fmaxf(M, ml[slot_of(i)].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
     float L = 0.f;
-    float o[PER];
+    for (int base = 0; base < total; base += 32) {
+        const int n = min(32, total - base);
+        float w = 0.f;
+        if (lane < n) {
+            const float2 v = base == 0 ? mine : ml[slot_of(base + lane)];
+            w = fast_exp2(v.x - M);
+            L = fmaf(w, v.y, L);
+        }
+        int j = 0;
+        if (base == 0) {
 #pragma unroll
-    for (int e = 0; e < PER; ++e) o[e] = 0.f;
-    for (int i = 0; i < total; ++i) {
-        const size_t p = slot_of(i);
-        const float w = fast_exp2(a.part_ml[p * 2] - M);
-        L = fmaf(w, a.part_ml[p * 2 + 1], L);
-        const float* po = a.part_o + p * D + lane * PER;
+            for (int u = 0; u < kPre; ++u)
+                if (u < n) V::fma(__shfl_sync(FULL_MASK, w, u), pre[u], acc);
+            j = min(n, kPre);
+        }
+        for (; j < n; j += kPre) {
+            VT v[kPre];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) o[e] = fmaf(w, po[e], o[e]);
+            for (int u = 0; u < kPre; ++u)
+                if (j + u < n) v[u] = o_at(base + j + u);
+#pragma unroll
+            for (int u = 0; u < kPre; ++u)
+                if (j + u < n) V::fma(__shfl_sync(FULL_MASK, w, j + u), v[u], acc);
+        }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(FULL_MASK, L, o);
     const float inv = 1.f / L;
     const int jr = g / mr.heads_per_row;
     T* out = static_cast<T*>(a.out) +
              ((size_t)(mr.row + jr) * a.num_q_heads + mr.q_head0 + (g - jr * mr.heads_per_row)) * D + lane * PER;
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
-        if constexpr (sizeof(T) == 4) out[e] = o[e] * inv;
-        else if constexpr (std::is_same<T, __half>::value) out[e] = __float2half_rn(o[e] * inv);
-        else out[e] = __float2bfloat16_rn(o[e] * inv);
+        if constexpr (sizeof(T) == 4) out[e] = acc[e] * inv;
+        else if constexpr (std::is_same<T, __half>::value) out[e] = __float2half_rn(acc[e] * inv);
+        else out[e] = __float2bfloat16_rn(acc[e] * inv);
     }
 }
 

@@ -47,7 +47,7 @@ class Plan(ctypes.Structure):
     _fields_ = [("magic", ctypes.c_uint32)] + [(n, ctypes.c_int32) for n in (
         "num_reqs", "num_q_tokens", "num_q_heads", "num_kv_heads", "head_dim", "dtype", "num_decode_rows",
         "num_prefill_rows", "num_items", "num_tiles", "num_merge_rows", "num_partials", "split_blocks",
-        "max_blocks", "heads_per_item", "rows_per_item", "decode_kernel", "part_stride")] + [(n, ctypes.c_int64) for n in (
+        "max_blocks", "heads_per_item", "rows_per_item", "decode_kernel", "part_stride", "merge_slots")] + [(n, ctypes.c_int64) for n in (
         "off_items", "off_tiles", "off_merge", "off_part_o", "off_part_ml", "meta_bytes", "ws_bytes", "kv_bytes",
         "attn_flops", "core_kv_bytes", "tile_kv_bytes", "tile_flops")]
 
@@ -69,6 +69,8 @@ _copy_blocks = _sig("pkv_copy_blocks", _I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, 
 _ws_size = _sig("pkv_attention_workspace_size", _I, [_P, _P, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_SZ)])
 _plan_host = _sig("pkv_attention_plan_host", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, ctypes.POINTER(Plan)])
 _plan = _sig("pkv_attention_plan", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, ctypes.POINTER(Plan), _P])
+_plan_async = _sig("pkv_attention_plan_async", _I,
+                   [_P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _SZ, _P, _P, ctypes.POINTER(Plan), _P])
 _attention = _sig("pkv_paged_attention", _I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _F, ctypes.POINTER(Plan), _P, _SZ, _P])
 _validate_tables = _sig("pkv_validate_tables", _I, [_P, _P, _I, _I, _I])
 _validate_slots = _sig("pkv_validate_slots", _I, [_P, _I, _I])
@@ -212,6 +214,7 @@ class AttentionPlan:
     def __init__(self, batch: dict, prior_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
                  dtype: torch.dtype, device, workspace: torch.Tensor | None = None, stream=None, **opts):
         self.num_q_heads, self.num_kv_heads, self.head_dim, self.dtype = num_q_heads, num_kv_heads, head_dim, dtype
+        self._code = _dtype_code(torch.empty(0, dtype=dtype))
         self.device = torch.device(device)
         shared = opts.pop("shared_tables", None)
         self._shared = None if shared is None else np.ascontiguousarray(shared, dtype=np.int32)
@@ -223,13 +226,15 @@ class AttentionPlan:
         self._meta = None       # pinned image of the work lists
         self._staged = None     # pinned query_start_loc + context_lens
         self._dev = None        # their device copy
+        self._views = (-1, None, None)  # (R, query_start_loc, context_lens) views of _dev
         self._uploaded = None   # event after the last upload from the pinned buffers
         self.replan(batch, prior_lens, stream=stream)
 
     def replan(self, batch: dict, prior_lens, stream=None, shared_tables=None) -> "AttentionPlan":
-        """Plans the batch on the host (pkv_attention_plan_host) into pinned memory and uploads the
-        work lists and the batch description with asynchronous copies on `stream`. shared_tables:
-        the batch's host block tables, when they changed (for shared-prefix detection)."""
+        """Plans the batch on the host straight into pinned memory and enqueues the uploads of the
+        work lists and of the batch description on `stream` (pkv_attention_plan_async: one library
+        call, no host wait). shared_tables: the batch's host block tables, when they changed (for
+        shared-prefix detection)."""
         if shared_tables is not None:
             self._shared = np.ascontiguousarray(shared_tables, dtype=np.int32)
             self.opts.h_block_tables = self._shared.ctypes.data
@@ -238,44 +243,41 @@ class AttentionPlan:
         self.h_query_start_loc, self.h_context_lens = qsl, ctx
         self.num_q_tokens = int(qsl[-1])
         R = ctx.shape[0]
-        code = _dtype_code(torch.empty(0, dtype=self.dtype))
+        n = 2 * R + 1
         if self._uploaded is not None:
             self._uploaded.synchronize()          # the pinned buffers are free again
-        for _ in range(2):
-            cap = self._meta.numel() if self._meta is not None else 0
-            status = _plan_host(_np_ptr(qsl), _np_ptr(ctx), R, self.num_q_heads, self.num_kv_heads, self.head_dim, code,
-                                ctypes.byref(self.opts), self._meta.data_ptr() if cap else None, cap,
-                                ctypes.byref(self.plan))
-            if status == 4 or (status == PKV_OK and cap == 0):
-                self._meta = torch.empty(max(int(self.plan.meta_bytes) * 5 // 4, 4096), dtype=torch.uint8).pin_memory()
-                continue
-            break
-        _check(status, "pkv_attention_plan_host")
-        if self.workspace is None or self.workspace.numel() < self.plan.ws_bytes:
-            self.workspace = torch.empty(max(int(self.plan.ws_bytes), 256), dtype=torch.uint8, device=self.device)
-        n = 2 * R + 1
         if self._staged is None or self._staged.numel() < n:
             cap = max(n, 64)
             self._staged = torch.empty(cap, dtype=torch.int32).pin_memory()
             self._dev = torch.empty(cap, dtype=torch.int32, device=self.device)
-        host = self._staged.numpy()
-        host[:R + 1] = qsl
-        host[R + 1:n] = ctx
+            self._views = (-1, None, None)
         if isinstance(stream, torch.cuda.Stream):
             s = stream
-        elif stream is None or _stream(stream) == torch.cuda.current_stream(self.device).cuda_stream:
+        elif stream is None:
             s = torch.cuda.current_stream(self.device)
         else:
             s = torch.cuda.ExternalStream(_stream(stream))
-        mb = int(self.plan.meta_bytes)
-        with torch.cuda.stream(s):
-            self.workspace[:mb].copy_(self._meta[:mb], non_blocking=True)
-            self._dev[:n].copy_(self._staged[:n], non_blocking=True)
-            if self._uploaded is None:
-                self._uploaded = torch.cuda.Event()
-            self._uploaded.record(s)
-        self.query_start_loc = self._dev[:R + 1]
-        self.context_lens = self._dev[R + 1:n]
+        qp, cp = qsl.ctypes.data, ctx.ctypes.data
+        for _ in range(3):
+            meta_cap = self._meta.numel() if self._meta is not None else 0
+            ws_cap = self.workspace.numel() if self.workspace is not None else 0
+            status = _plan_async(qp, cp, R, self.num_q_heads, self.num_kv_heads, self.head_dim, self._code,
+                                 ctypes.byref(self.opts), self._meta.data_ptr() if meta_cap else None, meta_cap,
+                                 self.workspace.data_ptr() if ws_cap else None, ws_cap, self._staged.data_ptr(),
+                                 self._dev.data_ptr(), ctypes.byref(self.plan), s.cuda_stream)
+            if status != 4:
+                break
+            if meta_cap < self.plan.meta_bytes:
+                self._meta = torch.empty(max(int(self.plan.meta_bytes) * 5 // 4, 4096), dtype=torch.uint8).pin_memory()
+            if ws_cap < self.plan.ws_bytes:
+                self.workspace = torch.empty(max(int(self.plan.ws_bytes), 256), dtype=torch.uint8, device=self.device)
+        _check(status, "pkv_attention_plan_async")
+        if self._uploaded is None:
+            self._uploaded = torch.cuda.Event()
+        self._uploaded.record(s)
+        if self._views[0] != R:
+            self._views = (R, self._dev[:R + 1], self._dev[R + 1:n])
+        self.query_start_loc, self.context_lens = self._views[1], self._views[2]
         return self
 
 

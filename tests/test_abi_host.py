@@ -176,6 +176,8 @@ def check_plan(pkv, plan, meta, qsl, ctx, Hq, Hkv, opts, dtype, tables=None):
                 assert src not in read
                 read[src] = target
     assert read == written
+    # the merge grid's stride: the largest merge row
+    assert plan.merge_slots == (int(merges[:, 2].max()) if len(merges) else 0)
     if opts.get("no_split") and tables is None:
         assert plan.num_merge_rows == 0
 
@@ -281,3 +283,54 @@ def test_workspace_size_matches_plan(pkv):
         # Algorithmic KV bytes: every (request, KV head, context token) once as K and once as V.
         eb = 4 if wl.dtype == "f32" else 2
         assert plan.kv_bytes == int(ctx.astype(np.int64).sum()) * wl.num_kv_heads * 2 * wl.head_dim * eb
+
+
+def test_plan_async_refuses_before_any_copy(pkv):
+    """pkv_attention_plan_async checks its buffers on the host: without room for the work lists it
+    enqueues nothing, reports the sizes it needs and leaves the plan unlaunchable; a half-given
+    batch-description pair is an argument error."""
+    from paged_kv_cache_446_b200 import workloads as W
+    wl = W.make("c3", small=True, with_tensors=False)
+    qsl, ctx = pkv.flatten_batch(wl.batch, wl.prior_lens)
+    ref, _ = pkv.plan_host(qsl, ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, with_meta=False,
+                           num_sms=148)
+    o = pkv._opts(num_sms=148)
+    plan = pkv.Plan()
+    args = (qsl.ctypes.data, ctx.ctypes.data, ctx.shape[0], wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+            pkv.DTYPE_NAME[wl.dtype], ctypes.byref(o))
+    meta = np.zeros(ref.meta_bytes, np.uint8)
+    # no device workspace: refused with the sizes filled in
+    assert pkv._plan_async(*args, meta.ctypes.data, meta.nbytes, None, 0, None, None, ctypes.byref(plan), None) == 4
+    assert plan.magic == 0 and plan.meta_bytes == ref.meta_bytes and plan.ws_bytes == ref.ws_bytes
+    # host image one byte short: refused (the device pointer is never touched)
+    assert pkv._plan_async(*args, meta.ctypes.data, meta.nbytes - 1, 1 << 20, ref.ws_bytes, None, None,
+                           ctypes.byref(plan), None) == 4
+    assert plan.magic == 0
+    # only one of the batch-description buffers
+    desc = np.zeros(2 * ctx.shape[0] + 1, np.int32)
+    assert pkv._plan_async(*args, meta.ctypes.data, meta.nbytes, 1 << 20, ref.ws_bytes, desc.ctypes.data, None,
+                           ctypes.byref(plan), None) == 1
+    assert "h_desc" in pkv._lib.pkv_last_error().decode()
+
+
+@pytest.mark.parametrize("config", ["c3", "c4", "c5"])
+def test_plan_image_independent_of_buffer_contents(pkv, config):
+    """The planner writes the work lists in place into the caller's image and zeroes every gap:
+    planning into a buffer full of stale bytes gives the same image as planning into zeros."""
+    from paged_kv_cache_446_b200 import workloads as W
+    wl = W.make(config, small=True, with_tensors=False)
+    qsl, ctx = pkv.flatten_batch(wl.batch, wl.prior_lens)
+    o = pkv._opts(num_sms=148, shared_tables=np.ascontiguousarray(wl.block_tables, dtype=np.int32))
+    plan = pkv.Plan()
+    assert pkv._plan_host(qsl.ctypes.data, ctx.ctypes.data, ctx.shape[0], wl.num_q_heads, wl.num_kv_heads,
+                          wl.head_dim, pkv.DTYPE_NAME[wl.dtype], ctypes.byref(o), None, 0, ctypes.byref(plan)) == 0
+    images = []
+    for fill in (0x00, 0xAB):
+        meta = np.full(plan.meta_bytes + 512, fill, np.uint8)
+        assert pkv._plan_host(qsl.ctypes.data, ctx.ctypes.data, ctx.shape[0], wl.num_q_heads, wl.num_kv_heads,
+                              wl.head_dim, pkv.DTYPE_NAME[wl.dtype], ctypes.byref(o), meta.ctypes.data, meta.nbytes,
+                              ctypes.byref(plan)) == 0
+        assert (meta[plan.meta_bytes:] == fill).all()          # nothing written past the image
+        images.append(meta[:plan.meta_bytes].copy())
+    assert np.array_equal(images[0], images[1])
+    assert plan.num_items > 0
