@@ -90,7 +90,24 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const LayerPtrs ptrs, 
     uint4* base = blockIdx.z == 0 ? ptrs.k[blockIdx.y] : ptrs.v[blockIdx.y];
     const uint4* s = base + (long long)src * chunks_per_block;
     uint4* d = base + (long long)dst * chunks_per_block;
-    for (long long i = threadIdx.x; i < chunks_per_block; i += blockDim.x) d[i] = s[i];
+    // Eight 16-byte loads in flight per thread before their stores (a copy that stored each chunk
+    // before loading the next paid one memory latency per chunk). Source and destination are
+    // distinct blocks, so they never overlap.
+    constexpr int U = 8;
+    const long long n = chunks_per_block;
+    for (long long i0 = threadIdx.x; i0 < n; i0 += (long long)blockDim.x * U) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long i = i0 + (long long)u * blockDim.x;
+            if (i < n) v[u] = s[i];
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long i = i0 + (long long)u * blockDim.x;
+            if (i < n) d[i] = v[u];
+        }
+    }
 }
 
 }  // namespace
