@@ -242,9 +242,12 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     }
     auto pieces_of = [&](const CoreRow& c) { return (int)ceil_div(c.be - c.bs, chunk); };
     auto with_partials = [&](const CoreRow& c, int pieces) { return c.kind != 0 || pieces > 1; };
-    // Items are placed directly at their position in a stable order by length, longest first:
-    // this balances the static round-robin over the persistent warps. Pass 1 counts the items of
-    // each length from the row lengths alone; pass 2 writes every item to its slot.
+    // Items are placed directly at their position in a stable order by length, longest first,
+    // dealt to the persistent warps (warp w runs positions w, w + W, w + 2W, ...) in a snake: the
+    // k-th longest item of an odd round goes to the warp that got the k-th shortest of the round
+    // before, so the warps' totals even out. Pass 1 counts the items of each length from the row
+    // lengths alone; pass 2 writes every item to its slot. W is the resident warp count of the
+    // decode kernels (8 per SM); a launch with another count still runs every item.
     size_t n_items = 0, n_merge = 0;
     int max_len = 0;
     for (const CoreRow& c : core_rows) {
@@ -253,6 +256,14 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
         if (c.kind == 2 || (c.kind == 0 && pieces > 1)) n_merge += (size_t)Hkv * groups;
         max_len = std::max(max_len, std::min(c.be - c.bs, chunk));
     }
+    const uint32_t deal = (uint32_t)std::max(num_sms, 1) * 8;
+    const uint32_t n_items32 = (uint32_t)n_items;  // the plan counts items in int32
+    auto snake = [&](size_t k) -> size_t {
+        const uint32_t k32 = (uint32_t)k, r = k32 / deal, w = k32 - r * deal;
+        if (!(r & 1)) return k;
+        const uint32_t in_round = std::min(deal, n_items32 - r * deal);
+        return (size_t)r * deal + (in_round - 1 - w);
+    };
     std::vector<size_t>& start = L->start;
     start.assign((size_t)max_len + 2, 0);
     for (const CoreRow& c : core_rows) {
@@ -321,7 +332,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
                 }
                 for (int p = 0; p < pieces; ++p) {
                     const int b0 = c.bs + p * chunk, b1 = std::min(c.be, b0 + chunk);
-                    items[pos[b1 - b0]++] = DecodeItem{c.row, c.req, (int16_t)h, (int16_t)c.nrows, g0, b0, b1, c.limit,
+                    items[snake(pos[b1 - b0]++)] = DecodeItem{c.row, c.req, (int16_t)h, (int16_t)c.nrows, g0, b0, b1, c.limit,
                                                        first >= 0 ? first + p : -1};
                 }
             }
