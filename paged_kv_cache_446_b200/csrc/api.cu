@@ -243,11 +243,12 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     auto pieces_of = [&](const CoreRow& c) { return (int)ceil_div(c.be - c.bs, chunk); };
     auto with_partials = [&](const CoreRow& c, int pieces) { return c.kind != 0 || pieces > 1; };
     // Items are placed directly at their position in a stable order by length, longest first,
-    // dealt to the persistent warps (warp w runs positions w, w + W, w + 2W, ...) in a snake: the
-    // k-th longest item of an odd round goes to the warp that got the k-th shortest of the round
-    // before, so the warps' totals even out. Pass 1 counts the items of each length from the row
-    // lengths alone; pass 2 writes every item to its slot. W is the resident warp count of the
-    // decode kernels (8 per SM); a launch with another count still runs every item.
+    // dealt to the persistent warps (warp w runs positions w, w + W, w + 2W, ...) in a snake: each
+    // odd round of W items is dealt in reverse, so the warps that took the longest items of one
+    // round take the shortest of the next and the warps' totals even out. Pass 1 counts the items
+    // of each length from the row lengths alone; pass 2 writes every item to its slot. W is the
+    // resident warp count of the decode kernels (8 per SM); a launch with another count still runs
+    // every item.
     size_t n_items = 0, n_merge = 0;
     int max_len = 0;
     for (const CoreRow& c : core_rows) {

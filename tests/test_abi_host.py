@@ -334,3 +334,28 @@ def test_plan_image_independent_of_buffer_contents(pkv, config):
         images.append(meta[:plan.meta_bytes].copy())
     assert np.array_equal(images[0], images[1])
     assert plan.num_items > 0
+
+
+@pytest.mark.parametrize("config", ["c2", "c3", "c4", "c6"])
+def test_items_dealt_longest_first_in_a_snake(pkv, config):
+    """The persistent decode warps run positions w, w + W, w + 2W, ... (W = 8 per SM): the planner
+    sorts the items longest first and deals every second round of W in reverse, so reading the
+    positions back in dealing order gives block counts that never increase, and the warps' totals
+    come out within a few percent of each other."""
+    from paged_kv_cache_446_b200 import workloads as W
+    wl = W.make(config, with_tensors=False)
+    qsl, ctx = pkv.flatten_batch(wl.batch, wl.prior_lens)
+    plan, meta = pkv.plan_host(qsl, ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, num_sms=148,
+                               shared_tables=wl.block_tables)
+    items, _, _ = parse_meta(plan, meta)
+    lens = items[:, 5] - items[:, 4]
+    n, deal = len(lens), 148 * 8
+    dealt = []
+    for k in range(n):
+        r, w = divmod(k, deal)
+        in_round = min(deal, n - r * deal)
+        dealt.append(lens[k] if r % 2 == 0 else lens[r * deal + in_round - 1 - w])
+    assert all(a >= b for a, b in zip(dealt, dealt[1:]))
+    per_warp = np.zeros(deal)
+    np.add.at(per_warp, np.arange(n) % deal, lens + 1)
+    assert per_warp.max() <= 1.1 * per_warp.mean() or n <= 3 * deal
