@@ -219,12 +219,13 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
         core_rows.insert(core_rows.begin(), shared.begin(), shared.end());
     }
 
-    // Chunk length: enough items per resident warp that the longest-first round-robin ends evenly,
-    // but never below 16 blocks. A split item of s (row, head) slots writes s partials that s merge
-    // warps read back, so items of few slots are cut finer: 8 per warp for s <= 2, 6 for s <= 4,
-    // 4 otherwise (measured on the decode batches against fixed lengths 8-96; c2-shaped rows of one
-    // slot: 36 -> 18 blocks, 2 % faster; 4-slot GQA rows: 39 -> 26, 1.5 %; parallel sampling:
-    // 8 -> 16, 4 %; 5- and 8-slot rows keep their length).
+    // Chunk length: enough items per resident warp that the snake-dealt longest-first order (below)
+    // ends evenly, but never below 16 blocks. A split item of s (row, head) slots writes s partials
+    // that s merge warps read back, so items of one or two slots are cut finer: 6 items per warp
+    // for s <= 2, 4 otherwise. Measured on the decode batches with the snake dealing against
+    // fixed lengths: one-slot rows (13B-shaped decode) best at 24 blocks (18: +0.9 %, 36: +0.8 %),
+    // 4-slot GQA rows at 39 (26: +1.7 %), 5-slot verify rows at 39 (24: +1.7 %, 52: +6 %);
+    // parallel sampling gains 4 % from the 16-block floor (8 before).
     const int groups = (int)ceil_div(G, hpi);
     int64_t total_blocks = 0;
     int max_slots = 1;
@@ -237,7 +238,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     else if (o.split_blocks > 0) chunk = o.split_blocks;
     else {
         const int64_t workers = (int64_t)std::max(num_sms, 1) * 8;
-        const int per_worker = max_slots <= 2 ? 8 : (max_slots <= 4 ? 6 : 4);
+        const int per_worker = max_slots <= 2 ? 6 : 4;
         chunk = (int)std::min<int64_t>(std::max<int64_t>(ceil_div(total_blocks, workers * per_worker), 16), 1 << 20);
     }
     auto pieces_of = [&](const CoreRow& c) { return (int)ceil_div(c.be - c.bs, chunk); };
