@@ -13,7 +13,6 @@ Two independent implementations live here:
 Arrays are NumPy; 16-bit storage types are passed as uint16 bit patterns.
 """
 import ctypes
-import os
 
 import numpy as np
 

@@ -30,7 +30,6 @@ namespace {
 
 constexpr int log2i(int x) { return x <= 1 ? 0 : 1 + log2i(x / 2); }
 constexpr int round16(int x) { return (x + 15) / 16 * 16; }
-constexpr int clampi(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
 
 template <typename T, int D, int GP, int NSTAGE>
 struct Dec {
