@@ -336,8 +336,9 @@ def test_plan_image_independent_of_buffer_contents(pkv, config):
     assert plan.num_items > 0
 
 
-@pytest.mark.parametrize("config", ["c2", "c3", "c4", "c6"])
-def test_items_dealt_longest_first_in_a_snake(pkv, config):
+@pytest.mark.parametrize("config,num_sms", [("c2", 148), ("c3", 148), ("c4", 148), ("c6", 148), ("c3", 2),
+                                            ("c5", 3), ("c6", 1)])
+def test_items_dealt_longest_first_in_a_snake(pkv, config, num_sms):
     """The persistent decode warps run positions w, w + W, w + 2W, ... (W = 8 per SM): the planner
     sorts the items longest first and deals every second round of W in reverse, so reading the
     positions back in dealing order gives block counts that never increase, and the warps' totals
@@ -345,11 +346,11 @@ def test_items_dealt_longest_first_in_a_snake(pkv, config):
     from paged_kv_cache_446_b200 import workloads as W
     wl = W.make(config, with_tensors=False)
     qsl, ctx = pkv.flatten_batch(wl.batch, wl.prior_lens)
-    plan, meta = pkv.plan_host(qsl, ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, num_sms=148,
+    plan, meta = pkv.plan_host(qsl, ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, num_sms=num_sms,
                                shared_tables=wl.block_tables)
     items, _, _ = parse_meta(plan, meta)
     lens = items[:, 5] - items[:, 4]
-    n, deal = len(lens), 148 * 8
+    n, deal = len(lens), num_sms * 8
     dealt = []
     for k in range(n):
         r, w = divmod(k, deal)
