@@ -56,6 +56,8 @@ struct PlanLists {
     std::vector<size_t> start;
     std::vector<int> req_keys;
     std::vector<int> shared_first;
+    struct Cursor { uint32_t round, index; };
+    std::vector<Cursor> cursor;
     int num_partials = 0;
     size_t num_items = 0, num_merges = 0;
     // Set when the planner wrote the whole image straight into the caller's buffer.
@@ -258,14 +260,6 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
         if (c.kind == 2 || (c.kind == 0 && pieces > 1)) n_merge += (size_t)Hkv * groups;
         max_len = std::max(max_len, std::min(c.be - c.bs, chunk));
     }
-    const uint32_t deal = (uint32_t)std::max(num_sms, 1) * 8;
-    const uint32_t n_items32 = (uint32_t)n_items;  // the plan counts items in int32
-    auto snake = [&](size_t k) -> size_t {
-        const uint32_t k32 = (uint32_t)k, r = k32 / deal, w = k32 - r * deal;
-        if (!(r & 1)) return k;
-        const uint32_t in_round = std::min(deal, n_items32 - r * deal);
-        return (size_t)r * deal + (in_round - 1 - w);
-    };
     std::vector<size_t>& start = L->start;
     start.assign((size_t)max_len + 2, 0);
     for (const CoreRow& c : core_rows) {
@@ -281,6 +275,25 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
         start[len] = acc;
         acc += cnt;
     }
+    // Dealing cursors: the items of length `len` take the sorted positions start[len], +1, ...;
+    // each cursor keeps its position as (round, index in the round) so the snake needs no
+    // division per item.
+    const uint32_t deal = (uint32_t)std::max(num_sms, 1) * 8;
+    const uint32_t n_items32 = (uint32_t)n_items;  // the plan counts items in int32
+    std::vector<PlanLists::Cursor>& cursor = L->cursor;
+    cursor.resize((size_t)max_len + 2);
+    for (int len = 1; len <= max_len; ++len)
+        cursor[len] = PlanLists::Cursor{(uint32_t)(start[len] / deal), (uint32_t)(start[len] % deal)};
+    auto place = [&](int len) -> size_t {
+        PlanLists::Cursor& q = cursor[len];
+        const size_t at = (size_t)q.round * deal +
+                          ((q.round & 1) ? std::min(deal, n_items32 - q.round * deal) - 1 - q.index : q.index);
+        if (++q.index == deal) {
+            q.index = 0;
+            ++q.round;
+        }
+        return at;
+    };
     // Image layout (header, items, tiles, merges; 256-byte aligned), known from the counts.
     const int64_t off_items = 256;
     const int64_t off_tiles = align256(off_items + (int64_t)n_items * sizeof(DecodeItem));
@@ -301,7 +314,6 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     L->num_items = n_items;
     L->num_merges = n_merge;
     if (direct) L->direct = out_meta;
-    size_t* pos = start.data();
     size_t mi = 0;
     int partials = 0;
     // First partial entry of each (shared row, KV head, head group): members' merges point there.
@@ -334,7 +346,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
                 }
                 for (int p = 0; p < pieces; ++p) {
                     const int b0 = c.bs + p * chunk, b1 = std::min(c.be, b0 + chunk);
-                    items[snake(pos[b1 - b0]++)] = DecodeItem{c.row, c.req, (int16_t)h, (int16_t)c.nrows, g0, b0, b1, c.limit,
+                    items[place(b1 - b0)] = DecodeItem{c.row, c.req, (int16_t)h, (int16_t)c.nrows, g0, b0, b1, c.limit,
                                                        first >= 0 ? first + p : -1};
                 }
             }
