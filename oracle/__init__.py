@@ -170,20 +170,29 @@ def max_threads() -> int:
 
 __all__ = ["paged_attention", "slot_mapping", "kv_cache_write", "copy_blocks", "blocks_for_tokens",
            "wasted_slots", "half_to_double", "bf16_to_double", "max_threads", "load", "F32", "F16", "BF16",
-           "OracleError"]
+           "OracleError", "flatten_batch"]
 
 
-def flatten_batch(batch: dict, prior_lens) -> tuple[np.ndarray, np.ndarray]:
+def flatten_batch(batch: dict, prior_lens, mutant=None) -> tuple[np.ndarray, np.ndarray]:
     """{request_id: num_tokens} (insertion order) -> (query_start_loc [R+1], context_lens [R]).
 
     blog.mckayzhao.com/?p=56, "V1 架构：推倒重来的勇气": one step is a dict giving each request's token
     count; rows of request r are consecutive, in dict order; its context after the step is its prior
-    context plus its tokens.
+    context plus its tokens. prior_lens[r] belongs to the r-th entry of the dict.
+
+    mutant (tests only) plants one mistake: "FLAT_CTX_PRIOR" leaves the step's tokens out of the
+    context, "FLAT_SORTED_IDS" lays rows out in request-id order instead of dict order,
+    "FLAT_QSL_SHIFT" drops the leading zero of the prefix sum.
     """
-    counts = [int(v) for v in batch.values()]
+    items = list(batch.items())
+    if mutant == "FLAT_SORTED_IDS":
+        items.sort(key=lambda kv: kv[0])
+    counts = [int(v) for _, v in items]
     qsl = [0]
     for c in counts:
         qsl.append(qsl[-1] + c)
+    if mutant == "FLAT_QSL_SHIFT":
+        qsl = qsl[1:] + [qsl[-1]]
     prior = [int(p) for p in prior_lens]
-    ctx = [p + c for p, c in zip(prior, counts)]
+    ctx = [p if mutant == "FLAT_CTX_PRIOR" else p + c for p, c in zip(prior, counts)]
     return np.asarray(qsl, dtype=np.int32), np.asarray(ctx, dtype=np.int32)

@@ -296,6 +296,32 @@ def pin_storage_decoders(mutant=None):
             assert lib.oracle_bf16_to_double(int(bits[i])) == b[i], f"bf16 {i:#06x}"
 
 
+def pin_flatten_batch(mutant=None):
+    """blog.mckayzhao.com/?p=56, "V1 架构：推倒重来的勇气": a step is {request_id: num_tokens}. Hand-derived
+    flattenings (tests/golden/flatten_batch.json) -- mixed prefill/decode rows, requests with 0 tokens,
+    ids out of order, an empty step -- and, on seeded random dicts, the defining properties: request
+    r's rows are the range [query_start_loc[r], query_start_loc[r+1]) of length num_tokens, laid out
+    in the dict's order, and context_lens[r] = prior + num_tokens."""
+    for case in golden("flatten_batch.json")["cases"]:
+        batch = {int(r): int(n) for r, n in case["batch"]}
+        qsl, ctx = oracle.flatten_batch(batch, case["prior_lens"], mutant=mutant)
+        assert qsl.dtype == np.int32 and ctx.dtype == np.int32
+        assert qsl.tolist() == case["query_start_loc"], (case["name"], qsl.tolist())
+        assert ctx.tolist() == case["context_lens"], (case["name"], ctx.tolist())
+    rng = np.random.default_rng(7)
+    for _ in range(50):
+        R = int(rng.integers(0, 40))
+        ids = rng.permutation(1000)[:R]
+        counts = rng.integers(0, 600, R) * (rng.random(R) < 0.8)
+        prior = rng.integers(0, 40000, R)
+        batch = {int(i): int(c) for i, c in zip(ids, counts)}
+        qsl, ctx = oracle.flatten_batch(batch, prior, mutant=mutant)
+        assert qsl.shape == (R + 1,) and ctx.shape == (R,) and qsl[0] == 0
+        for r, (rid, n) in enumerate(batch.items()):
+            assert qsl[r + 1] - qsl[r] == n, (rid, n)
+            assert ctx[r] == prior[r] + n
+
+
 ALL_PINS = [pin_brute_force, pin_permutation, pin_closed_forms, pin_chunked_equals_incremental,
             pin_batch_independence, pin_sharing, pin_slot_mapping_figure, pin_append_then_attend,
-            pin_copy_on_write, pin_block_accounting, pin_storage_decoders]
+            pin_copy_on_write, pin_block_accounting, pin_storage_decoders, pin_flatten_batch]
