@@ -4,9 +4,13 @@
 One step = one pass of the whole path over one batch of synthetic input: copy-on-write block
 copies (when the workload has shared blocks), slot mapping, KV append, then paged attention over
 the mixed batch (split-K decode kernel, tcgen05 prefill tiles when present, log-sum-exp merge).
-The default workload is the LLaMA-13B-shaped fp16 decode batch (64 rows, 40/40 heads, head_dim
-128, context U[128,2048], one appended token per row). Its KV pool is ~1.4 GB, larger than the
-126 MB L2, so no explicit L2 flush is used between steps.
+The default workload is the largest single-GPU one: the 70B-shaped bf16 mixed batch (64/8 heads,
+head_dim 128; 4 chunked-prefill requests of 512 rows at prior contexts 0/4k/16k/32k and 128 decode
+rows with contexts U[256, 16384], one {request_id: num_tokens} step). --config c2 selects the
+LLaMA-13B-shaped fp16 decode batch, and so on. Every workload's KV pool (>= 0.6 GB, 4.8 GB for the
+default) is larger than the 126 MB L2; a second timed pass (--l2-flush, on by default) also
+writes a 2 x L2-sized buffer between steps, outside the timed events, and reports that figure
+beside the unflushed one.
 
 Metric: KV bytes the step must read (every (request, KV head, context token) once as K and once as
 V) divided by the step time, in GB/s; also decode sequence-tokens per second (sum of decode rows'
@@ -43,9 +47,11 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5", "c6"])
+    ap.add_argument("--config", default="c5", choices=["c1", "c2", "c3", "c4", "c5", "c6"])
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-l2-flush", action="store_true",
+                    help="skip the second timed pass that flushes L2 between steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--split-blocks", type=int, default=0)
@@ -406,6 +412,34 @@ def main():
     code, detail = pkv.device_error()
     assert code == 0, f"device error {code} at {detail}"
 
+    # ---- the same steps with L2 flushed between them ----
+    # A write of twice the L2 size runs before every step, outside that step's event pair, so no
+    # step finds its predecessor's K/V (or its own inputs) in L2. Step time = sum of the per-step
+    # event intervals.
+    flushed_ms, prof_flushed = None, None
+    if not args.no_l2_flush:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size or (126 << 20)
+        flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        for a, b in pairs:
+            flush_buf.fill_(1)
+            a.record()
+            run_step()
+            b.record()
+        torch.cuda.synchronize()
+        flushed_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in pairs), dist, dev) / args.steps
+        # once more with every library launch timed, for the kernels' flushed rooflines
+        pkv.profile_start(capacity=16 * args.steps + 16)
+        for _ in range(args.steps):
+            flush_buf.fill_(1)
+            run_step()
+        torch.cuda.synchronize()
+        prof_flushed = pkv.profile_stop()
+        del flush_buf
+
     # ---- end to end through the public API: pinned host inputs in, output back to the host ----
     e2e = None
     if not args.no_e2e:
@@ -506,32 +540,43 @@ def main():
         return
     peak, peak_kind = peaks()
     value = whole_job_gbs(kv_bytes(wl), world, ms_per_step)
-    # Roofline of the kernel that takes the most time per step.
+    # Rooflines of both attention kernels (each launch timed with CUDA events on its stream in the
+    # profiling pass): the tcgen05 prefill tiles against the dense 16-bit tensor peak, the split-K
+    # kernel against the HBM copy peak; `roofline` is the one that takes the most time per step.
     work = kernel_work(step.plan.plan, wl)
-    names = {"decode": ("decode_mma_kernel (warp-MMA split-K)" if step.plan.plan.decode_kernel == 2
-                        else "decode_kernel (FMA split-K)"),
-             "prefill_tc": "prefill_tc_kernel (tcgen05 tiles)"}
-    timed = {k: prof[k] for k in work if prof[k][1]}
-    roof = None
-    if timed:
-        k = max(timed, key=lambda x: timed[x][0])
-        avg_ms = timed[k][0] / timed[k][1]
+    tc_peak, tc_kind = tensor_peak()
+    rooflines = {}
+    for k, w in work.items():
+        if not prof[k][1]:
+            continue
+        avg_ms = prof[k][0] / prof[k][1]
         kname = "decode_mma_kernel" if (k == "decode" and step.plan.plan.decode_kernel == 2) else k + "_kernel"
-        w = work[k]
-        tc_peak, tc_kind = tensor_peak()
-        t_hbm = w["bytes"] / (peak * 1e9)
-        t_tc = w.get("flops", 0) / (tc_peak * 1e12)
-        if t_tc > t_hbm:
+        if k == "prefill_tc":
             achieved = w["flops"] / (avg_ms * 1e-3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                    "frac": achieved / tc_peak, "traffic": recorded_traffic(kname, wl.name),
-                    "algorithmic_flops": w["flops"], "peak_source": f"{tc_kind} bf16_tflops (burst cuBLAS)"}
+            r = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                 "frac": achieved / tc_peak, "traffic": recorded_traffic(kname, wl.name),
+                 "algorithmic_flops": w["flops"], "algorithmic_bytes": w["bytes"],
+                 "peak_source": f"{tc_kind} bf16_tflops (burst cuBLAS)"}
         else:
             achieved = w["bytes"] / (avg_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": recorded_traffic(kname, wl.name), "algorithmic_bytes": w["bytes"],
-                    "peak_source": f"{peak_kind} hbm_gbs (burst copy)"}
-        roof.update(kernel=names[k], kernel_ms=avg_ms)
+            r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                 "traffic": recorded_traffic(kname, wl.name), "algorithmic_bytes": w["bytes"],
+                 "peak_source": f"{peak_kind} hbm_gbs (burst copy)"}
+        r.update(kernel=kname, kernel_ms=avg_ms, launches_per_step=prof[k][1] / max(1, args.steps))
+        if prof_flushed and prof_flushed[k][1]:
+            fms = prof_flushed[k][0] / prof_flushed[k][1]
+            r["l2_flushed"] = {"kernel_ms": fms, "frac": r["frac"] * avg_ms / fms}
+        rooflines[k] = r
+    roof = None
+    if rooflines:
+        dom = max(rooflines, key=lambda k: prof[k][0])
+        roof = dict(rooflines[dom])
+    # The step's own bound: every K/V byte once at the HBM peak, or every prefill flop at the tensor
+    # peak, whichever is longer (the two can overlap in one step).
+    t_bytes = kv_bytes(wl) / (peak * 1e9) * 1e3
+    t_flops = work["prefill_tc"]["flops"] / (tc_peak * 1e12) * 1e3
+    step_bound = {"ms": max(t_bytes, t_flops), "hbm_ms": t_bytes, "tensor_ms": t_flops,
+                  "frac": max(t_bytes, t_flops) / ms_per_step}
     launches = sum(v[1] for k, v in prof.items() if k != "dropped")
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -541,7 +586,8 @@ def main():
         "config": {"workload": wl.name, "requests": len(wl.batch), "num_q_heads": wl.num_q_heads,
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
                    "num_blocks": wl.num_blocks, "kv_bytes_per_step_per_gpu": kv_bytes(wl),
-                   "l2": "inputs larger than L2 (KV pool read per step >> 126 MB); no flush",
+                   "l2": "inputs larger than L2 (KV pool read per step >> 126 MB); value taken without a "
+                         "flush, l2_flushed taken with a 2 x L2 write between steps",
                    "parallelism": f"replicas x{world} (independent requests per GPU)",
                    "plan_options": opts},
         "frac_of_hbm_peak": value / world / peak,
@@ -551,6 +597,11 @@ def main():
         "decode_steps_per_s": 1e3 / ms_per_step,
         "kernel_ms_per_step": {k: v[0] / max(1, args.steps) for k, v in prof.items() if k != "dropped"},
         "roofline": roof,
+        "rooflines": rooflines,
+        "step_bound": step_bound,
+        "l2_flushed": None if flushed_ms is None else {
+            "ms_per_step": flushed_ms, "value": whole_job_gbs(kv_bytes(wl), world, flushed_ms), "unit": "GB/s",
+            "frac_of_hbm_peak": kv_bytes(wl) / (flushed_ms * 1e-3) / 1e9 / peak},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
         "gpu_launches": launches,

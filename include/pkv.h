@@ -7,8 +7,10 @@
  * 一文搞懂vLLM：为啥它能让一张GPU扛住几十倍用户？, "PagedAttention：核心思路").
  *
  * Conventions for every call:
- *   - Device pointers are caller-owned (typically torch tensors); the library allocates no device
- *     memory. Host pointers are read during the call only.
+ *   - Device pointers are caller-owned (typically torch tensors). The library makes no device
+ *     allocation; the only device memory it owns is module-scope: a 16-byte error word per device
+ *     (pkv_device_error) and the fixed scratch array of pkv_paged_attention_static_ws, the one
+ *     call that does not take a caller workspace. Host pointers are read during the call only.
  *   - Kernels run asynchronously on the caller's stream `stream` (0 = legacy default stream).
  *   - Argument errors are detected on the host before any launch and returned as a pkv_status;
  *     no call traps on the device. Kernels that find an out-of-range block id or slot at run time
@@ -290,8 +292,9 @@ pkv_status pkv_device_error(int* code, int64_t* detail, pkv_stream_t stream);
  * of PKV_STATIC_WS_BYTES, held by every GPU that loads the library until the process exits.
  * Arguments: the host batch description and options of pkv_attention_plan, then the device
  * tensors and scale of pkv_paged_attention (same layouts and meaning); out receives the result.
- * The array's device address is looked up on the first call made on each device, so make that
- * first call before any stream capture begins. Every call reuses the same array, which keeps the
+ * The array's device address is looked up on the first call made on each device (and again when
+ * that device's current CUDA context is a different one, e.g. after cudaDeviceReset), so make that
+ * first call before any stream capture begins. The batch is planned once per call, on the host. Every call reuses the same array, which keeps the
  * last call's contents; calls that may overlap on the GPU (other streams or host threads) race on
  * it and must be serialised by the caller. No part of it has to start zeroed: each call writes
  * what its kernels read.

@@ -242,8 +242,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = kt & 1;
             if (ids_base < 0 || kt * 8 >= ids_base + 32) {
                 ids_base = kt * 8;
+                // Entries past the context are never read (-2: zero fill). The context comes from the
+                // device lengths, so an entry past the table's width (device lengths larger than the
+                // planned ones) is not read either: -3 is recorded as a range error below.
                 const int b = ids_base + lane;
-                ids = b < nblk_ctx ? __ldg(a.block_tables + (size_t)req * a.max_blocks_per_seq + b) : -2;
+                ids = b >= nblk_ctx ? -2
+                      : b < a.max_blocks_per_seq ? __ldg(a.block_tables + (size_t)req * a.max_blocks_per_seq + b) : -3;
             }
             int y[8];
 #pragma unroll

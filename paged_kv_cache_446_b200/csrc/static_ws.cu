@@ -9,12 +9,16 @@
 // work lists and the split-K partials move into the library's own array.
 //
 // The array (PKV_STATIC_WS_BYTES) is part of this file's device module: every GPU that loads it
-// holds the memory until the process exits. Its device address is looked up once per device, on
-// the first call made with that device current, so make that first call before any stream
-// capture begins. All calls share the one array and it keeps the contents of the last call:
-// calls that can overlap on the GPU (different streams, or different host threads) race on it and
-// must be serialised by the caller. Nothing in it has to start at zero -- each call writes every
-// byte its kernels read (the uploaded work lists, then the partials) before reading it.
+// holds the memory until the process exits. Its device address is looked up with
+// cudaGetSymbolAddress on the first call made with a device current, so make that first call before
+// any stream capture begins; the address is kept per CUDA context and looked up again when the
+// device's current context is a different one (for example after cudaDeviceReset). All calls share
+// the one array and it keeps the contents of the last call: calls that can overlap on the GPU
+// (different streams, or different host threads) race on it and must be serialised by the caller.
+// Nothing in it has to start at zero -- each call writes every byte its kernels read (the uploaded
+// work lists, then the partials) before reading it.
+#include <cuda.h>
+
 #include <cstdio>
 #include <mutex>
 
@@ -26,10 +30,35 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_ws[PKV_STATIC_WS_BYTES];
 
-// Device address of g_static_ws for the current device (host code may not use the symbol itself).
+// Unique id of the calling thread's current CUDA context (0 if it cannot be read).
+unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrent)(CUcontext*);
+    typedef CUresult (*GetId)(CUcontext, unsigned long long*);
+    static std::once_flag once;
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_static_ws for the current device and context (host code may not use the
+// symbol itself: in host code its name is a host-side stand-in, not a device address).
 void* static_ws_address(pkv_status* st) {
     static std::mutex mu;
     static void* addr[64] = {nullptr};
+    static unsigned long long ctx_of[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) {
@@ -37,8 +66,9 @@ void* static_ws_address(pkv_status* st) {
         *st = PKV_ERR_CUDA;
         return nullptr;
     }
+    const unsigned long long ctx = current_context_id();  // 0 while no context is current yet
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || ctx == 0 || ctx != ctx_of[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_ws);
         if (e != cudaSuccess || !p) {
@@ -47,6 +77,7 @@ void* static_ws_address(pkv_status* st) {
             return nullptr;
         }
         addr[dev] = p;
+        ctx_of[dev] = current_context_id();  // the lookup made the device's context current
     }
     *st = PKV_OK;
     return addr[dev];
@@ -60,24 +91,23 @@ extern "C" pkv_status pkv_paged_attention_static_ws(
     int head_dim, pkv_dtype dtype, const pkv_plan_options* opts, void* out, const void* q, const void* k_pool,
     const void* v_pool, const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
     const int32_t* query_start_loc, int num_blocks, float scale, pkv_stream_t stream) {
-    size_t need = 0;
-    pkv_status st = pkv_attention_workspace_size(h_query_start_loc, h_context_lens, num_reqs, num_q_heads,
-                                                 num_kv_heads, head_dim, dtype, opts, &need);
-    if (st != PKV_OK) return st;
-    if (need > (size_t)PKV_STATIC_WS_BYTES) {
-        char msg[256];
-        snprintf(msg, sizeof msg,
-                 "batch needs %zu bytes of scratch, above the static workspace limit of %zu bytes "
-                 "(use pkv_attention_plan with a caller workspace, or larger split_blocks)",
-                 need, (size_t)PKV_STATIC_WS_BYTES);
-        pkv::set_last_error(msg);
-        return PKV_ERR_WORKSPACE_TOO_SMALL;
-    }
+    pkv_status st = PKV_OK;
     void* ws = pkv::static_ws_address(&st);
     if (!ws) return st;
+    // One planning pass: the planner refuses a batch whose scratch exceeds the array before it
+    // uploads anything.
     pkv_plan plan;
     st = pkv_attention_plan(h_query_start_loc, h_context_lens, num_reqs, num_q_heads, num_kv_heads, head_dim, dtype,
                             opts, ws, PKV_STATIC_WS_BYTES, &plan, stream);
+    if (st == PKV_ERR_WORKSPACE_TOO_SMALL) {
+        char msg[256];
+        snprintf(msg, sizeof msg,
+                 "batch needs %lld bytes of scratch, above the static workspace limit of %zu bytes "
+                 "(use pkv_attention_plan with a caller workspace, or larger split_blocks)",
+                 (long long)plan.ws_bytes, (size_t)PKV_STATIC_WS_BYTES);
+        pkv::set_last_error(msg);
+        return st;
+    }
     if (st != PKV_OK) return st;
     return pkv_paged_attention(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens,
                                query_start_loc, num_blocks, scale, &plan, ws, PKV_STATIC_WS_BYTES, stream);

@@ -210,6 +210,25 @@ def test_device_error_on_out_of_range_table_entry(dev):
     assert code == 6 and detail >= 0
 
 
+def test_device_lengths_beyond_the_table_are_reported(dev):
+    """The prefill tiles take each request's context from the device lengths. When those exceed
+    what the host plan (and the table's width) covers, the entries past the table are not read:
+    the kernel zero-fills those keys and records a range error."""
+    from paged_kv_cache_446_b200 import pkv
+    wl = custom(dev, "bf16", 64, 8, 128, [(300, 80)])
+    assert wl.block_tables.shape[1] == 24                  # ceil(380 / 16) blocks: the table's width
+    plan = pkv.AttentionPlan(wl.batch, wl.prior_lens, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                             W.TORCH_DTYPES[wl.dtype], dev, tc_min_rows=2)
+    assert plan.plan.num_tiles > 0
+    bt = torch.from_numpy(wl.block_tables).to(dev)
+    plan.context_lens.add_(64)                             # 444 tokens: 28 blocks on the device
+    out = pkv.paged_attention(plan, wl.q, wl.k_pool, wl.v_pool, bt, wl.scale)
+    torch.cuda.synchronize()
+    code, detail = pkv.device_error()
+    assert code == 6 and detail >= 24, (code, detail)
+    assert torch.isfinite(out.float()).all()
+
+
 PREFILL_CASES = [
     ("bf16", 64, 8, 128, [(0, 512)]),                              # first 512-row chunk, G = 8
     ("bf16", 64, 8, 128, [(300, 80), (0, 1), (17, 33)]),           # mixed rows, ragged tiles

@@ -4,8 +4,10 @@ Such callers (an engine whose memory manager already holds nearly all of HBM, a 
 runtime that owns every allocation, code where allocation calls are forbidden) get the planner's
 work lists and the split-K partials placed in a library-owned device array instead of a workspace
 they would have to allocate. This test calls the entry point through the C ABI, twice in a row, and
-checks each result against the workspace-based entry point on the same inputs. It also checks that
-a batch needing more scratch than the array holds is refused on the host before any launch.
+checks each result against the workspace-based entry point on the same inputs (the same plan and the
+same deterministic kernels, so the two must agree bit for bit) and against the CPU oracle within the
+attention tolerance. It also checks that a batch needing more scratch than the array holds is
+refused on the host before any launch.
 """
 import ctypes
 
@@ -13,7 +15,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_harness import TOL
+import oracle
+from gpu_harness import TOL, max_err, storage
 
 pytestmark = pytest.mark.gpu
 
@@ -49,13 +52,22 @@ def test_static_workspace_matches_workspace_entry(config, small):
     plan = pkv.AttentionPlan(wl.batch, wl.prior_lens, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, dt, dev)
     ref = pkv.paged_attention(plan, wl.q, wl.k_pool, wl.v_pool, bt, wl.scale)
     stream = torch.cuda.current_stream().cuda_stream
+    # The oracle on host copies of the same inputs (every row of the small cases, sampled rows of
+    # the full-size one).
+    qsl, ctx = oracle.flatten_batch(wl.batch, wl.prior_lens)
+    T = int(qsl[-1])
+    rows = None if small else np.random.default_rng(3).choice(T, size=min(T, 8), replace=False).astype(np.int32)
+    expect = oracle.paged_attention(storage(wl.q), storage(wl.k_pool), storage(wl.v_pool), wl.block_tables, ctx, qsl,
+                                    wl.scale, wl.dtype, rows=rows)
     for _ in range(2):
         out = torch.full_like(wl.q, float("nan"))
         status = _call(pkv, f, wl, plan, bt, out, stream)
         assert status == 0, pkv._lib.pkv_last_error().decode()
         torch.cuda.synchronize()
-        err = (out.double() - ref.double()).abs().max().item()
-        assert err <= TOL[wl.dtype], f"{wl.name}: max |err| {err}"
+        assert torch.equal(out, ref), f"{wl.name}: differs from the workspace entry point"
+        got = out if rows is None else out[torch.as_tensor(rows, device=dev, dtype=torch.long)]
+        err = max_err(got, expect)
+        assert err <= TOL[wl.dtype], f"{wl.name}: max |err| {err} against the oracle"
     code, detail = pkv.device_error()
     assert code == 0, (code, detail)
 
