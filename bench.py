@@ -64,6 +64,9 @@ def parse():
     ap.add_argument("--cuda-core-only", action="store_true", help="serve every row on CUDA cores")
     ap.add_argument("--decode-kernel", type=int, default=0, choices=[0, 1, 2],
                     help="kernel for split-K rows: 0 planner's choice, 1 FMA, 2 warp MMA")
+    ap.add_argument("--decode-sms", type=int, default=0,
+                    help="mixed batches: SMs of the split-K kernel running beside the tcgen05 tiles "
+                         "(0 planner's choice, -1 the two kernels one after the other)")
     return ap.parse_args()
 
 
@@ -356,6 +359,8 @@ def main():
         opts["cuda_core_only"] = True
     if args.decode_kernel:
         opts["decode_kernel"] = args.decode_kernel
+    if args.decode_sms:
+        opts["decode_sms"] = args.decode_sms
     step = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,
                               wl.num_kv_heads, wl.head_dim, dt, dev, write_batch=wl.write_batch or None,
                               copy_pairs=wl.copy_pairs, **opts)
@@ -409,6 +414,26 @@ def main():
     torch.cuda.synchronize()
     prof = pkv.profile_stop()
     ms_per_step = max_over_ranks(ms_total, dist, dev) / args.steps
+    # When the step runs its split-K kernel beside the tcgen05 tiles, the intervals above are the
+    # two kernels' overlapped spans; each kernel's own roofline comes from the same steps launched
+    # one kernel after the other.
+    prof_alone, run_alone = prof, run_step
+    if step.plan.plan.decode_sms > 0:
+        serial = PagedAttentionStep(wl.batch, wl.prior_lens, wl.block_tables, wl.num_blocks, wl.num_q_heads,
+                                    wl.num_kv_heads, wl.head_dim, dt, dev, write_batch=wl.write_batch or None,
+                                    copy_pairs=wl.copy_pairs, **dict(opts, decode_sms=-1))
+
+        def run_alone():
+            serial.run(wl.q, wl.k_pool, wl.v_pool, wl.scale, wl.k_new, wl.v_new, out=out)
+
+        for _ in range(args.warmup):
+            run_alone()
+        torch.cuda.synchronize()
+        pkv.profile_start(capacity=16 * args.steps + 16)
+        for _ in range(args.steps):
+            run_alone()
+        torch.cuda.synchronize()
+        prof_alone = pkv.profile_stop()
     code, detail = pkv.device_error()
     assert code == 0, f"device error {code} at {detail}"
 
@@ -435,7 +460,7 @@ def main():
         pkv.profile_start(capacity=16 * args.steps + 16)
         for _ in range(args.steps):
             flush_buf.fill_(1)
-            run_step()
+            run_alone()
         torch.cuda.synchronize()
         prof_flushed = pkv.profile_stop()
         del flush_buf
@@ -547,9 +572,9 @@ def main():
     tc_peak, tc_kind = tensor_peak()
     rooflines = {}
     for k, w in work.items():
-        if not prof[k][1]:
+        if not prof_alone[k][1]:
             continue
-        avg_ms = prof[k][0] / prof[k][1]
+        avg_ms = prof_alone[k][0] / prof_alone[k][1]
         kname = "decode_mma_kernel" if (k == "decode" and step.plan.plan.decode_kernel == 2) else k + "_kernel"
         if k == "prefill_tc":
             achieved = w["flops"] / (avg_ms * 1e-3) / 1e12
@@ -562,14 +587,17 @@ def main():
             r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                  "traffic": recorded_traffic(kname, wl.name), "algorithmic_bytes": w["bytes"],
                  "peak_source": f"{peak_kind} hbm_gbs (burst copy)"}
-        r.update(kernel=kname, kernel_ms=avg_ms, launches_per_step=prof[k][1] / max(1, args.steps))
+        r.update(kernel=kname, kernel_ms=avg_ms, launches_per_step=prof_alone[k][1] / max(1, args.steps),
+                 timed="alone (kernels one after the other)" if prof_alone is not prof else "in the step")
+        if prof_alone is not prof and prof[k][1]:
+            r["kernel_ms_overlapped"] = prof[k][0] / prof[k][1]
         if prof_flushed and prof_flushed[k][1]:
             fms = prof_flushed[k][0] / prof_flushed[k][1]
             r["l2_flushed"] = {"kernel_ms": fms, "frac": r["frac"] * avg_ms / fms}
         rooflines[k] = r
     roof = None
     if rooflines:
-        dom = max(rooflines, key=lambda k: prof[k][0])
+        dom = max(rooflines, key=lambda k: prof_alone[k][0])
         roof = dict(rooflines[dom])
     # The step's own bound: every K/V byte once at the HBM peak, or every prefill flop at the tensor
     # peak, whichever is longer (the two can overlap in one step).
@@ -589,7 +617,7 @@ def main():
                    "l2": "inputs larger than L2 (KV pool read per step >> 126 MB); value taken without a "
                          "flush, l2_flushed taken with a 2 x L2 write between steps",
                    "parallelism": f"replicas x{world} (independent requests per GPU)",
-                   "plan_options": opts},
+                   "plan_options": opts, "decode_sms": int(step.plan.plan.decode_sms)},
         "frac_of_hbm_peak": value / world / peak,
         "frac_of_8tbs_spec": value / world / 8000.0,
         "kv_block_waste": pool_waste(wl),

@@ -141,6 +141,13 @@ typedef struct pkv_plan_options {
     const int32_t* h_block_tables;   /* host copy of block_tables, or NULL (no sharing) */
     int32_t block_table_stride;      /* its row length (max_blocks_per_seq) */
     int32_t min_shared_blocks;       /* 0 = 4 */
+    /* Mixed batches (tcgen05 tiles and warp-MMA split-K items in one plan): the tile kernel's
+     * persistent CTAs (one per SM) serve both queues in one launch -- decode_sms of them start on
+     * the split-K items and the others on the tiles, and each turns to the other queue once its own
+     * is empty -- so the tensor-bound tiles and the HBM-bound items share the GPU. 0 = sized by the
+     * planner from the two parts' estimated times; -1 = no overlap (the split-K kernel runs after
+     * the tiles). */
+    int32_t decode_sms;
 } pkv_plan_options;
 
 /*
@@ -174,6 +181,10 @@ typedef struct pkv_plan {
                                     with a prefix shared by a run of requests counted once */
     int64_t tile_kv_bytes;       /* part of kv_bytes read by the tcgen05 tiles */
     int64_t tile_flops;          /* part of attn_flops computed by the tcgen05 tiles */
+    int32_t decode_sms;          /* > 0: one launch of the tile kernel also serves the split-K items,
+                                    with this many CTAs starting on them; 0: the split-K kernel runs
+                                    after the tiles */
+    int32_t pad0;
 } pkv_plan;
 
 /*
@@ -252,10 +263,13 @@ pkv_status pkv_attention_plan_async(const int32_t* h_query_start_loc, const int3
  *   out[row][h][:] = sum_t softmax_t(scale * q[row][h] . K_r[t]) V_r[t],  t = 0 .. ctx_r - n_r + j
  * with K_r[t] = k_pool[block_tables[r][t/16]][h / (Hq/Hkv)][t%16]. Softmax and accumulation in fp32;
  * the output is rounded to the element type. Launches, on `stream`: the tcgen05 prefill tile
- * kernel (if the plan has tiles), the split-K decode kernel the plan names (warp-MMA or FMA, if
- * it has items) and the
- * log-sum-exp merge kernel (if it has merge rows). The plan and workspace must come from
- * pkv_attention_plan with the same batch; q/out shapes must match it.
+ * kernel (if the plan has tiles; persistent CTAs, one per SM, taking tiles longest first), the
+ * split-K decode kernel the plan names (warp-MMA or FMA, if it has items) -- or, when
+ * plan->decode_sms > 0, one tile-kernel launch that serves the warp-MMA items as well -- and the
+ * log-sum-exp merge kernel (if it has merge rows). The kernels take their work from ticket
+ * counters in the workspace header, which the plan upload zeroes and each launch leaves at zero.
+ * The plan and workspace must come from pkv_attention_plan with the same batch; q/out shapes must
+ * match it; launches sharing one workspace must not overlap on the GPU.
  * Errors: INVALID_ARG (null pointers, plan magic/shape mismatch), WORKSPACE_TOO_SMALL, CUDA.
  */
 pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, const void* v_pool,

@@ -8,6 +8,8 @@
 #include <string>
 #include <vector>
 
+#include <cuda.h>
+
 #include "internal.h"
 #include "pkv.h"
 
@@ -245,13 +247,13 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     }
     auto pieces_of = [&](const CoreRow& c) { return (int)ceil_div(c.be - c.bs, chunk); };
     auto with_partials = [&](const CoreRow& c, int pieces) { return c.kind != 0 || pieces > 1; };
-    // Items are placed directly at their position in a stable order by length, longest first,
-    // dealt to the persistent warps (warp w runs positions w, w + W, w + 2W, ...) in a snake: each
-    // odd round of W items is dealt in reverse, so the warps that took the longest items of one
-    // round take the shortest of the next and the warps' totals even out. Pass 1 counts the items
-    // of each length from the row lengths alone; pass 2 writes every item to its slot. W is the
-    // resident warp count of the decode kernels (8 per SM); a launch with another count still runs
-    // every item.
+    // Items are placed directly at their position in a stable order by length, longest first. For
+    // the FMA kernel, whose persistent warps run fixed positions (warp w runs w, w + W, w + 2W, ...),
+    // they are dealt in a snake: each odd round of W items is dealt in reverse, so the warps that
+    // took the longest items of one round take the shortest of the next and the warps' totals even
+    // out (W = 8 resident warps per SM; a launch with another count still runs every item). Pass 1
+    // counts the items of each length from the row lengths alone; pass 2 writes every item to its
+    // slot.
     size_t n_items = 0, n_merge = 0;
     int max_len = 0;
     for (const CoreRow& c : core_rows) {
@@ -278,7 +280,9 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     // Dealing cursors: the items of length `len` take the sorted positions start[len], +1, ...;
     // each cursor keeps its position as (round, index in the round) so the snake needs no
     // division per item.
-    const uint32_t deal = (uint32_t)std::max(num_sms, 1) * 8;
+    // The warp-MMA kernel takes items greedily from a ticket counter: plain longest-first order
+    // (one round). The FMA kernel's warps run fixed positions: the snake over its W warps.
+    const uint32_t deal = kind == 2 ? (uint32_t)std::max<size_t>(n_items, 1) : (uint32_t)std::max(num_sms, 1) * 8;
     const uint32_t n_items32 = (uint32_t)n_items;  // the plan counts items in int32
     std::vector<PlanLists::Cursor>& cursor = L->cursor;
     cursor.resize((size_t)max_len + 2);
@@ -409,6 +413,28 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->core_kv_bytes = kv_bytes - tile_kv - shared_saved_tokens * Hkv * 2 * D * eb;
     plan->tile_kv_bytes = tile_kv;
     plan->tile_flops = tile_flops;
+    // Mixed batch: the tcgen05 kernel's persistent CTAs (one per SM) also serve the warp-MMA items;
+    // decode_sms of them start on items, the rest on tiles, and each turns to the other queue when
+    // its own empties. Automatic share: the items' part of the two parts' estimated SM time (a key
+    // tile of a CTA ~2.5 us at the tiles' measured tensor rate; an SM streaming items ~100 GB/s when
+    // the HBM is not saturated), but never so many that a tile longer than half the estimated step
+    // has to wait for a CTA: every such tile gets one from the start.
+    plan->decode_sms = 0;
+    if (o.decode_sms >= 0 && kind == 2 && n_items > 0 && !L->tiles.empty() && num_sms >= 2) {
+        int nd = o.decode_sms;
+        if (nd == 0) {
+            constexpr double kKeyTileSec = 2.5e-6, kItemBytesPerSec = 100e9;
+            double t_p = 0.0;
+            for (const PrefillTile& t : L->tiles) t_p += t.key_tiles * kKeyTileSec;
+            const double t_d = (double)plan->core_kv_bytes / kItemBytesPerSec;
+            const double t_step = (t_p + t_d) / num_sms;
+            int n_long = 0;
+            for (const PrefillTile& t : L->tiles) n_long += t.key_tiles * kKeyTileSec > 0.5 * t_step;
+            if (t_d > 20e-6 * num_sms && t_p > 20e-6 * num_sms)  // each part worth overlapping
+                nd = std::min((int)std::lround(num_sms * t_d / (t_p + t_d)), num_sms - n_long);
+        }
+        if (nd > 0) plan->decode_sms = std::min(nd, num_sms - 1);
+    }
     return PKV_OK;
 }
 
@@ -467,6 +493,30 @@ struct ProfileScope {
 }  // namespace
 
 void set_last_error(const char* msg) { t_last_error = msg ? msg : ""; }
+
+unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrent)(CUcontext*);
+    typedef CUresult (*GetId)(CUcontext, unsigned long long*);
+    static std::once_flag once;
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+
 
 DeviceError* device_error_word() {
     static std::mutex mu;
@@ -681,35 +731,46 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
     const float scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t s = (cudaStream_t)stream;
     const int G = plan->num_q_heads / plan->num_kv_heads;
+    // Mixed batch: the tcgen05 kernel's persistent CTAs also serve the warp-MMA split-K items
+    // (plan->decode_sms of them start on items, the others on tiles; each turns to the other queue
+    // once its own is empty), so the HBM-bound items and the tensor-bound tiles share the GPU.
+    const bool mixed = plan->decode_sms > 0 && plan->num_tiles > 0 && plan->num_items > 0 && plan->decode_kernel == 2;
+    int* work = reinterpret_cast<int*>(ws);  // the header's first 16 bytes: zeroed by the plan upload
+    DecodeArgs d{};
+    d.q = q; d.out = out; d.k_pool = k_pool; d.v_pool = v_pool; d.block_tables = block_tables;
+    d.items = reinterpret_cast<const DecodeItem*>(ws + plan->off_items);
+    d.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
+    d.part_ml = reinterpret_cast<float*>(ws + plan->off_part_ml);
+    d.err = err; d.work = work; d.num_items = plan->num_items; d.max_blocks_per_seq = max_blocks_per_seq;
+    d.num_blocks = num_blocks; d.num_q_heads = plan->num_q_heads; d.num_kv_heads = plan->num_kv_heads;
+    d.group = G; d.heads_per_item = plan->heads_per_item;
+    d.slots_per_item = plan->heads_per_item * std::max(plan->rows_per_item, 1);
+    d.part_stride = plan->part_stride;
+    d.scale_log2 = scale_log2;
+    d.pdl = true;
+    pkv_status st = PKV_OK;
     if (plan->num_tiles > 0) {
         PrefillArgs a{};
         a.q = q; a.out = out; a.k_pool = k_pool; a.v_pool = v_pool; a.block_tables = block_tables;
         a.context_lens = context_lens; a.query_start_loc = query_start_loc;
         a.tiles = reinterpret_cast<const PrefillTile*>(ws + plan->off_tiles);
-        a.err = err; a.num_tiles = plan->num_tiles; a.max_blocks_per_seq = max_blocks_per_seq;
+        a.err = err; a.work = work; a.decode_ctas = mixed ? plan->decode_sms : 0;
+        a.num_tiles = plan->num_tiles; a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks; a.num_q_heads = plan->num_q_heads; a.num_kv_heads = plan->num_kv_heads;
-        a.group = G; a.num_q_tokens = plan->num_q_tokens; a.scale_log2 = scale_log2;
+        a.group = G; a.num_q_tokens = plan->num_q_tokens; a.scale_log2 = scale_log2; a.pdl = true;
+        DecodeArgs none = d;
+        none.num_items = 0;
         ProfileScope prof(PKV_KERNEL_PREFILL_TC, s);
-        cudaError_t e = launch_prefill_tc(plan->dtype, a, sms, s);
-        if (e != cudaSuccess) return cuda_fail(e, "prefill tile launch");
+        cudaError_t e = launch_prefill_tc(plan->dtype, a, mixed ? d : none, sms, s);
+        if (e != cudaSuccess) st = cuda_fail(e, "prefill tile launch");
     }
-    if (plan->num_items > 0) {
-        DecodeArgs a{};
-        a.q = q; a.out = out; a.k_pool = k_pool; a.v_pool = v_pool; a.block_tables = block_tables;
-        a.items = reinterpret_cast<const DecodeItem*>(ws + plan->off_items);
-        a.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
-        a.part_ml = reinterpret_cast<float*>(ws + plan->off_part_ml);
-        a.err = err; a.num_items = plan->num_items; a.max_blocks_per_seq = max_blocks_per_seq;
-        a.num_blocks = num_blocks; a.num_q_heads = plan->num_q_heads; a.num_kv_heads = plan->num_kv_heads;
-        a.group = G; a.heads_per_item = plan->heads_per_item;
-        a.slots_per_item = plan->heads_per_item * std::max(plan->rows_per_item, 1);
-        a.part_stride = plan->part_stride;
-        a.scale_log2 = scale_log2;
+    if (st == PKV_OK && plan->num_items > 0 && !mixed) {
         ProfileScope prof(PKV_KERNEL_DECODE, s);
-        cudaError_t e = plan->decode_kernel == 2 ? launch_decode_mma(plan->dtype, a, sms, s)
-                                                 : launch_decode(plan->dtype, plan->head_dim, a, sms, s);
-        if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+        cudaError_t e = plan->decode_kernel == 2 ? launch_decode_mma(plan->dtype, d, sms, s)
+                                                 : launch_decode(plan->dtype, plan->head_dim, d, sms, s);
+        if (e != cudaSuccess) st = cuda_fail(e, "decode launch");
     }
+    if (st != PKV_OK) return st;
     if (plan->num_merge_rows > 0) {
         MergeArgs m{};
         m.out = out;
@@ -722,6 +783,7 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
         // item (a shared-prefix item packs several requests' rows; each member's merge row is one).
         m.slots_per_entry = std::max(plan->merge_slots, 1);
         m.part_stride = plan->part_stride;
+        m.pdl = true;
         ProfileScope prof(PKV_KERNEL_MERGE, s);
         cudaError_t e = launch_merge(plan->dtype, plan->head_dim, m, s);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");

@@ -244,9 +244,12 @@ __device__ __forceinline__ DecodeItem load_item(const DecodeItem* items, int i) 
 // predecessor has completed and its memory is visible (immediately when launched normally).
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Launches `kernel` on `s` with the programmatic-stream-serialisation attribute.
+// Launches `kernel` on `s`, with the programmatic-stream-serialisation attribute when `pdl` is set
+// (the kernel may then start while its predecessor on `s` finishes; it waits in griddep_wait()).
+// Launches that follow an event wait on a side stream go without it.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+cudaError_t launch_k(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -256,8 +259,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+    return launch_k(true, kernel, grid, block, smem, s, std::forward<Args>(args)...);
 }
 
 }  // namespace pkv

@@ -504,7 +504,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     int grid = num_sms * per_sm;
     if (grid > need) grid = need;
     if (grid < 1) return cudaSuccess;
-    return launch_pdl(decode_kernel<T, D, GP, NSTAGE>, dim3(grid), dim3(kDecodeWarps * 32), smem, s, a);
+    return launch_k(a.pdl, decode_kernel<T, D, GP, NSTAGE>, dim3(grid), dim3(kDecodeWarps * 32), smem, s, a);
 }
 
 // Ring depth: the default per group size, or PKV_DECODE_STAGES (2..4) as a tuning override.
@@ -546,8 +546,8 @@ cudaError_t launch_merge_d(int head_dim, const MergeArgs& a, cudaStream_t s) {
     const long long warps = (long long)a.num_rows * a.slots_per_entry;
     const int grid = (int)((warps * 32 + 127) / 128);
     if (grid < 1) return cudaSuccess;
-    if (head_dim == 64) return launch_pdl(merge_kernel<T, 64>, dim3(grid), dim3(128), 0, s, a);
-    return launch_pdl(merge_kernel<T, 128>, dim3(grid), dim3(128), 0, s, a);
+    if (head_dim == 64) return launch_k(a.pdl, merge_kernel<T, 64>, dim3(grid), dim3(128), 0, s, a);
+    return launch_k(a.pdl, merge_kernel<T, 128>, dim3(grid), dim3(128), 0, s, a);
 }
 
 }  // namespace

@@ -72,6 +72,7 @@ struct DecodeArgs {
     float* part_o;       // [num_partials][part_stride][D]
     float* part_ml;      // [num_partials][part_stride][2] (max in log2 units, sum)
     DeviceError* err;
+    int* work;           // warp-MMA items: [0] item ticket counter, [1] finished warps (zero at launch)
     int num_items;
     int max_blocks_per_seq;
     int num_blocks;
@@ -82,6 +83,7 @@ struct DecodeArgs {
     int slots_per_item;  // largest num_rows x heads of any item: selects the kernel variant
     int part_stride;     // slots per partial-result entry (8 for the FMA kernel, 16 for the MMA kernel)
     float scale_log2;    // scale * log2(e)
+    bool pdl;            // launch with programmatic dependent launch (false after an event wait)
 };
 
 struct MergeArgs {
@@ -93,6 +95,7 @@ struct MergeArgs {
     int num_q_heads;
     int slots_per_entry;  // largest num_slots of any merge row: warps launched per row
     int part_stride;      // slots per partial-result entry
+    bool pdl;             // launch with programmatic dependent launch (false after an event wait)
 };
 
 struct PrefillArgs {
@@ -105,6 +108,8 @@ struct PrefillArgs {
     const int32_t* query_start_loc;
     const PrefillTile* tiles;
     DeviceError* err;
+    int* work;           // [2] tile ticket counter, [3] finished CTAs (zero at launch)
+    int decode_ctas;     // CTAs that start on the split-K items passed beside the tiles
     int num_tiles;
     int max_blocks_per_seq;
     int num_blocks;
@@ -113,6 +118,7 @@ struct PrefillArgs {
     int group;
     int num_q_tokens;
     float scale_log2;
+    bool pdl;            // launch with programmatic dependent launch (false after an event wait)
 };
 
 // Launchers (return the launch error, if any).
@@ -120,7 +126,9 @@ cudaError_t launch_decode(int dtype, int head_dim, const DecodeArgs& a, int num_
 cudaError_t launch_merge(int dtype, int head_dim, const MergeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_mma(int dtype, const DecodeArgs& a, int num_sms, cudaStream_t s);
 bool decode_mma_supported(int dtype, int head_dim);
-cudaError_t launch_prefill_tc(int dtype, const PrefillArgs& a, int num_sms, cudaStream_t s);
+// The tcgen05 tile kernel: persistent CTAs over the tiles and, when d.num_items > 0, the split-K
+// items of d (warp-MMA kind) as well.
+cudaError_t launch_prefill_tc(int dtype, const PrefillArgs& a, const DecodeArgs& d, int num_sms, cudaStream_t s);
 bool prefill_tc_supported(int dtype, int head_dim, int group);
 cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, const int32_t* qsl, const int32_t* ctx,
                                 int num_reqs, int num_blocks, int64_t* slots, int num_tokens, DeviceError* err,
@@ -137,5 +145,9 @@ DeviceError* device_error_word();
 
 // Replaces the calling thread's pkv_last_error() message.
 void set_last_error(const char* msg);
+
+// Unique id of the calling thread's current CUDA context (0 when none is current or the driver
+// cannot say).
+unsigned long long current_context_id();
 
 }  // namespace pkv

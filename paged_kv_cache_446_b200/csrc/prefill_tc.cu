@@ -9,7 +9,7 @@
 //
 // CTA: two 128-row MMA tiles (A, B), each (128/G) consecutive query rows x the G query heads of one
 // KV head (GQA packing), sharing one stream of 128-key K/V tiles (8 blocks), so every K/V byte
-// fetched from L2 serves 256 rows. Warp roles (320 threads):
+// fetched from L2 serves 256 rows. Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: one thread per row
 //   warp  8    TMA producer: both Q tiles once (3-D tensor map, SWIZZLE_128B), then per key tile
 //              8 blocks x 2 column halves of K and of V (2-D tensor map over the pool rows),
@@ -17,13 +17,20 @@
 //   warp  9    MMA issuer (one thread): S_X = Q_X K^T into TMEM; after softmax X has written
 //              P_X (16-bit, over the first 64 columns of S_X), O_X += P_X V with A read from TMEM.
 //              The two tiles ping-pong: one tile's softmax overlaps the other tile's MMAs.
+//   warps 10-11 idle; they complete the third warpgroup, whose registers move to the softmax
+//              warpgroups (setmaxnreg).
+// The CTAs are persistent (one per SM): they take tiles, longest first, from a ticket counter. In a
+// mixed batch they also serve the split-K decode items (warps 0-7 run the warp-MMA loop of
+// decode_mma.cuh over buffers carved from the tile stages), so the HBM-bound decode rows and the
+// tensor-bound tiles share the GPU in one launch.
+// A softmax thread reads its row's key tile in two halves of 64 columns (one TMEM round trip each).
 // O accumulates in TMEM across key tiles. A row's exponentials use a reference maximum that is
 // raised only when a tile's maximum exceeds it by 2^8; O is then rescaled in TMEM (exact: softmax is
 // shift invariant, and p stays <= 2^8).
 // Blocks past the context are fetched at an out-of-range coordinate (TMA fills zeros); V rows past
 // the context inside the last block are zeroed before PV (stale slots may hold anything).
 // Every wait is bounded; on expiry the CTA records PKV_ERR_DEVICE_TIMEOUT, drains its own copies
-// and MMAs (bounded), frees its tensor memory and returns. No TMA multicast.
+// and MMAs (bounded), frees its tensor memory and stops taking work. No TMA multicast.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -32,12 +39,20 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "decode_mma.cuh"
 #include "tma_host.h"
 
 namespace pkv {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Registers per thread after the split (setmaxnreg): the third warpgroup gives up registers so the
+// two softmax warpgroups may grow. The launch holds kThreads x 168 registers (the most 384 threads
+// get: three warps share each SM sub-partition's 16384); the split needs exactly as many,
+// 2 x 128 x 216 + 128 x 72 = 64512 = 384 x 168, so the growing warpgroups never wait for more than
+// the shrinking one releases. ptxas fits both regions without spilling at these counts.
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
 constexpr int kHalf = 128 * 128;        // 128 rows x 64 elements x 2 bytes
 constexpr int kTile = 2 * kHalf;        // 128 x 128 x 2 bytes
 constexpr int OFF_Q = 0;                // Q_A, Q_B
@@ -51,8 +66,16 @@ enum {
 };
 constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;     // tcgen05.alloc result
 constexpr int OFF_ABORT = OFF_TMEM + 4;
-constexpr int SMEM_USED = OFF_ABORT + 12;
+constexpr int OFF_CTRL = OFF_ABORT + 4;              // the CTA's next step (thread 0 writes it)
+// Rounds of split-K items: warps 0-7 each use kDecodeStages stages of the tile buffers (8 x 2 x 12 KiB
+// = 192 KiB, below OFF_BAR), with their own mbarriers and item rings after the tile barriers.
+constexpr int kDecodeStages = 2;
+constexpr int OFF_DBAR = OFF_TMEM + 16;
+constexpr int OFF_FIFO = OFF_DBAR + 8 * kDecodeStages * 8;
+constexpr int SMEM_USED = OFF_FIFO + 8 * mma::kFifo * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;         // slack to align the base to 1024 bytes
+static_assert(8 * kDecodeStages * mma::kStage <= OFF_BAR, "split-K stages overlap the tile barriers");
+static_assert(OFF_DBAR % 8 == 0, "mbarrier alignment");
 constexpr uint32_t kTmemCols = 512;                  // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 // A row's exponentials use a reference max that is only raised when the tile max exceeds it by
 // more than this (log2 units); the result is exact (softmax is shift invariant) and p <= 2^8.
@@ -157,6 +180,21 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     return true;
 }
 
+// Three-input maximum / minimum (one instruction on sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float min3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// CTA-wide barrier 0 that the warps may reach at different instructions (the two register-split
+// branches each end with one).
+__device__ __forceinline__ void cta_sync() { asm volatile("barrier.sync 0;" ::: "memory"); }
+
 // Warp-uniform "all succeeded" for the lanes of one warp.
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(FULL_MASK, v); }
 
@@ -172,48 +210,404 @@ __device__ __forceinline__ float2 row_sum_term(float2 p, uint32_t packed) {
     else return p;
 }
 
+// What every role needs to know about one tile (request, KV head, 2 x 128 packed rows).
+struct TileCtx {
+    int req, kvh, tok0, q0, n, ctx, prior, G, tt, nkt, nblk_ctx, rows_total;
+    int nkt_x[2];   // key tiles each MMA tile needs: keys visible to its last valid row
+    bool has_b, sane;
+};
+
+__device__ __forceinline__ TileCtx tile_ctx(const PrefillArgs& a, int t) {
+    TileCtx c;
+    const PrefillTile pt = a.tiles[t];
+    c.req = pt.req;
+    c.kvh = pt.kv_head;
+    c.tok0 = pt.tok0;
+    c.q0 = a.query_start_loc[c.req];
+    c.n = a.query_start_loc[c.req + 1] - c.q0;
+    c.ctx = a.context_lens[c.req];
+    c.prior = c.ctx - c.n;
+    c.G = a.group;
+    c.tt = 128 / c.G;
+    c.has_b = c.tok0 + c.tt < c.n;
+    c.nkt_x[0] = (min(c.ctx, c.prior + min(c.n, c.tok0 + c.tt)) + 127) / 128;
+    c.nkt_x[1] = c.has_b ? (min(c.ctx, c.prior + min(c.n, c.tok0 + 2 * c.tt)) + 127) / 128 : 0;
+    c.nkt = max(c.nkt_x[0], c.nkt_x[1]);
+    c.nblk_ctx = (c.ctx + kBlockSize - 1) / kBlockSize;
+    c.rows_total = a.num_blocks * a.num_kv_heads * kBlockSize;
+    c.sane = c.nkt >= 1 && c.n > 1 && c.tok0 < c.n;
+    return c;
+}
+
+// Arms the tile barriers for a new tile (thread 0; they are idle: the previous tile waited for
+// every phase it started).
+__device__ __forceinline__ void init_tile_barriers(uint64_t* bars) {
+    mbar_init(&bars[B_Q], 1);
+    for (int s = 0; s < 2; ++s) {
+        mbar_init(&bars[B_KF0 + s], 1);
+        mbar_init(&bars[B_VF0 + s], 1);
+        mbar_init(&bars[B_KE0 + s], 1);
+        mbar_init(&bars[B_VE0 + s], 1);
+        mbar_init(&bars[B_SF0 + s], 1);
+        mbar_init(&bars[B_PF0 + s], 128);
+        mbar_init(&bars[B_OF0 + s], 1);
+    }
+    mbar_init(&bars[B_DRAIN], 1);
+    fence_mbar_init();
+}
+
+// ---- TMA producer (warp 8) ----
+__device__ __forceinline__ void tile_producer(const PrefillArgs& a, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                              const CUtensorMap* tm_v, unsigned char* smem, uint64_t* bars,
+                                              volatile int* abort_flag, const TileCtx& tile, int lane) {
+    if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[B_Q], tile.has_b ? 2 * kTile : kTile);
+        for (int x = 0; x < (tile.has_b ? 2 : 1); ++x) {
+            const int z = tile.q0 + tile.tok0 + x * tile.tt;
+            tma_load_3d(smem + OFF_Q + x * kTile, tm_q, 0, tile.kvh * tile.G, z, &bars[B_Q]);
+            tma_load_3d(smem + OFF_Q + x * kTile + kHalf, tm_q, 64, tile.kvh * tile.G, z, &bars[B_Q]);
+        }
+    }
+    int ids = -1, ids_base = -1;
+    int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
+    bool ok = true;
+    for (int kt = 0; kt < tile.nkt && ok; ++kt) {
+        const int s = kt & 1;
+        if (ids_base < 0 || kt * 8 >= ids_base + 32) {
+            ids_base = kt * 8;
+            // Entries past the context are never read (-2: zero fill). The context comes from the
+            // device lengths, so an entry past the table's width (device lengths larger than the
+            // planned ones) is not read either: -3 is recorded as a range error below.
+            const int b = ids_base + lane;
+            ids = b >= tile.nblk_ctx ? -2
+                  : b < a.max_blocks_per_seq ? __ldg(a.block_tables + (size_t)tile.req * a.max_blocks_per_seq + b) : -3;
+        }
+        int y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int id = __shfl_sync(FULL_MASK, ids, kt * 8 - ids_base + i);
+            if (id == -2) y[i] = tile.rows_total;                       // past the context: zero fill
+            else if (id < 0 || id >= a.num_blocks) {
+                if (lane == 0) record_error(a.err, 6 /*PKV_ERR_DEVICE_RANGE*/, (long long)tile.req * a.max_blocks_per_seq + kt * 8 + i);
+                y[i] = tile.rows_total;
+            } else y[i] = (id * a.num_kv_heads + tile.kvh) * kBlockSize;
+        }
+        // K of tile kt may land once both QK^T of tile kt-2 are done; V once both PV of tile kt-2.
+        if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_KE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 100));
+        if (!ok) break;
+        if (lane == 0) {
+            unsigned char* ks = smem + OFF_K + s * kTile;
+            mbar_arrive_expect_tx(&bars[B_KF0 + s], kTile);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                tma_load_2d(ks + i * 2048, tm_k, 0, y[i], &bars[B_KF0 + s]);
+                tma_load_2d(ks + kHalf + i * 2048, tm_k, 64, y[i], &bars[B_KF0 + s]);
+            }
+        }
+        issued_k[s] = kt;
+        if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_VE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 101));
+        if (!ok) break;
+        if (lane == 0) {
+            unsigned char* vs = smem + OFF_V + s * kTile;
+            mbar_arrive_expect_tx(&bars[B_VF0 + s], kTile);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                tma_load_2d(vs + i * 2048, tm_v, 0, y[i], &bars[B_VF0 + s]);
+                tma_load_2d(vs + kHalf + i * 2048, tm_v, 64, y[i], &bars[B_VF0 + s]);
+            }
+        }
+        issued_v[s] = kt;
+        __syncwarp();
+    }
+    if (!ok && lane == 0) {
+        // Drain: wait (bounded) for the last loads issued into each stage.
+        for (int s = 0; s < 2; ++s) {
+            if (issued_k[s] >= 0) (void)mbar_wait(&bars[B_KF0 + s], (issued_k[s] >> 1) & 1);
+            if (issued_v[s] >= 0) (void)mbar_wait(&bars[B_VF0 + s], (issued_v[s] >> 1) & 1);
+        }
+        (void)mbar_wait(&bars[B_Q], 0);
+    }
+}
+
+// ---- MMA issuer (warp 9, one thread) ----
+template <typename T>
+__device__ __forceinline__ void tile_mma(const PrefillArgs& a, unsigned char* smem, uint64_t* bars,
+                                         volatile int* abort_flag, uint32_t tmem, const TileCtx& tile, int lane) {
+    if (lane == 0) {
+        const uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
+        const uint32_t id_qk = idesc_f16(fmt, 0);
+        const uint32_t id_pv = idesc_f16(fmt, 1);
+        auto issue_qk = [&](int x, int kt) {
+            const unsigned char* ks = smem + OFF_K + (kt & 1) * kTile;
+            const unsigned char* qs = smem + OFF_Q + x * kTile;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int half = k >> 2, off = (k & 3) * 32;
+                tc_mma(tmem + x * 128, smem_desc(qs + half * kHalf + off, 16, 1024),
+                       smem_desc(ks + half * kHalf + off, 16, 1024), id_qk, k > 0);
+            }
+            tc_commit(&bars[B_SF0 + x]);
+        };
+        auto issue_pv = [&](int x, int kt) {
+            const unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
+            // P_X(kt) sits as packed 16-bit pairs in the first 64 columns of S_X; each K step of
+            // 16 keys is 8 columns.
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc_mma_ts(tmem + 256 + x * 128, tmem + x * 128 + k * 8, smem_desc(vs + k * 2048, kHalf, 1024),
+                          id_pv, kt > 0 || k > 0);
+            tc_commit(&bars[B_OF0 + x]);
+        };
+        bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, a.err, 200);
+        if (ok) ok = wait_or_abort(&bars[B_KF0], 0, abort_flag, a.err, 201);
+        if (ok) {
+            tc_fence_after();
+            issue_qk(0, 0);
+            if (tile.has_b) issue_qk(1, 0);
+            tc_commit(&bars[B_KE0]);
+        }
+        for (int kt = 0; kt < tile.nkt && ok; ++kt) {
+            const int s = kt & 1;
+            const bool next = kt + 1 < tile.nkt;
+            bool k_ready = false, v_ready = false;
+            for (int x = 0; x < 2 && ok; ++x) {
+                if (kt < tile.nkt_x[x]) {
+                    ok = wait_or_abort(&bars[B_PF0 + x], kt & 1, abort_flag, a.err, 202 + x);
+                    if (ok && !v_ready) ok = v_ready = wait_or_abort(&bars[B_VF0 + s], (kt >> 1) & 1, abort_flag, a.err, 204);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(x, kt);
+                }
+                if (kt + 1 < tile.nkt_x[x]) {
+                    if (!k_ready) ok = k_ready = wait_or_abort(&bars[B_KF0 + (s ^ 1)], ((kt + 1) >> 1) & 1, abort_flag, a.err, 206);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk(x, kt + 1);
+                }
+            }
+            if (!ok) break;
+            tc_commit(&bars[B_VE0 + s]);
+            if (next) tc_commit(&bars[B_KE0 + (s ^ 1)]);
+        }
+        if (ok) {
+            // Every commit of this tile has arrived before the barriers are armed for the next one:
+            // the last phase of each K and V stage and of each tile's O.
+            for (int st = 0; st < 2 && ok; ++st) {
+                const int last = st < tile.nkt ? tile.nkt - 1 - ((tile.nkt - 1 - st) & 1) : -1;  // last key tile of stage st
+                if (last >= 0) {
+                    ok = wait_or_abort(&bars[B_KE0 + st], (last >> 1) & 1, abort_flag, a.err, 207);
+                    if (ok) ok = wait_or_abort(&bars[B_VE0 + st], (last >> 1) & 1, abort_flag, a.err, 208);
+                }
+                if (ok && tile.nkt_x[st] > 0)
+                    ok = wait_or_abort(&bars[B_OF0 + st], (tile.nkt_x[st] - 1) & 1, abort_flag, a.err, 209);
+            }
+        } else {
+            tc_commit(&bars[B_DRAIN]);
+            (void)mbar_wait(&bars[B_DRAIN], 0);
+        }
+    }
+}
+
+// ---- softmax (warps 0-7: one thread per row of tile A or B) ----
 template <typename T, int POLY>
+__device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char* smem, uint64_t* bars,
+                                             volatile int* abort_flag, uint32_t tmem, const TileCtx& tile, int warp,
+                                             int lane) {
+    const int x = warp >> 2;                 // tile
+    const int row = (warp & 3) * 32 + lane;
+    const int t_local = row / tile.G, g = row % tile.G;
+    const int j = tile.tok0 + x * tile.tt + t_local;
+    const bool row_valid = j < tile.n;
+    const int limit = row_valid ? tile.prior + j + 1 : tile.prior + 1;  // keys visible: [0, limit)
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t ts = tl + x * 128, to = tl + 256 + x * 128;
+    // Keys below this bound are visible to every row of the tile: no masking needed there.
+    const int all_visible = tile.prior + tile.tok0 + x * tile.tt + 1;
+    const int my_nkt = tile.nkt_x[x];
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int kt = 0; kt < my_nkt && ok; ++kt) {
+        ok = warp_all(wait_or_abort(&bars[B_SF0 + x], kt & 1, abort_flag, a.err, 300));
+        if (!ok) break;
+        tc_fence_after();
+        const bool full = kt * 128 + 128 <= all_visible;   // no masking anywhere in this key tile
+        float alpha = 1.f;
+        float2 ps2 = make_float2(0.f, 0.f);
+        if (full && a.scale_log2 >= 0.f) {
+            // Two TMEM round trips, one per half of the key tile: the half's maximum is taken in
+            // registers and P computed from the same registers against the row's reference m,
+            // raised first when the half exceeds it by more than the threshold. P of keys
+            // 64*h.. goes to columns 32*h.. (over S already read). If the second half raises m,
+            // the first half's P, already stored, is scaled down by the same factor.
+            const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                float sv[64];
+                tmem_ld32(ts + h * 64, sv);
+                tmem_ld32(ts + h * 64 + 32, sv + 32);
+                tmem_wait_ld();
+                float hm = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) hm = fmaxf(hm, sv[i]);
+                hm *= a.scale_log2;
+                const bool raise = hm > m + kRescaleThreshold;
+                const float f = raise ? fast_exp2(m - hm) : 1.f;  // 0 while m is -inf
+                // The TMEM accesses are warp-collective: the whole warp takes this branch when
+                // any of its rows raised, each lane scaling its own row by its own factor.
+                if (h == 1 && __any_sync(FULL_MASK, raise)) {
+                    tmem_wait_st();
+                    float pv[32];
+                    tmem_ld32(ts, pv);
+                    tmem_wait_ld();
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float2 q = unpack2<T>(__float_as_uint(pv[i]));
+                        pk[i] = pack2<T>(q.x * f, q.y * f);
+                    }
+                    tmem_st32(ts, pk);
+                }
+                if (raise) {
+                    ps2 = make_float2(ps2.x * f, ps2.y * f);
+                    alpha *= f;
+                    m = hm;
+                }
+                const float2 nm2 = make_float2(-m, -m);
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
+                    const float2 p = (i & 15) < POLY ? exp2_poly2(e) : make_float2(fast_exp2(e.x), fast_exp2(e.y));
+                    pk[i] = pack2<T>(p.x, p.y);
+                    ps2 = __fadd2_rn(ps2, row_sum_term<T>(p, pk[i]));
+                }
+                tmem_st32(ts + h * 32, pk);
+            }
+        } else {
+            // pass 1: row maximum of scale * s over the visible keys
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float sv[32];
+                tmem_ld32(ts + c * 32, sv);
+                tmem_wait_ld();
+                const int key0 = kt * 128 + c * 32;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    mx = fmaxf(mx, (full || key0 + i < limit) ? sv[i] * a.scale_log2 : -INFINITY);
+            }
+            if (mx > m + kRescaleThreshold) {
+                alpha = fast_exp2(m - mx);  // 0 on the first tile
+                m = mx;
+            }
+            // pass 2: p = 2^(s*scale - m), rounded to T, written over S as the A operand of PV.
+            // Chunk c's P goes to columns 16c.., which pass 2 has already read.
+            const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float sv[32];
+                tmem_ld32(ts + c * 32, sv);
+                tmem_wait_ld();
+                uint32_t pk[16];
+                const int key0 = kt * 128 + c * 32;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
+                    const float p0 = (full || key0 + 2 * i < limit) ? fast_exp2(e.x) : 0.f;
+                    const float p1 = (full || key0 + 2 * i + 1 < limit) ? fast_exp2(e.y) : 0.f;
+                    pk[i] = pack2<T>(p0, p1);
+                    ps2 = __fadd2_rn(ps2, row_sum_term<T>(make_float2(p0, p1), pk[i]));
+                }
+                tmem_st16(ts + c * 16, pk);
+            }
+        }
+        const float ps = ps2.x + ps2.y;
+        l = l * alpha + ps;
+        // Rescale O in TMEM when a row of this warp raised its reference (rare after the first
+        // tiles). PV(kt-1) must be complete before O is read.
+        if (kt >= 1 && __any_sync(FULL_MASK, alpha != 1.f)) {
+            ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (kt - 1) & 1, abort_flag, a.err, 301));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float o[32];
+                tmem_ld32(to + c * 32, o);
+                tmem_wait_ld();
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
+                tmem_st32(to + c * 32, w);
+            }
+        }
+        tmem_wait_st();
+        // V rows past the context (only possible in the CTA's final key tile) are zeroed by the
+        // tile whose PV of that key tile is issued first: A when it reaches it, else B.
+        if (kt == tile.nkt - 1 && (kt + 1) * 128 > tile.ctx && x == (tile.nkt_x[0] == tile.nkt ? 0 : 1)) {
+            ok = warp_all(wait_or_abort(&bars[B_VF0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 302));
+            if (!ok) break;
+            unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
+            const int r0 = tile.ctx - kt * 128;  // first V row past the context
+            const int chunks = (128 - r0) * 16;  // 16-byte chunks over both halves
+            for (int c = (warp & 3) * 32 + lane; c < chunks; c += 128) {
+                const int r = r0 + (c >> 4), h = (c >> 3) & 1, k = c & 7;
+                *reinterpret_cast<uint4*>(vs + h * kHalf + r * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[B_PF0 + x]);
+    }
+    if (ok) ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (my_nkt - 1) & 1, abort_flag, a.err, 303));
+    if (ok) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        unsigned char* dst = static_cast<unsigned char*>(a.out) +
+                             ((size_t)(tile.q0 + (row_valid ? j : 0)) * a.num_q_heads + (size_t)tile.kvh * tile.G + g) * 256;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(to + c * 32, o);
+            tmem_wait_ld();
+            if (row_valid) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = o[q * 8 + e] * inv;
+                    *reinterpret_cast<uint4*>(dst + c * 64 + q * 16) = Chunk<T>::pack(v);
+                }
+            }
+        }
+    }
+}
+
+// Control word written by thread 0 before each step of the CTA: a tile index, or one of these.
+constexpr int kJobExit = -1;    // the CTA is done
+constexpr int kJobDecode = -2;  // a round of split-K items (warps 0-7)
+constexpr int kJobNone = -3;    // nothing in this step
+
+// Persistent CTAs (one per SM) over the batch's tcgen05 tiles and, in a mixed batch, its split-K
+// work items: tiles come from a ticket counter (a.work[2], longest first), items from the split-K
+// counter (d.work[0]). A CTA b < a.decode_ctas first serves items until none is left; every CTA
+// then serves tiles until none is left, then items again if any remain. So the HBM-bound items and
+// the tensor-bound tiles run side by side, and whichever queue empties first hands its CTAs to the
+// other. In a round of items, warps 0-7 each run the warp-MMA loop over two stages carved from the
+// tile buffers (the third warpgroup waits). The last CTA to finish (a.work[3] counts them) resets
+// the counters for the next launch.
+template <typename T, int POLY, bool MIXED>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
+    prefill_tc_kernel(const PrefillArgs a, const DecodeArgs d, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+    volatile int* ctrl = reinterpret_cast<volatile int*>(smem + OFF_CTRL);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     griddep_wait();
 
-    const PrefillTile tile = a.tiles[blockIdx.x];
-    const int req = tile.req, kvh = tile.kv_head, tok0 = tile.tok0;
-    const int q0 = a.query_start_loc[req];
-    const int n = a.query_start_loc[req + 1] - q0;
-    const int ctx = a.context_lens[req];
-    const int prior = ctx - n;
-    const int G = a.group;
-    const int tt = 128 / G;                      // query rows of one MMA tile
-    const bool has_b = tok0 + tt < n;
-    // key tiles each MMA tile needs: keys visible to its last valid row
-    const int nkt_x[2] = {(min(ctx, prior + min(n, tok0 + tt)) + 127) / 128,
-                          has_b ? (min(ctx, prior + min(n, tok0 + 2 * tt)) + 127) / 128 : 0};
-    const int nkt = max(nkt_x[0], nkt_x[1]);
-    const int nblk_ctx = (ctx + kBlockSize - 1) / kBlockSize;
-    const int rows_total = a.num_blocks * a.num_kv_heads * kBlockSize;
-
-    if (threadIdx.x == 0) {
-        mbar_init(&bars[B_Q], 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars[B_KF0 + s], 1);
-            mbar_init(&bars[B_VF0 + s], 1);
-            mbar_init(&bars[B_KE0 + s], 1);
-            mbar_init(&bars[B_VE0 + s], 1);
-            mbar_init(&bars[B_SF0 + s], 1);
-            mbar_init(&bars[B_PF0 + s], 128);
-            mbar_init(&bars[B_OF0 + s], 1);
-        }
-        mbar_init(&bars[B_DRAIN], 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
+    if (threadIdx.x == 0) *abort_flag = 0;
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem + OFF_TMEM)),
                      "r"(kTmemCols)
@@ -224,321 +618,100 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
-    const bool sane = nkt >= 1 && n > 1 && tok0 < n;
-
-    if (warp == 8 && sane) {
-        // ------------------------------ TMA producer ------------------------------
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&bars[B_Q], has_b ? 2 * kTile : kTile);
-            for (int x = 0; x < (has_b ? 2 : 1); ++x) {
-                tma_load_3d(smem + OFF_Q + x * kTile, &tm_q, 0, kvh * G, q0 + tok0 + x * tt, &bars[B_Q]);
-                tma_load_3d(smem + OFF_Q + x * kTile + kHalf, &tm_q, 64, kvh * G, q0 + tok0 + x * tt, &bars[B_Q]);
-            }
-        }
-        int ids = -1, ids_base = -1;
-        int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
-        bool ok = true;
-        for (int kt = 0; kt < nkt && ok; ++kt) {
-            const int s = kt & 1;
-            if (ids_base < 0 || kt * 8 >= ids_base + 32) {
-                ids_base = kt * 8;
-                // Entries past the context are never read (-2: zero fill). The context comes from the
-                // device lengths, so an entry past the table's width (device lengths larger than the
-                // planned ones) is not read either: -3 is recorded as a range error below.
-                const int b = ids_base + lane;
-                ids = b >= nblk_ctx ? -2
-                      : b < a.max_blocks_per_seq ? __ldg(a.block_tables + (size_t)req * a.max_blocks_per_seq + b) : -3;
-            }
-            int y[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int id = __shfl_sync(FULL_MASK, ids, kt * 8 - ids_base + i);
-                if (id == -2) y[i] = rows_total;                       // past the context: zero fill
-                else if (id < 0 || id >= a.num_blocks) {
-                    if (lane == 0) record_error(a.err, 6 /*PKV_ERR_DEVICE_RANGE*/, (long long)req * a.max_blocks_per_seq + kt * 8 + i);
-                    y[i] = rows_total;
-                } else y[i] = (id * a.num_kv_heads + kvh) * kBlockSize;
-            }
-            // K of tile kt may land once both QK^T of tile kt-2 are done; V once both PV of tile kt-2.
-            if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_KE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 100));
-            if (!ok) break;
-            if (lane == 0) {
-                unsigned char* ks = smem + OFF_K + s * kTile;
-                mbar_arrive_expect_tx(&bars[B_KF0 + s], kTile);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    tma_load_2d(ks + i * 2048, &tm_k, 0, y[i], &bars[B_KF0 + s]);
-                    tma_load_2d(ks + kHalf + i * 2048, &tm_k, 64, y[i], &bars[B_KF0 + s]);
+    // Register split: the third warpgroup (producer, MMA issuer, two idle warps) shrinks to
+    // kOtherRegs, the softmax warpgroups grow to kSoftmaxRegs. Each warpgroup runs in its own branch;
+    // every step is bracketed by two CTA barriers: (1) thread 0 has written the step into *ctrl,
+    // (2) the step is done.
+    if (warp >= 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+        while (true) {
+            cta_sync();                                   // (1)
+            const int job = *ctrl;
+            if (job == kJobExit) break;
+            if (job >= 0) {
+                const TileCtx tile = tile_ctx(a, job);
+                if (tile.sane) {
+                    if (warp == 8) tile_producer(a, &tm_q, &tm_k, &tm_v, smem, bars, abort_flag, tile, lane);
+                    else if (warp == 9) tile_mma<T>(a, smem, bars, abort_flag, tmem, tile, lane);
                 }
-            }
-            issued_k[s] = kt;
-            if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_VE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 101));
-            if (!ok) break;
-            if (lane == 0) {
-                unsigned char* vs = smem + OFF_V + s * kTile;
-                mbar_arrive_expect_tx(&bars[B_VF0 + s], kTile);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    tma_load_2d(vs + i * 2048, &tm_v, 0, y[i], &bars[B_VF0 + s]);
-                    tma_load_2d(vs + kHalf + i * 2048, &tm_v, 64, y[i], &bars[B_VF0 + s]);
-                }
-            }
-            issued_v[s] = kt;
-            __syncwarp();
-        }
-        if (!ok && lane == 0) {
-            // Drain: wait (bounded) for the last loads issued into each stage.
-            for (int s = 0; s < 2; ++s) {
-                if (issued_k[s] >= 0) (void)mbar_wait(&bars[B_KF0 + s], (issued_k[s] >> 1) & 1);
-                if (issued_v[s] >= 0) (void)mbar_wait(&bars[B_VF0 + s], (issued_v[s] >> 1) & 1);
-            }
-            (void)mbar_wait(&bars[B_Q], 0);
-        }
-    } else if (warp == 9 && sane) {
-        // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
-            const uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
-            const uint32_t id_qk = idesc_f16(fmt, 0);
-            const uint32_t id_pv = idesc_f16(fmt, 1);
-            auto issue_qk = [&](int x, int kt) {
-                const unsigned char* ks = smem + OFF_K + (kt & 1) * kTile;
-                const unsigned char* qs = smem + OFF_Q + x * kTile;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int half = k >> 2, off = (k & 3) * 32;
-                    tc_mma(tmem + x * 128, smem_desc(qs + half * kHalf + off, 16, 1024),
-                           smem_desc(ks + half * kHalf + off, 16, 1024), id_qk, k > 0);
-                }
-                tc_commit(&bars[B_SF0 + x]);
-            };
-            auto issue_pv = [&](int x, int kt) {
-                const unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
-                // P_X(kt) sits as packed 16-bit pairs in the first 64 columns of S_X; each K step of
-                // 16 keys is 8 columns.
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    tc_mma_ts(tmem + 256 + x * 128, tmem + x * 128 + k * 8, smem_desc(vs + k * 2048, kHalf, 1024),
-                              id_pv, kt > 0 || k > 0);
-                tc_commit(&bars[B_OF0 + x]);
-            };
-            bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, a.err, 200);
-            if (ok) ok = wait_or_abort(&bars[B_KF0], 0, abort_flag, a.err, 201);
-            if (ok) {
-                tc_fence_after();
-                issue_qk(0, 0);
-                if (has_b) issue_qk(1, 0);
-                tc_commit(&bars[B_KE0]);
-            }
-            for (int kt = 0; kt < nkt && ok; ++kt) {
-                const int s = kt & 1;
-                const bool next = kt + 1 < nkt;
-                bool k_ready = false, v_ready = false;
-                for (int x = 0; x < 2 && ok; ++x) {
-                    if (kt < nkt_x[x]) {
-                        ok = wait_or_abort(&bars[B_PF0 + x], kt & 1, abort_flag, a.err, 202 + x);
-                        if (ok && !v_ready) ok = v_ready = wait_or_abort(&bars[B_VF0 + s], (kt >> 1) & 1, abort_flag, a.err, 204);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(x, kt);
-                    }
-                    if (kt + 1 < nkt_x[x]) {
-                        if (!k_ready) ok = k_ready = wait_or_abort(&bars[B_KF0 + (s ^ 1)], ((kt + 1) >> 1) & 1, abort_flag, a.err, 206);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_qk(x, kt + 1);
-                    }
-                }
-                if (!ok) break;
-                tc_commit(&bars[B_VE0 + s]);
-                if (next) tc_commit(&bars[B_KE0 + (s ^ 1)]);
-            }
-            if (ok) {
-                (void)wait_or_abort(&bars[B_VE0 + ((nkt - 1) & 1)], ((nkt - 1) >> 1) & 1, abort_flag, a.err, 207);
-            } else {
-                tc_commit(&bars[B_DRAIN]);
-                (void)mbar_wait(&bars[B_DRAIN], 0);
-            }
-        }
-    } else if (warp < 8 && sane && (warp < 4 || has_b)) {
-        // ------------------------------ softmax (one thread per row) ------------------------------
-        const int x = warp >> 2;                 // tile
-        const int row = (warp & 3) * 32 + lane;
-        const int t_local = row / G, g = row % G;
-        const int j = tok0 + x * tt + t_local;
-        const bool row_valid = j < n;
-        const int limit = row_valid ? prior + j + 1 : prior + 1;  // keys visible: [0, limit)
-        const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const uint32_t ts = tl + x * 128, to = tl + 256 + x * 128;
-        // Keys below this bound are visible to every row of the tile: no masking needed there.
-        const int all_visible = prior + tok0 + x * tt + 1;
-        const int my_nkt = nkt_x[x];
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int kt = 0; kt < my_nkt && ok; ++kt) {
-            ok = warp_all(wait_or_abort(&bars[B_SF0 + x], kt & 1, abort_flag, a.err, 300));
-            if (!ok) break;
-            tc_fence_after();
-            const bool full = kt * 128 + 128 <= all_visible;   // no masking anywhere in this key tile
-            float alpha = 1.f;
-            float2 ps2 = make_float2(0.f, 0.f);
-            if (full && a.scale_log2 >= 0.f) {
-                // Two TMEM round trips, one per half of the key tile: the half's maximum is taken in
-                // registers and P computed from the same registers against the row's reference m,
-                // raised first when the half exceeds it by more than the threshold. P of keys
-                // 64*h.. goes to columns 32*h.. (over S already read). If the second half raises m,
-                // the first half's P, already stored, is scaled down by the same factor.
-                const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-#pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    float sv[64];
-                    tmem_ld32(ts + h * 64, sv);
-                    tmem_ld32(ts + h * 64 + 32, sv + 32);
-                    tmem_wait_ld();
-                    float hm = -INFINITY;
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) hm = fmaxf(hm, sv[i]);
-                    hm *= a.scale_log2;
-                    const bool raise = hm > m + kRescaleThreshold;
-                    const float f = raise ? fast_exp2(m - hm) : 1.f;  // 0 while m is -inf
-                    // The TMEM accesses are warp-collective: the whole warp takes this branch when
-                    // any of its rows raised, each lane scaling its own row by its own factor.
-                    if (h == 1 && __any_sync(FULL_MASK, raise)) {
-                        tmem_wait_st();
-                        float pv[32];
-                        tmem_ld32(ts, pv);
-                        tmem_wait_ld();
-                        uint32_t pk[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float2 q = unpack2<T>(__float_as_uint(pv[i]));
-                            pk[i] = pack2<T>(q.x * f, q.y * f);
-                        }
-                        tmem_st32(ts, pk);
-                    }
-                    if (raise) {
-                        ps2 = make_float2(ps2.x * f, ps2.y * f);
-                        alpha *= f;
-                        m = hm;
-                    }
-                    const float2 nm2 = make_float2(-m, -m);
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
-                        const float2 p = (i & 15) < POLY ? exp2_poly2(e) : make_float2(fast_exp2(e.x), fast_exp2(e.y));
-                        pk[i] = pack2<T>(p.x, p.y);
-                        ps2 = __fadd2_rn(ps2, row_sum_term<T>(p, pk[i]));
-                    }
-                    tmem_st32(ts + h * 32, pk);
-                }
-            } else {
-                // pass 1: row maximum of scale * s over the visible keys
-                float mx = -INFINITY;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float sv[32];
-                    tmem_ld32(ts + c * 32, sv);
-                    tmem_wait_ld();
-                    const int key0 = kt * 128 + c * 32;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        mx = fmaxf(mx, (full || key0 + i < limit) ? sv[i] * a.scale_log2 : -INFINITY);
-                }
-                if (mx > m + kRescaleThreshold) {
-                    alpha = fast_exp2(m - mx);  // 0 on the first tile
-                    m = mx;
-                }
-                // pass 2: p = 2^(s*scale - m), rounded to T, written over S as the A operand of PV.
-                // Chunk c's P goes to columns 16c.., which pass 2 has already read.
-                const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float sv[32];
-                    tmem_ld32(ts + c * 32, sv);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-                    const int key0 = kt * 128 + c * 32;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
-                        const float p0 = (full || key0 + 2 * i < limit) ? fast_exp2(e.x) : 0.f;
-                        const float p1 = (full || key0 + 2 * i + 1 < limit) ? fast_exp2(e.y) : 0.f;
-                        pk[i] = pack2<T>(p0, p1);
-                        ps2 = __fadd2_rn(ps2, row_sum_term<T>(make_float2(p0, p1), pk[i]));
-                    }
-                    tmem_st16(ts + c * 16, pk);
-                }
-            }
-            const float ps = ps2.x + ps2.y;
-            l = l * alpha + ps;
-            // Rescale O in TMEM when a row of this warp raised its reference (rare after the first
-            // tiles). PV(kt-1) must be complete before O is read.
-            if (kt >= 1 && __any_sync(FULL_MASK, alpha != 1.f)) {
-                ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (kt - 1) & 1, abort_flag, a.err, 301));
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float o[32];
-                    tmem_ld32(to + c * 32, o);
-                    tmem_wait_ld();
-                    uint32_t w[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
-                    tmem_st32(to + c * 32, w);
-                }
-            }
-            tmem_wait_st();
-            // V rows past the context (only possible in the CTA's final key tile) are zeroed by the
-            // tile whose PV of that key tile is issued first: A when it reaches it, else B.
-            if (kt == nkt - 1 && (kt + 1) * 128 > ctx && x == (nkt_x[0] == nkt ? 0 : 1)) {
-                ok = warp_all(wait_or_abort(&bars[B_VF0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 302));
-                if (!ok) break;
-                unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
-                const int r0 = ctx - kt * 128;  // first V row past the context
-                const int chunks = (128 - r0) * 16;  // 16-byte chunks over both halves
-                for (int c = (warp & 3) * 32 + lane; c < chunks; c += 128) {
-                    const int r = r0 + (c >> 4), h = (c >> 3) & 1, k = c & 7;
-                    *reinterpret_cast<uint4*>(vs + h * kHalf + r * 128 + k * 16) = make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
             }
             tc_fence_before();
-            mbar_arrive(&bars[B_PF0 + x]);
+            cta_sync();                                   // (2)
         }
-        if (ok) ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (my_nkt - 1) & 1, abort_flag, a.err, 303));
-        if (ok) {
-            tc_fence_after();
-            const float inv = 1.f / l;
-            unsigned char* dst = static_cast<unsigned char*>(a.out) +
-                                 ((size_t)(q0 + (row_valid ? j : 0)) * a.num_q_heads + (size_t)kvh * G + g) * 256;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float o[32];
-                tmem_ld32(to + c * 32, o);
-                tmem_wait_ld();
-                if (row_valid) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float v[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[e] = o[q * 8 + e] * inv;
-                        *reinterpret_cast<uint4*>(dst + c * 64 + q * 16) = Chunk<T>::pack(v);
-                    }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+        // A round of split-K items: this warp takes tickets until none is left.
+        [[maybe_unused]] auto decode_round = [&]() {
+            int first = 0;
+            if (lane == 0) first = atomicAdd(&d.work[0], 1);
+            first = __shfl_sync(FULL_MASK, first, 0);
+            uint64_t* dbars = reinterpret_cast<uint64_t*>(smem + OFF_DBAR) + warp * kDecodeStages;
+            volatile int* fifo = reinterpret_cast<volatile int*>(smem + OFF_FIFO) + warp * mma::kFifo;
+            if (!mma::decode_warp<T, kDecodeStages>(d, &tm_k, &tm_v, smem + warp * kDecodeStages * mma::kStage, dbars,
+                                                    fifo, first, 0) && lane == 0)
+                *abort_flag = 1;
+            fence_proxy_async_smem();   // its generic writes (zeroed V rows) before later TMA writes
+        };
+        [[maybe_unused]] auto items_left = [&]() {
+            return d.num_items > 0 && *reinterpret_cast<volatile int*>(&d.work[0]) < d.num_items && !*abort_flag;
+        };
+        // (a) CTAs that start on items: a round of them first.
+        if constexpr (MIXED) {
+            if (threadIdx.x == 0) *ctrl = ((int)blockIdx.x < a.decode_ctas && items_left()) ? kJobDecode : kJobNone;
+            cta_sync();                                   // (1)
+            if (*ctrl == kJobDecode) decode_round();
+            tc_fence_before();
+            cta_sync();                                   // (2)
+        }
+        // (b) tiles, longest first, while any is left.
+        while (true) {
+            if (threadIdx.x == 0) {
+                int t = kJobNone;
+                if (!*abort_flag && *reinterpret_cast<volatile int*>(&a.work[2]) < a.num_tiles) {
+                    t = atomicAdd(&a.work[2], 1);
+                    if (t < a.num_tiles) init_tile_barriers(bars);
+                    else t = kJobNone;
                 }
+                *ctrl = t;
+            }
+            cta_sync();                                   // (1)
+            const int job = *ctrl;
+            if (job >= 0) {
+                tc_fence_after();
+                const TileCtx tile = tile_ctx(a, job);
+                if (tile.sane && (warp < 4 || tile.has_b)) tile_softmax<T, POLY>(a, smem, bars, abort_flag, tmem, tile, warp, lane);
+            }
+            tc_fence_before();
+            cta_sync();                                   // (2)
+            if (job < 0) break;
+        }
+        // (c) the items still left once the tiles are gone.
+        if constexpr (MIXED) {
+            if (threadIdx.x == 0) *ctrl = items_left() ? kJobDecode : kJobNone;
+            cta_sync();                                   // (1)
+            if (*ctrl == kJobDecode) decode_round();
+            tc_fence_before();
+            cta_sync();                                   // (2)
+        }
+        if (threadIdx.x == 0) *ctrl = kJobExit;
+        cta_sync();                                       // (1)
+        if (warp == 0) {
+            tc_fence_after();
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        }
+        if (threadIdx.x == 0) {
+            __threadfence();
+            if (atomicAdd(&a.work[3], 1) == (int)gridDim.x - 1) {
+                atomicExch(&a.work[2], 0);
+                atomicExch(&a.work[3], 0);
+                if (d.num_items > 0) atomicExch(&d.work[0], 0);
             }
         }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
-template <typename T, int POLY>
-cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
+template <typename T, int POLY, bool MIXED>
+cudaError_t launch_t(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cudaStream_t s) {
     const CUtensorMapDataType dt =
         std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int G = a.group;
@@ -550,6 +723,8 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     const cuuint64_t kdims[2] = {128, (cuuint64_t)rows};
     const cuuint64_t kstr[1] = {128 * 2};
     const cuuint32_t kbox[2] = {64, (cuuint32_t)kBlockSize};
+    // One map over the pool rows serves the tiles (8 blocks per key tile) and the split-K items
+    // (one block per stage): the same 64-column x 16-row box with the 128-byte swizzle.
     if (!encode_tiled(&mq, dt, 3, a.q, qdims, qstr, qbox) || !encode_tiled(&mk, dt, 2, a.k_pool, kdims, kstr, kbox) ||
         !encode_tiled(&mv, dt, 2, a.v_pool, kdims, kstr, kbox))
         return cudaErrorInvalidValue;
@@ -558,11 +733,16 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(prefill_tc_kernel<T, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        e = cudaFuncSetAttribute(prefill_tc_kernel<T, POLY, MIXED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = 1;
     }
-    return launch_pdl(prefill_tc_kernel<T, POLY>, dim3(a.num_tiles), dim3(kThreads), SMEM_BYTES, s, a, mq, mk, mv);
+    // One persistent CTA per SM (fewer when the batch has fewer tiles and no split-K items).
+    int grid = num_sms;
+    if (d.num_items <= 0 && a.num_tiles < grid) grid = a.num_tiles;
+    return launch_k(a.pdl, prefill_tc_kernel<T, POLY, MIXED>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, a, d, mq, mk,
+                    mv);
 }
 
 int poly_pairs() {
@@ -573,13 +753,20 @@ int poly_pairs() {
     return v;
 }
 
-template <typename T>
-cudaError_t launch_p(const PrefillArgs& a, cudaStream_t s) {
+template <typename T, bool MIXED>
+cudaError_t launch_p(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cudaStream_t s) {
     switch (poly_pairs()) {
-        case 2: return launch_t<T, 2>(a, s);
-        case 4: return launch_t<T, 4>(a, s);
-        default: return launch_t<T, kPolyPairs>(a, s);
+        case 2: return launch_t<T, 2, MIXED>(a, d, num_sms, s);
+        case 4: return launch_t<T, 4, MIXED>(a, d, num_sms, s);
+        default: return launch_t<T, kPolyPairs, MIXED>(a, d, num_sms, s);
     }
+}
+
+// Batches with tcgen05 tiles only run an instantiation without the split-K rounds (fewer registers
+// live in the softmax warps).
+template <typename T>
+cudaError_t launch_m(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cudaStream_t s) {
+    return d.num_items > 0 ? launch_p<T, true>(a, d, num_sms, s) : launch_p<T, false>(a, d, num_sms, s);
 }
 
 }  // namespace
@@ -588,11 +775,12 @@ bool prefill_tc_supported(int dtype, int head_dim, int group) {
     return (dtype == 1 || dtype == 2) && head_dim == 128 && group >= 1 && group <= 16 && (128 % group) == 0;
 }
 
-cudaError_t launch_prefill_tc(int dtype, const PrefillArgs& a, int /*num_sms*/, cudaStream_t s) {
-    if (a.num_tiles <= 0) return cudaSuccess;
+cudaError_t launch_prefill_tc(int dtype, const PrefillArgs& a, const DecodeArgs& d, int num_sms, cudaStream_t s) {
+    if (a.num_tiles <= 0 && d.num_items <= 0) return cudaSuccess;
+    if (!a.work || (d.num_items > 0 && !d.work)) return cudaErrorInvalidValue;
     if ((long long)a.num_blocks * a.num_kv_heads * kBlockSize >= (1LL << 31) - 1) return cudaErrorInvalidValue;
     if (((uintptr_t)a.q | (uintptr_t)a.k_pool | (uintptr_t)a.v_pool) & 15) return cudaErrorInvalidValue;
-    return dtype == 1 ? launch_p<__half>(a, s) : launch_p<__nv_bfloat16>(a, s);
+    return dtype == 1 ? launch_m<__half>(a, d, num_sms, s) : launch_m<__nv_bfloat16>(a, d, num_sms, s);
 }
 
 }  // namespace pkv

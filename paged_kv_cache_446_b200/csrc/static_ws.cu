@@ -30,29 +30,6 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_ws[PKV_STATIC_WS_BYTES];
 
-// Unique id of the calling thread's current CUDA context (0 if it cannot be read).
-unsigned long long current_context_id() {
-    typedef CUresult (*GetCurrent)(CUcontext*);
-    typedef CUresult (*GetId)(CUcontext, unsigned long long*);
-    static std::once_flag once;
-    static GetCurrent get_current = nullptr;
-    static GetId get_id = nullptr;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_current = reinterpret_cast<GetCurrent>(p);
-        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_id = reinterpret_cast<GetId>(p);
-    });
-    CUcontext c = nullptr;
-    unsigned long long id = 0;
-    if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
-    return id;
-}
-
 // Device address of g_static_ws for the current device and context (host code may not use the
 // symbol itself: in host code its name is a host-side stand-in, not a device address).
 void* static_ws_address(pkv_status* st) {

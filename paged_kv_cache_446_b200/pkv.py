@@ -40,7 +40,7 @@ class PlanOptions(ctypes.Structure):
                 ("cuda_core_only", ctypes.c_int32), ("num_sms", ctypes.c_int32), ("heads_per_item", ctypes.c_int32),
                 ("rows_per_item", ctypes.c_int32), ("tc_min_rows", ctypes.c_int32), ("decode_kernel", ctypes.c_int32),
                 ("h_block_tables", ctypes.c_void_p), ("block_table_stride", ctypes.c_int32),
-                ("min_shared_blocks", ctypes.c_int32)]
+                ("min_shared_blocks", ctypes.c_int32), ("decode_sms", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):
@@ -49,7 +49,8 @@ class Plan(ctypes.Structure):
         "num_prefill_rows", "num_items", "num_tiles", "num_merge_rows", "num_partials", "split_blocks",
         "max_blocks", "heads_per_item", "rows_per_item", "decode_kernel", "part_stride", "merge_slots")] + [(n, ctypes.c_int64) for n in (
         "off_items", "off_tiles", "off_merge", "off_part_o", "off_part_ml", "meta_bytes", "ws_bytes", "kv_bytes",
-        "attn_flops", "core_kv_bytes", "tile_kv_bytes", "tile_flops")]
+        "attn_flops", "core_kv_bytes", "tile_kv_bytes", "tile_flops")] + [
+        ("decode_sms", ctypes.c_int32), ("pad0", ctypes.c_int32)]
 
 
 def _sig(name, restype, argtypes):
@@ -122,9 +123,10 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _opts(split_blocks=0, no_split=False, cuda_core_only=False, num_sms=0, heads_per_item=0, rows_per_item=0,
-          tc_min_rows=0, decode_kernel=0, shared_tables=None, min_shared_blocks=0) -> PlanOptions:
+          tc_min_rows=0, decode_kernel=0, shared_tables=None, min_shared_blocks=0, decode_sms=0) -> PlanOptions:
     """Planner options. shared_tables: host int32 block tables [R, max_blocks] for shared-prefix
-    detection (the caller keeps the array alive while planning), or None."""
+    detection (the caller keeps the array alive while planning), or None. decode_sms: SMs of the
+    split-K kernel when it runs concurrently with the tcgen05 tiles (0 planner's choice, -1 serial)."""
     o = PlanOptions(int(split_blocks), int(bool(no_split)), int(bool(cuda_core_only)), int(num_sms),
                     int(heads_per_item), int(rows_per_item), int(tc_min_rows), int(decode_kernel))
     if shared_tables is not None:
@@ -132,6 +134,7 @@ def _opts(split_blocks=0, no_split=False, cuda_core_only=False, num_sms=0, heads
         o.h_block_tables = shared_tables.ctypes.data
         o.block_table_stride = int(shared_tables.shape[1])
     o.min_shared_blocks = int(min_shared_blocks)
+    o.decode_sms = int(decode_sms)
     return o
 
 

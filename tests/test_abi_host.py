@@ -338,16 +338,17 @@ def test_plan_image_independent_of_buffer_contents(pkv, config):
 
 @pytest.mark.parametrize("config,num_sms", [("c2", 148), ("c3", 148), ("c4", 148), ("c6", 148), ("c3", 2),
                                             ("c5", 3), ("c6", 1)])
-def test_items_dealt_longest_first_in_a_snake(pkv, config, num_sms):
-    """The persistent decode warps run positions w, w + W, w + 2W, ... (W = 8 per SM): the planner
-    sorts the items longest first and deals every second round of W in reverse, so reading the
-    positions back in dealing order gives block counts that never increase, and the warps' totals
-    come out within a few percent of each other."""
+def test_fma_items_dealt_longest_first_in_a_snake(pkv, config, num_sms):
+    """The FMA kernel's persistent warps run positions w, w + W, w + 2W, ... (W = 8 per SM): the
+    planner sorts the items longest first and deals every second round of W in reverse, so reading
+    the positions back in dealing order gives block counts that never increase, and the warps'
+    totals come out within a few percent of each other (or within one item of the mean)."""
     from paged_kv_cache_446_b200 import workloads as W
     wl = W.make(config, with_tensors=False)
     qsl, ctx = pkv.flatten_batch(wl.batch, wl.prior_lens)
     plan, meta = pkv.plan_host(qsl, ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, num_sms=num_sms,
-                               shared_tables=wl.block_tables)
+                               shared_tables=wl.block_tables, decode_kernel=1, tc_min_rows=1 << 20)
+    assert plan.decode_kernel == 1
     items, _, _ = parse_meta(plan, meta)
     lens = items[:, 5] - items[:, 4]
     n, deal = len(lens), num_sms * 8
@@ -359,4 +360,31 @@ def test_items_dealt_longest_first_in_a_snake(pkv, config, num_sms):
     assert all(a >= b for a, b in zip(dealt, dealt[1:]))
     per_warp = np.zeros(deal)
     np.add.at(per_warp, np.arange(n) % deal, lens + 1)
-    assert per_warp.max() <= 1.1 * per_warp.mean() or n <= 3 * deal
+    assert per_warp.max() <= max(1.1 * per_warp.mean(), per_warp.mean() + lens.max() + 1) or n <= 3 * deal
+
+
+@pytest.mark.parametrize("config,num_sms", [("c2", 148), ("c3", 148), ("c4", 148), ("c5", 148), ("c6", 148),
+                                            ("c3", 2), ("c6", 1)])
+def test_mma_items_longest_first_for_greedy_warps(pkv, config, num_sms):
+    """The warp-MMA kernel's warps take items greedily (warp w starts with item w, then each takes
+    the next unclaimed item from a ticket counter): the planner lists the items longest first, and a
+    greedy simulation of W = 8 warps per SM over that list ends within a few percent of the mean
+    load (or within one item of it)."""
+    import heapq
+    from paged_kv_cache_446_b200 import workloads as W
+    wl = W.make(config, with_tensors=False)
+    qsl, ctx = pkv.flatten_batch(wl.batch, wl.prior_lens)
+    plan, meta = pkv.plan_host(qsl, ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, num_sms=num_sms,
+                               shared_tables=wl.block_tables)
+    assert plan.decode_kernel == 2
+    items, _, _ = parse_meta(plan, meta)
+    lens = (items[:, 5] - items[:, 4]).astype(np.int64)
+    assert all(a >= b for a, b in zip(lens, lens[1:]))
+    W_ = num_sms * 8
+    heap = [(0, w) for w in range(W_)]
+    for ln in lens:
+        t, w = heapq.heappop(heap)
+        heapq.heappush(heap, (t + int(ln) + 1, w))
+    finish = max(t for t, _ in heap)
+    mean = (lens + 1).sum() / W_
+    assert finish <= max(1.1 * mean, mean + lens.max() + 1)

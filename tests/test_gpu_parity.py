@@ -414,3 +414,40 @@ def test_pool_too_large_for_tensor_maps_is_refused(dev):
                             pkv._ptr(p.workspace), p.workspace.numel(), pkv._stream(None))
     torch.cuda.synchronize()
     assert status == 3
+
+
+@pytest.mark.parametrize("decode_sms", [1, 16, 74, 147])
+def test_overlapped_mixed_batch(dev, decode_sms):
+    """A mixed batch served by one persistent launch: decode_sms CTAs of the tcgen05 kernel start on
+    the split-K items, the rest on the tiles, each turning to the other queue when its own empties.
+    Within tolerance of the oracle, and bit for bit the output of the two kernels run one after the
+    other (every output element is computed by the same item or tile either way)."""
+    wl = W.make("c5", device=dev, small=True)
+    _, step = run_and_compare(wl, dev, decode_sms=decode_sms)
+    p = step.plan.plan
+    assert p.num_tiles > 0 and p.num_items > 0 and p.decode_sms == decode_sms
+    a = step.run(wl.q, wl.k_pool, wl.v_pool, wl.scale, wl.k_new, wl.v_new).clone()
+    b = make_step(wl, dev, decode_sms=-1).run(wl.q, wl.k_pool, wl.v_pool, wl.scale, wl.k_new, wl.v_new)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("config", ["c2", "c4", "c5"])
+def test_plan_reused_across_launches(dev, config):
+    """One plan run many times in a row (as every layer of a model step does): the split-K kernel's
+    item ticket counter resets itself at the end of each launch, so every launch serves every item
+    and the outputs agree bit for bit."""
+    from paged_kv_cache_446_b200 import pkv
+    wl = W.make(config, device=dev, small=True)
+    bt = torch.from_numpy(wl.block_tables).to(dev)
+    plan = pkv.AttentionPlan(wl.batch, wl.prior_lens, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                             W.TORCH_DTYPES[wl.dtype], dev, decode_sms=8)
+    outs = []
+    for _ in range(4):
+        out = torch.full_like(wl.q, float("nan"))
+        pkv.paged_attention(plan, wl.q, wl.k_pool, wl.v_pool, bt, wl.scale, out=out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert torch.isfinite(outs[0].float()).all()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
