@@ -85,6 +85,39 @@ PlanLists& thread_lists() {
 // Query rows per tcgen05 CTA: two 128-row MMA tiles, each (128 / G) consecutive query rows x G heads.
 int tile_tokens(int group) { return 2 * (128 / group); }
 
+// CTAs of the tile kernel that should start on the split-K items of a mixed batch (0: run the two
+// kernels one after the other). Model, with rates measured on B200 for these kernels: a tile CTA
+// spends ~2.4 us per 128-key tile; an SM serving items streams their K/V at ~72 GB/s while the
+// others run tiles; once the tiles are done every SM serves items, ~6.6 TB/s together. For a few
+// candidate splits, the tiles (already longest first) are dealt to the other CTAs; the step ends
+// when the tiles end plus the time the items left over take on the whole GPU. The split with the
+// shortest estimate wins.
+int mixed_split(const std::vector<PrefillTile>& tiles, int64_t item_bytes, int num_sms) {
+    constexpr double kKeyTileSec = 2.4e-6, kSmBytesPerSec = 72e9, kGpuBytesPerSec = 6.6e12;
+    static thread_local std::vector<double> load;
+    auto tiles_end = [&](int ctas) {  // longest first, dealt in a snake (a close stand-in for greedy)
+        load.assign((size_t)ctas, 0.0);
+        for (size_t i = 0; i < tiles.size(); ++i) {
+            const size_t r = i / ctas, k = i % ctas;
+            load[(r & 1) ? ctas - 1 - k : k] += tiles[i].key_tiles * kKeyTileSec;
+        }
+        return *std::max_element(load.begin(), load.end());
+    };
+    const double all_items = (double)item_bytes / kGpuBytesPerSec;
+    double best = tiles_end(num_sms) + all_items;  // one kernel after the other
+    int best_nd = 0;
+    for (int nd = 8; nd <= num_sms / 2; nd += 8) {
+        const double t = tiles_end(num_sms - nd);
+        const double left = std::max(0.0, (double)item_bytes - nd * kSmBytesPerSec * t);
+        const double est = t + left / kGpuBytesPerSec;
+        if (est < best) {
+            best = est;
+            best_nd = nd;
+        }
+    }
+    return best_nd;
+}
+
 // out_meta / out_cap: when given and large enough, the work lists are written straight into that
 // image (the layout write_meta produces), skipping the intermediate lists.
 pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int Hkv, int D, pkv_dtype dt,
@@ -415,24 +448,11 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->tile_flops = tile_flops;
     // Mixed batch: the tcgen05 kernel's persistent CTAs (one per SM) also serve the warp-MMA items;
     // decode_sms of them start on items, the rest on tiles, and each turns to the other queue when
-    // its own empties. Automatic share: the items' part of the two parts' estimated SM time (a key
-    // tile of a CTA ~2.5 us at the tiles' measured tensor rate; an SM streaming items ~100 GB/s when
-    // the HBM is not saturated), but never so many that a tile longer than half the estimated step
-    // has to wait for a CTA: every such tile gets one from the start.
+    // its own empties.
     plan->decode_sms = 0;
     if (o.decode_sms >= 0 && kind == 2 && n_items > 0 && !L->tiles.empty() && num_sms >= 2) {
         int nd = o.decode_sms;
-        if (nd == 0) {
-            constexpr double kKeyTileSec = 2.5e-6, kItemBytesPerSec = 100e9;
-            double t_p = 0.0;
-            for (const PrefillTile& t : L->tiles) t_p += t.key_tiles * kKeyTileSec;
-            const double t_d = (double)plan->core_kv_bytes / kItemBytesPerSec;
-            const double t_step = (t_p + t_d) / num_sms;
-            int n_long = 0;
-            for (const PrefillTile& t : L->tiles) n_long += t.key_tiles * kKeyTileSec > 0.5 * t_step;
-            if (t_d > 20e-6 * num_sms && t_p > 20e-6 * num_sms)  // each part worth overlapping
-                nd = std::min((int)std::lround(num_sms * t_d / (t_p + t_d)), num_sms - n_long);
-        }
+        if (nd == 0) nd = mixed_split(L->tiles, plan->core_kv_bytes, num_sms);
         if (nd > 0) plan->decode_sms = std::min(nd, num_sms - 1);
     }
     return PKV_OK;

@@ -221,17 +221,25 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
             lim1 = v1 ? ci.limit + (g + 8) / nh : 0;
         }
 
-        // ---- S = Q K^T: two 8-token n-tiles ----
-        float s[2][4];
+        // ---- S = Q K^T: two 8-token n-tiles, each accumulated in two chains (even / odd k-steps)
+        // so that the dependent MMAs per chain are four, not eight ----
+        float s[2][4], s2[2][4];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+        for (int j = 0; j < 2; ++j) {
+            s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+            s2[j][0] = s2[j][1] = s2[j][2] = s2[j][3] = 0.f;
+        }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             uint32_t b0, b1, b2, b3;
             ldsm_x4(kb + sw_off(((mi >> 1) << 3) + mr, 2 * kk + (mi & 1)), b0, b1, b2, b3);
-            mma16816<T>(s[0], qa[kk], b0, b1);
-            mma16816<T>(s[1], qa[kk], b2, b3);
+            mma16816<T>((kk & 1) ? s2[0] : s[0], qa[kk], b0, b1);
+            mma16816<T>((kk & 1) ? s2[1] : s[1], qa[kk], b2, b3);
         }
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[j][e] += s2[j][e];
 
         // ---- online softmax per slot (log2 domain), masked by each slot's own limit ----
         const int t0 = c_blk * kBlockSize + 2 * c4;
@@ -269,15 +277,11 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
         // add the weights as rounded, so that they match what P V accumulates.
         const uint32_t pa[4] = {pack2<T>(p[0][0], p[0][1]), pack2<T>(p[0][2], p[0][3]), pack2<T>(p[1][0], p[1][1]),
                                 pack2<T>(p[1][2], p[1][3])};
+        // Each lane keeps the sum of its own weights; the quad's four partial sums are added once,
+        // when the item ends (the rescale factors are the same on all four lanes of a slot).
         const float2 r00 = unpack2<T>(pa[0]), r01 = unpack2<T>(pa[1]), r10 = unpack2<T>(pa[2]), r11 = unpack2<T>(pa[3]);
-        float rs0 = (r00.x + r00.y) + (r10.x + r10.y);
-        float rs1 = (r01.x + r01.y) + (r11.x + r11.y);
-        rs0 += __shfl_xor_sync(FULL_MASK, rs0, 1);
-        rs1 += __shfl_xor_sync(FULL_MASK, rs1, 1);
-        rs0 += __shfl_xor_sync(FULL_MASK, rs0, 2);
-        rs1 += __shfl_xor_sync(FULL_MASK, rs1, 2);
-        l0 = l0 * al0 + rs0;
-        l1 = l1 * al1 + rs1;
+        l0 = l0 * al0 + ((r00.x + r00.y) + (r10.x + r10.y));
+        l1 = l1 * al1 + ((r01.x + r01.y) + (r11.x + r11.y));
         if (al0 != 1.f || al1 != 1.f) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -318,6 +322,10 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
 
         if (c_blk + 1 == ci.blk_end) {
             // ---- item done: normalised output, or the chunk's partial ----
+            l0 += __shfl_xor_sync(FULL_MASK, l0, 1);
+            l1 += __shfl_xor_sync(FULL_MASK, l1, 1);
+            l0 += __shfl_xor_sync(FULL_MASK, l0, 2);
+            l1 += __shfl_xor_sync(FULL_MASK, l1, 2);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int slot = g + 8 * h;
