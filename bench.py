@@ -246,9 +246,14 @@ def cpu_model() -> str:
 
 
 def run_oracle_sample(wl, h, target_seconds: float, threads: int = 0, append: bool = True):
-    """The oracle, as it stands, on the first m requests (all heads, all rows) of the step, with the
-    step's own KV append applied first (unless append=False: already applied to h). Returns
-    dict(value_gbs, seconds, requests, cores, bytes). threads = 0: every host core."""
+    """The oracle, as it stands, on a bounded sample of the step's query rows (all heads of each row):
+    every k-th row of the flattened batch, so decode and prefill rows appear in their proportions,
+    with the step's own KV append applied first (unless append=False: already applied to h). A
+    sampled row counts its request's K/V bytes divided by the request's row count, so the whole
+    batch counts each (request, KV head, context token) once, as the GPU metric does. The stride
+    shrinks until the oracle has run for about target_seconds (the whole batch is repeated when it
+    is faster than that). Returns dict(value_gbs, seconds, rows, of, cores, bytes, repeats).
+    threads = 0: every host core."""
     import oracle
     cores = threads or os.cpu_count() or 1
     qsl, ctx = oracle.flatten_batch(wl.batch, wl.prior_lens)
@@ -261,32 +266,33 @@ def run_oracle_sample(wl, h, target_seconds: float, threads: int = 0, append: bo
         slots = oracle.slot_mapping(wl.block_tables, wqsl, wctx)
         oracle.kv_cache_write(h["k_new"], h["v_new"], h["k_pool"], h["v_pool"], slots)
     eb = 4 if wl.dtype == "f32" else 2
-    per_req = ctx.astype(np.int64) * wl.num_kv_heads * 2 * wl.head_dim * eb
-    order = [r for r in range(len(ctx)) if counts[r] > 0]
+    T = int(qsl[-1])
+    req_of_row = np.repeat(np.arange(len(ctx)), counts)
+    row_bytes = (ctx.astype(np.float64) * wl.num_kv_heads * 2 * wl.head_dim * eb / np.maximum(counts, 1))[req_of_row]
 
-    def run(m):
-        rows = np.concatenate([np.arange(qsl[r], qsl[r + 1]) for r in order[:m]]).astype(np.int32)
+    def run(stride):
+        rows = np.arange(stride // 2, T, stride, dtype=np.int32)
         t0 = time.perf_counter()
         oracle.paged_attention(h["q"], h["k_pool"], h["v_pool"], wl.block_tables, ctx, qsl, wl.scale, wl.dtype,
                                rows=rows, nthreads=cores)
-        return time.perf_counter() - t0, int(per_req[order[:m]].sum())
+        return time.perf_counter() - t0, float(row_bytes[rows].sum()), len(rows)
 
-    m = 1
-    dt, by = run(m)
-    while dt < target_seconds * 0.3 and m < len(order):
-        m = min(len(order), max(m + 1, int(m * min(8.0, target_seconds / max(dt, 1e-3)))))
-        dt, by = run(m)
+    stride = max(1, T // 8)
+    dt, by, n = run(stride)
+    while dt < target_seconds * 0.3 and stride > 1:
+        stride = max(1, int(stride / min(8.0, max(1.5, 0.6 * target_seconds / max(dt, 1e-3)))))
+        dt, by, n = run(stride)
     reps = 1
-    if m == len(order) and dt < target_seconds * 0.5:
+    if stride == 1 and dt < target_seconds * 0.5:
         # the whole batch is quick: repeat it to fill the measurement window
         reps = max(1, int(target_seconds / max(dt, 1e-3)))
-        dt, by = 0.0, 0
+        dt, by = 0.0, 0.0
         for _ in range(reps):
-            t, b = run(m)
+            t, b, n = run(1)
             dt += t
             by += b
-    return {"value_gbs": by / dt / 1e9, "seconds": dt, "requests": m, "of": len(order), "cores": cores, "bytes": by,
-            "repeats": reps}
+    return {"value_gbs": by / dt / 1e9, "seconds": dt, "rows": n, "of": T, "stride": stride, "cores": cores,
+            "bytes": int(by), "repeats": reps}
 
 
 def storage(t):
@@ -316,11 +322,11 @@ def reference_arm(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(samples),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1) q/k/v; seeded block placement)",
-            "config": {"workload": wl.name, "requests_per_step_sample": samples[-1]["requests"],
-                       "requests": samples[-1]["of"]},
+            "config": {"workload": wl.name, "rows_per_step_sample": samples[-1]["rows"],
+                       "rows": samples[-1]["of"]},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": samples[-1]["cores"], "kind": "oracle",
-                             "sample": f"first {samples[-1]['requests']} of {samples[-1]['of']} requests of "
-                                       f"{wl.name} per step (all heads and rows, after the step's KV append)"},
+                             "sample": f"every {samples[-1]['stride']}th of the {samples[-1]['of']} query rows of "
+                                       f"{wl.name} per step (all heads, after the step's KV append)"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -370,14 +376,14 @@ def main():
         h = {k: storage(getattr(wl, k)) for k in ("q", "k_pool", "v_pool", "k_new", "v_new")}
         r = run_oracle_sample(wl, h, args.cpu_seconds)
         cpu_baseline = {"value": r["value_gbs"], "unit": "GB/s", "cores": r["cores"], "kind": "oracle",
-                        "sample": f"first {r['requests']} of {r['of']} requests of {wl.name} (all heads and rows, "
-                                  f"after the step's KV append) x{r['repeats']}, {r['seconds']:.1f} s",
+                        "sample": f"every {r['stride']}th of the {r['of']} query rows of {wl.name} ({r['rows']} rows, all "
+                                  f"heads, after the step's KV append) x{r['repeats']}, {r['seconds']:.1f} s",
                         "cpu_model": cpu_model()}
         if args.config in ("c1", "c2"):
             r1 = run_oracle_sample(wl, h, args.cpu_seconds / 3, threads=1, append=False)
             cpu_baseline["single_thread"] = {
                 "value": r1["value_gbs"], "unit": "GB/s", "cores": 1,
-                "sample": f"first {r1['requests']} of {r1['of']} requests x{r1['repeats']}, {r1['seconds']:.1f} s"}
+                "sample": f"every {r1['stride']}th of {r1['of']} rows x{r1['repeats']}, {r1['seconds']:.1f} s"}
         del h
 
     def run_step():

@@ -47,7 +47,7 @@ constexpr int smem_bytes() { return 1024 + kMmaWarps * NSTAGE * (kStage + 8) + k
 
 // Warp gw of the W launched starts with item gw; further items come from tickets (item W + ticket).
 // The last warp to finish (a.work[1] counts them) resets both counters for the next launch.
-template <typename T, int NSTAGE>
+template <typename T, int NSTAGE, bool T8>
 __global__ void __launch_bounds__(kMmaWarps * 32)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v) {
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32)
     volatile int* fifo = reinterpret_cast<int*>(smem + kMmaWarps * NSTAGE * (kStage + 8)) + warp * kFifo;
     griddep_wait();
     const int W = gridDim.x * kMmaWarps;
-    (void)decode_warp<T, NSTAGE>(a, &tm_k, &tm_v, wbase, bars, fifo, blockIdx.x * kMmaWarps + warp, W);
+    (void)decode_warp<T, NSTAGE, T8>(a, &tm_k, &tm_v, wbase, bars, fifo, blockIdx.x * kMmaWarps + warp, W);
     // Every warp passes here exactly once on its way out.
     if (lane == 0 && atomicAdd(&a.work[1], 1) == W - 1) {
         atomicExch(&a.work[0], 0);
@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32)
     }
 }
 
-template <typename T, int NSTAGE>
+template <typename T, int NSTAGE, bool T8>
 cudaError_t launch_mma_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     const CUtensorMapDataType dt =
         std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -86,9 +86,9 @@ cudaError_t launch_mma_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     int per_sm = (dev >= 0 && dev < 64) ? per_sm_cache[dev] : 0;
     if (per_sm == 0) {
-        e = cudaFuncSetAttribute(decode_mma_kernel<T, NSTAGE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(decode_mma_kernel<T, NSTAGE, T8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_mma_kernel<T, NSTAGE>, kMmaWarps * 32, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_mma_kernel<T, NSTAGE, T8>, kMmaWarps * 32, smem);
         if (e != cudaSuccess) return e;
         if (per_sm < 1) per_sm = 1;
         if (dev >= 0 && dev < 64) per_sm_cache[dev] = per_sm;
@@ -97,7 +97,7 @@ cudaError_t launch_mma_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     int grid = num_sms * per_sm;
     if (grid > need) grid = need;
     if (grid < 1) return cudaSuccess;
-    return launch_k(a.pdl, decode_mma_kernel<T, NSTAGE>, dim3(grid), dim3(kMmaWarps * 32), smem, s, a, mk, mv);
+    return launch_k(a.pdl, decode_mma_kernel<T, NSTAGE, T8>, dim3(grid), dim3(kMmaWarps * 32), smem, s, a, mk, mv);
 }
 
 // Ring depth: 2 stages (24 KiB per warp, so 4 CTAs = 8 warps fit an SM; measured best on every
@@ -111,13 +111,19 @@ inline int mma_stages() {
     return v;
 }
 
-template <typename T>
+template <typename T, bool T8>
 cudaError_t launch_mma_s(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     switch (mma_stages()) {
-        case 3: return launch_mma_t<T, 3>(a, num_sms, s);
-        case 4: return launch_mma_t<T, 4>(a, num_sms, s);
-        default: return launch_mma_t<T, 2>(a, num_sms, s);
+        case 3: return launch_mma_t<T, 3, T8>(a, num_sms, s);
+        case 4: return launch_mma_t<T, 4, T8>(a, num_sms, s);
+        default: return launch_mma_t<T, 2, T8>(a, num_sms, s);
     }
+}
+
+// Items of at most 8 (row, head) slots run the transposed form (half the MMAs per block).
+template <typename T>
+cudaError_t launch_mma_k(const DecodeArgs& a, int num_sms, cudaStream_t s) {
+    return a.slots_per_item <= 8 ? launch_mma_s<T, true>(a, num_sms, s) : launch_mma_s<T, false>(a, num_sms, s);
 }
 
 }  // namespace
@@ -129,7 +135,7 @@ cudaError_t launch_decode_mma(int dtype, const DecodeArgs& a, int num_sms, cudaS
     if (!a.work) return cudaErrorInvalidValue;
     if ((long long)a.num_blocks * a.num_kv_heads * kBlockSize >= (1LL << 31) - 1) return cudaErrorInvalidValue;
     if (((uintptr_t)a.q | (uintptr_t)a.k_pool | (uintptr_t)a.v_pool) & 15) return cudaErrorInvalidValue;
-    return dtype == 1 ? launch_mma_s<__half>(a, num_sms, s) : launch_mma_s<__nv_bfloat16>(a, num_sms, s);
+    return dtype == 1 ? launch_mma_k<__half>(a, num_sms, s) : launch_mma_k<__nv_bfloat16>(a, num_sms, s);
 }
 
 }  // namespace pkv

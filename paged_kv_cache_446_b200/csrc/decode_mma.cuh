@@ -82,6 +82,14 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
     }
 }
 
+// Transpose of an 8 x 8 matrix of 16-bit elements held as one fragment (lane l: row l / 4, columns
+// 2 (l % 4) and 2 (l % 4) + 1): afterwards lane l holds row l / 4 of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 // One warp's run over split-K work items. `first` is the warp's first item (none when it is
 // >= num_items); every further item is base + a ticket taken from a.work[0], so warps that finish
 // early take more items and the planner's longest-first order is served greedily. The producer
@@ -90,7 +98,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 // here (they must be idle); fifo: kFifo ints of shared memory (the items the producer has started,
 // in order, for the consumer). On return every copy the warp issued has landed. Returns false when
 // a bounded wait expired (recorded in the device error word; the warp's copies then drained).
-template <typename T, int NSTAGE>
+template <typename T, int NSTAGE, bool T8>
 __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                             unsigned char* wbase, uint64_t* bars, volatile int* fifo, int first,
                                             int base) {
@@ -179,189 +187,358 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
     int c_blk = ci.blk_begin;
     uint32_t consumed = 0;
 
-    const int g = lane >> 2;       // fragment row: slots g and g + 8
+    const int g = lane >> 2;       // fragment row
     const int c4 = lane & 3;       // fragment column pair
     const int mi = lane >> 3;      // ldmatrix: which 8x8 matrix this lane addresses
     const int mr = lane & 7;       //           and which of its rows
 
-    uint32_t qa[8][4];             // Q as A fragments, one set per 16-column k-step
-    float o[16][4];                // O accumulators, one per 8-column n-tile
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    int lim0 = 0, lim1 = 0, nh = 1, ns = 0;
+    if constexpr (T8) {
+        // Items of at most 8 (row, head) slots, transposed: S^T = K Q^T (16 tokens x 8 slots, K as the
+        // A operand, q rows as the B operand) and O^T = V^T P^T (128 x 8, V as the A operand through
+        // transposing ldmatrix, P^T as the B operand moved into place by movmatrix): 16 MMAs per block
+        // instead of 32. Lane (g, c4) holds tokens g and g + 8 of slots 2c4 and 2c4 + 1; a slot's
+        // reductions over tokens run across the 8 lanes that share its c4.
+        uint32_t qb[8][2];         // Q^T as B fragments, one pair per 16-column k-step
+        float ot[8][4];            // O^T accumulators, one per 16-row (head_dim) m-tile
+        float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+        int lima = 0, limb = 0, nh = 1, ns = 0;
+        const int sa = 2 * c4, sb = 2 * c4 + 1;   // this lane's slots
 
-    while (true) {
-        const int stage = consumed % NSTAGE;
-        const uint32_t parity = (consumed / NSTAGE) & 1u;
-        if (!mbar_wait(&bars[stage], parity)) {
-            if (lane == 0) record_error(a.err, 5 /*PKV_ERR_DEVICE_TIMEOUT*/, c_it);
-            for (uint32_t k = consumed; k < issued; ++k) (void)mbar_wait(&bars[k % NSTAGE], (k / NSTAGE) & 1u);
-            return false;
-        }
-        unsigned char* st = wbase + stage * kStage;
-        const uint32_t kb = smem_u32(st);
-        const uint32_t vb = kb + 2 * kHalf;
+        while (true) {
+            const int stage = consumed % NSTAGE;
+            const uint32_t parity = (consumed / NSTAGE) & 1u;
+            if (!mbar_wait(&bars[stage], parity)) {
+                if (lane == 0) record_error(a.err, 5 /*PKV_ERR_DEVICE_TIMEOUT*/, c_it);
+                for (uint32_t k = consumed; k < issued; ++k) (void)mbar_wait(&bars[k % NSTAGE], (k / NSTAGE) & 1u);
+                return false;
+            }
+            unsigned char* st = wbase + stage * kStage;
+            const uint32_t kb = smem_u32(st);
+            const uint32_t vb = kb + 2 * kHalf;
 
-        if (c_blk == ci.blk_begin) {
-            nh = min(a.heads_per_item, a.group - ci.head0);
-            ns = nh * ci.num_rows;
-            const uint32_t* qs = reinterpret_cast<const uint32_t*>(st + kKV);
-            const bool v0 = g < ns, v1 = g + 8 < ns;
+            if (c_blk == ci.blk_begin) {
+                nh = min(a.heads_per_item, a.group - ci.head0);
+                ns = nh * ci.num_rows;
+                const uint32_t* qs = reinterpret_cast<const uint32_t*>(st + kKV);
+                const bool vq = g < ns;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    qb[kk][0] = vq ? qs[g * 64 + kk * 8 + c4] : 0u;
+                    qb[kk][1] = vq ? qs[g * 64 + kk * 8 + 4 + c4] : 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ot[j][0] = ot[j][1] = ot[j][2] = ot[j][3] = 0.f;
+                ma = mb = -INFINITY;
+                la = lb = 0.f;
+                lima = sa < ns ? ci.limit + sa / nh : 0;   // keys visible to slot sa (row sa / nh of the item)
+                limb = sb < ns ? ci.limit + sb / nh : 0;
+            }
+
+            // ---- S^T = K Q^T, accumulated in two chains (even / odd k-steps) ----
+            float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                qa[kk][0] = v0 ? qs[g * 64 + kk * 8 + c4] : 0u;
-                qa[kk][1] = v1 ? qs[(g + 8) * 64 + kk * 8 + c4] : 0u;
-                qa[kk][2] = v0 ? qs[g * 64 + kk * 8 + 4 + c4] : 0u;
-                qa[kk][3] = v1 ? qs[(g + 8) * 64 + kk * 8 + 4 + c4] : 0u;
+                uint32_t ka[4];
+                ldsm_x4(kb + sw_off(((mi & 1) << 3) + mr, 2 * kk + (mi >> 1)), ka[0], ka[1], ka[2], ka[3]);
+                mma16816<T>((kk & 1) ? s2 : s, ka, qb[kk][0], qb[kk][1]);
             }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-            m0 = m1 = -INFINITY;
-            l0 = l1 = 0.f;
-            lim0 = v0 ? ci.limit + g / nh : 0;         // keys visible to slot g (row g / nh of the item)
-            lim1 = v1 ? ci.limit + (g + 8) / nh : 0;
-        }
+            for (int e = 0; e < 4; ++e) s[e] += s2[e];
 
-        // ---- S = Q K^T: two 8-token n-tiles, each accumulated in two chains (even / odd k-steps)
-        // so that the dependent MMAs per chain are four, not eight ----
-        float s[2][4], s2[2][4];
+            // ---- online softmax per slot (log2 domain), masked by each slot's own limit ----
+            const int t0 = c_blk * kBlockSize + g;
+            s[0] = t0 < lima ? s[0] * a.scale_log2 : -INFINITY;
+            s[1] = t0 < limb ? s[1] * a.scale_log2 : -INFINITY;
+            s[2] = t0 + 8 < lima ? s[2] * a.scale_log2 : -INFINITY;
+            s[3] = t0 + 8 < limb ? s[3] * a.scale_log2 : -INFINITY;
+            float mxa = fmaxf(s[0], s[2]), mxb = fmaxf(s[1], s[3]);
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-            s2[j][0] = s2[j][1] = s2[j][2] = s2[j][3] = 0.f;
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(kb + sw_off(((mi >> 1) << 3) + mr, 2 * kk + (mi & 1)), b0, b1, b2, b3);
-            mma16816<T>((kk & 1) ? s2[0] : s[0], qa[kk], b0, b1);
-            mma16816<T>((kk & 1) ? s2[1] : s[1], qa[kk], b2, b3);
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[j][e] += s2[j][e];
-
-        // ---- online softmax per slot (log2 domain), masked by each slot's own limit ----
-        const int t0 = c_blk * kBlockSize + 2 * c4;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int t = t0 + 8 * j;
-            s[j][0] = t < lim0 ? s[j][0] * a.scale_log2 : -INFINITY;
-            s[j][1] = t + 1 < lim0 ? s[j][1] * a.scale_log2 : -INFINITY;
-            s[j][2] = t < lim1 ? s[j][2] * a.scale_log2 : -INFINITY;
-            s[j][3] = t + 1 < lim1 ? s[j][3] * a.scale_log2 : -INFINITY;
-        }
-        float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-        float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        // A slot may see no key of this block (a chunk past an earlier row's limit, a padded slot):
-        // subtracting 0 instead of -inf keeps alpha and p at 0 rather than NaN.
-        const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
-        const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-        const float al0 = fast_exp2(m0 - mu0), al1 = fast_exp2(m1 - mu1);
-        m0 = mn0;
-        m1 = mn1;
-        float p[2][4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            p[j][0] = fast_exp2(s[j][0] - mu0);
-            p[j][1] = fast_exp2(s[j][1] - mu0);
-            p[j][2] = fast_exp2(s[j][2] - mu1);
-            p[j][3] = fast_exp2(s[j][3] - mu1);
-        }
-        // P as the A operand of P V: rows g / g + 8, token columns 2c, 2c+1 (+8). The row sums
-        // add the weights as rounded, so that they match what P V accumulates.
-        const uint32_t pa[4] = {pack2<T>(p[0][0], p[0][1]), pack2<T>(p[0][2], p[0][3]), pack2<T>(p[1][0], p[1][1]),
-                                pack2<T>(p[1][2], p[1][3])};
-        // Each lane keeps the sum of its own weights; the quad's four partial sums are added once,
-        // when the item ends (the rescale factors are the same on all four lanes of a slot).
-        const float2 r00 = unpack2<T>(pa[0]), r01 = unpack2<T>(pa[1]), r10 = unpack2<T>(pa[2]), r11 = unpack2<T>(pa[3]);
-        l0 = l0 * al0 + ((r00.x + r00.y) + (r10.x + r10.y));
-        l1 = l1 * al1 + ((r01.x + r01.y) + (r11.x + r11.y));
-        if (al0 != 1.f || al1 != 1.f) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                o[j][0] *= al0;
-                o[j][1] *= al0;
-                o[j][2] *= al1;
-                o[j][3] *= al1;
+            for (int sh = 4; sh < 32; sh <<= 1) {
+                mxa = fmaxf(mxa, __shfl_xor_sync(FULL_MASK, mxa, sh));
+                mxb = fmaxf(mxb, __shfl_xor_sync(FULL_MASK, mxb, sh));
             }
-        }
+            const float mna = fmaxf(ma, mxa), mnb = fmaxf(mb, mxb);
+            // A slot may see no key of this block: subtracting 0 instead of -inf keeps alpha and p at
+            // 0 rather than NaN.
+            const float mua = mna == -INFINITY ? 0.f : mna;
+            const float mub = mnb == -INFINITY ? 0.f : mnb;
+            const float ala = fast_exp2(ma - mua), alb = fast_exp2(mb - mub);
+            ma = mna;
+            mb = mnb;
+            // P^T rounded to T, as two 8 x 8 fragments (tokens 0-7 and 8-15; rows = tokens, columns =
+            // slots). The row sums add the weights as rounded; each lane keeps its own part, the 8
+            // lanes of a slot are added when the item ends.
+            const uint32_t w0 = pack2<T>(fast_exp2(s[0] - mua), fast_exp2(s[1] - mub));
+            const uint32_t w1 = pack2<T>(fast_exp2(s[2] - mua), fast_exp2(s[3] - mub));
+            const float2 r0 = unpack2<T>(w0), r1 = unpack2<T>(w1);
+            la = la * ala + (r0.x + r1.x);
+            lb = lb * alb + (r0.y + r1.y);
+            if (ala != 1.f || alb != 1.f) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    ot[j][0] *= ala;
+                    ot[j][1] *= alb;
+                    ot[j][2] *= ala;
+                    ot[j][3] *= alb;
+                }
+            }
 
-        // ---- V rows past the last visible key may hold anything: zero them ----
-        const int vis = ci.limit + ci.num_rows - 1 - c_blk * kBlockSize;
-        if (vis < kBlockSize) {
-            const int first = vis > 0 ? vis : 0;
-            for (int idx = lane; idx < (kBlockSize - first) * 16; idx += 32) {
-                const int r = first + (idx >> 4);
-                *reinterpret_cast<uint4*>(st + 2 * kHalf + sw_off(r, idx & 15)) = make_uint4(0u, 0u, 0u, 0u);
+            // ---- V rows past the last visible key may hold anything: zero them ----
+            const int vis = ci.limit + ci.num_rows - 1 - c_blk * kBlockSize;
+            if (vis < kBlockSize) {
+                const int first_row = vis > 0 ? vis : 0;
+                for (int idx = lane; idx < (kBlockSize - first_row) * 16; idx += 32) {
+                    const int r = first_row + (idx >> 4);
+                    *reinterpret_cast<uint4*>(st + 2 * kHalf + sw_off(r, idx & 15)) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                __syncwarp();
+            }
+
+            // ---- O^T += V^T P^T: eight 16-row m-tiles of head_dim ----
+            const uint32_t pb0 = movmatrix_trans(w0), pb1 = movmatrix_trans(w1);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                uint32_t va[4];
+                ldsm_x4_t(vb + sw_off(((mi >> 1) << 3) + mr, 2 * mt + (mi & 1)), va[0], va[1], va[2], va[3]);
+                mma16816<T>(ot[mt], va, pb0, pb1);
             }
             __syncwarp();
-        }
+            ++consumed;
 
-        // ---- O += P V: sixteen 8-column n-tiles ----
-#pragma unroll
-        for (int jp = 0; jp < 8; ++jp) {
-            uint32_t v0, v1, v2, v3;
-            ldsm_x4_t(vb + sw_off(((mi & 1) << 3) + mr, 2 * jp + (mi >> 1)), v0, v1, v2, v3);
-            mma16816<T>(o[2 * jp], pa, v0, v1);
-            mma16816<T>(o[2 * jp + 1], pa, v2, v3);
-        }
-        __syncwarp();
-        ++consumed;
+            // Refill this stage with the producer's next block.
+            if (!p_done) {
+                fence_proxy_async_smem();
+                issue(stage);
+            }
 
-        // Refill this stage with the producer's next block.
-        if (!p_done) {
-            fence_proxy_async_smem();
-            issue(stage);
-        }
-
-        if (c_blk + 1 == ci.blk_end) {
-            // ---- item done: normalised output, or the chunk's partial ----
-            l0 += __shfl_xor_sync(FULL_MASK, l0, 1);
-            l1 += __shfl_xor_sync(FULL_MASK, l1, 1);
-            l0 += __shfl_xor_sync(FULL_MASK, l0, 2);
-            l1 += __shfl_xor_sync(FULL_MASK, l1, 2);
+            if (c_blk + 1 == ci.blk_end) {
+                // ---- item done: normalised output, or the chunk's partial ----
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int slot = g + 8 * h;
-                if (slot < ns) {
-                    const int jr = slot / nh;
-                    const float m = h ? m1 : m0, l = h ? l1 : l0;
-                    if (ci.partial < 0) {
-                        const float inv = 1.f / l;
-                        T* orow = static_cast<T*>(a.out) +
-                                  ((size_t)(ci.row + jr) * a.num_q_heads + (size_t)ci.kv_head * a.group + ci.head0 +
-                                   (slot - jr * nh)) * 128;
+                for (int sh = 4; sh < 32; sh <<= 1) {
+                    la += __shfl_xor_sync(FULL_MASK, la, sh);
+                    lb += __shfl_xor_sync(FULL_MASK, lb, sh);
+                }
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            *reinterpret_cast<uint32_t*>(orow + 8 * j + 2 * c4) =
-                                pack2<T>(o[j][2 * h] * inv, o[j][2 * h + 1] * inv);
-                    } else {
-                        float* po = a.part_o + ((size_t)ci.partial * a.part_stride + slot) * 128;
+                for (int h = 0; h < 2; ++h) {
+                    const int slot = h ? sb : sa;
+                    if (slot < ns) {
+                        const int jr = slot / nh;
+                        const float m = h ? mb : ma, l = h ? lb : la;
+                        if (ci.partial < 0) {
+                            const float inv = 1.f / l;
+                            T* orow = static_cast<T*>(a.out) +
+                                      ((size_t)(ci.row + jr) * a.num_q_heads + (size_t)ci.kv_head * a.group + ci.head0 +
+                                       (slot - jr * nh)) * 128;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            *reinterpret_cast<float2*>(po + 8 * j + 2 * c4) = make_float2(o[j][2 * h], o[j][2 * h + 1]);
-                        if (c4 == 0) {
-                            float* pm = a.part_ml + ((size_t)ci.partial * a.part_stride + slot) * 2;
-                            pm[0] = m;
-                            pm[1] = l;
+                            for (int mt = 0; mt < 8; ++mt) {
+                                orow[16 * mt + g] = T(ot[mt][h] * inv);
+                                orow[16 * mt + 8 + g] = T(ot[mt][2 + h] * inv);
+                            }
+                        } else {
+                            float* po = a.part_o + ((size_t)ci.partial * a.part_stride + slot) * 128;
+#pragma unroll
+                            for (int mt = 0; mt < 8; ++mt) {
+                                po[16 * mt + g] = ot[mt][h];
+                                po[16 * mt + 8 + g] = ot[mt][2 + h];
+                            }
+                            if (g == 0) {
+                                float* pm = a.part_ml + ((size_t)ci.partial * a.part_stride + slot) * 2;
+                                pm[0] = m;
+                                pm[1] = l;
+                            }
                         }
                     }
                 }
+                // The next item is the producer's next one; none was started: the work is done.
+                if (++popped == pushed) break;
+                __syncwarp();
+                c_it = fifo[popped % kFifo];
+                ci = load_item(a.items, c_it);
+                c_blk = ci.blk_begin;
+            } else {
+                ++c_blk;
             }
-            // The next item is the producer's next one; none was started: the work is done.
-            if (++popped == pushed) break;
+        }
+    } else {
+        uint32_t qa[8][4];             // Q as A fragments, one set per 16-column k-step
+        float o[16][4];                // O accumulators, one per 8-column n-tile
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        int lim0 = 0, lim1 = 0, nh = 1, ns = 0;
+
+        while (true) {
+            const int stage = consumed % NSTAGE;
+            const uint32_t parity = (consumed / NSTAGE) & 1u;
+            if (!mbar_wait(&bars[stage], parity)) {
+                if (lane == 0) record_error(a.err, 5 /*PKV_ERR_DEVICE_TIMEOUT*/, c_it);
+                for (uint32_t k = consumed; k < issued; ++k) (void)mbar_wait(&bars[k % NSTAGE], (k / NSTAGE) & 1u);
+                return false;
+            }
+            unsigned char* st = wbase + stage * kStage;
+            const uint32_t kb = smem_u32(st);
+            const uint32_t vb = kb + 2 * kHalf;
+
+            if (c_blk == ci.blk_begin) {
+                nh = min(a.heads_per_item, a.group - ci.head0);
+                ns = nh * ci.num_rows;
+                const uint32_t* qs = reinterpret_cast<const uint32_t*>(st + kKV);
+                const bool v0 = g < ns, v1 = g + 8 < ns;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    qa[kk][0] = v0 ? qs[g * 64 + kk * 8 + c4] : 0u;
+                    qa[kk][1] = v1 ? qs[(g + 8) * 64 + kk * 8 + c4] : 0u;
+                    qa[kk][2] = v0 ? qs[g * 64 + kk * 8 + 4 + c4] : 0u;
+                    qa[kk][3] = v1 ? qs[(g + 8) * 64 + kk * 8 + 4 + c4] : 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+                m0 = m1 = -INFINITY;
+                l0 = l1 = 0.f;
+                lim0 = v0 ? ci.limit + g / nh : 0;         // keys visible to slot g (row g / nh of the item)
+                lim1 = v1 ? ci.limit + (g + 8) / nh : 0;
+            }
+
+            // ---- S = Q K^T: two 8-token n-tiles, each accumulated in two chains (even / odd k-steps)
+            // so that the dependent MMAs per chain are four, not eight ----
+            float s[2][4], s2[2][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+                s2[j][0] = s2[j][1] = s2[j][2] = s2[j][3] = 0.f;
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kb + sw_off(((mi >> 1) << 3) + mr, 2 * kk + (mi & 1)), b0, b1, b2, b3);
+                mma16816<T>((kk & 1) ? s2[0] : s[0], qa[kk], b0, b1);
+                mma16816<T>((kk & 1) ? s2[1] : s[1], qa[kk], b2, b3);
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s[j][e] += s2[j][e];
+
+            // ---- online softmax per slot (log2 domain), masked by each slot's own limit ----
+            const int t0 = c_blk * kBlockSize + 2 * c4;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int t = t0 + 8 * j;
+                s[j][0] = t < lim0 ? s[j][0] * a.scale_log2 : -INFINITY;
+                s[j][1] = t + 1 < lim0 ? s[j][1] * a.scale_log2 : -INFINITY;
+                s[j][2] = t < lim1 ? s[j][2] * a.scale_log2 : -INFINITY;
+                s[j][3] = t + 1 < lim1 ? s[j][3] * a.scale_log2 : -INFINITY;
+            }
+            float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+            float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, 2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, 2));
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            // A slot may see no key of this block (a chunk past an earlier row's limit, a padded slot):
+            // subtracting 0 instead of -inf keeps alpha and p at 0 rather than NaN.
+            const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
+            const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float al0 = fast_exp2(m0 - mu0), al1 = fast_exp2(m1 - mu1);
+            m0 = mn0;
+            m1 = mn1;
+            float p[2][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                p[j][0] = fast_exp2(s[j][0] - mu0);
+                p[j][1] = fast_exp2(s[j][1] - mu0);
+                p[j][2] = fast_exp2(s[j][2] - mu1);
+                p[j][3] = fast_exp2(s[j][3] - mu1);
+            }
+            // P as the A operand of P V: rows g / g + 8, token columns 2c, 2c+1 (+8). The row sums
+            // add the weights as rounded, so that they match what P V accumulates.
+            const uint32_t pa[4] = {pack2<T>(p[0][0], p[0][1]), pack2<T>(p[0][2], p[0][3]), pack2<T>(p[1][0], p[1][1]),
+                                    pack2<T>(p[1][2], p[1][3])};
+            // Each lane keeps the sum of its own weights; the quad's four partial sums are added once,
+            // when the item ends (the rescale factors are the same on all four lanes of a slot).
+            const float2 r00 = unpack2<T>(pa[0]), r01 = unpack2<T>(pa[1]), r10 = unpack2<T>(pa[2]), r11 = unpack2<T>(pa[3]);
+            l0 = l0 * al0 + ((r00.x + r00.y) + (r10.x + r10.y));
+            l1 = l1 * al1 + ((r01.x + r01.y) + (r11.x + r11.y));
+            if (al0 != 1.f || al1 != 1.f) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    o[j][0] *= al0;
+                    o[j][1] *= al0;
+                    o[j][2] *= al1;
+                    o[j][3] *= al1;
+                }
+            }
+
+            // ---- V rows past the last visible key may hold anything: zero them ----
+            const int vis = ci.limit + ci.num_rows - 1 - c_blk * kBlockSize;
+            if (vis < kBlockSize) {
+                const int first = vis > 0 ? vis : 0;
+                for (int idx = lane; idx < (kBlockSize - first) * 16; idx += 32) {
+                    const int r = first + (idx >> 4);
+                    *reinterpret_cast<uint4*>(st + 2 * kHalf + sw_off(r, idx & 15)) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                __syncwarp();
+            }
+
+            // ---- O += P V: sixteen 8-column n-tiles ----
+#pragma unroll
+            for (int jp = 0; jp < 8; ++jp) {
+                uint32_t v0, v1, v2, v3;
+                ldsm_x4_t(vb + sw_off(((mi & 1) << 3) + mr, 2 * jp + (mi >> 1)), v0, v1, v2, v3);
+                mma16816<T>(o[2 * jp], pa, v0, v1);
+                mma16816<T>(o[2 * jp + 1], pa, v2, v3);
+            }
             __syncwarp();
-            c_it = fifo[popped % kFifo];
-            ci = load_item(a.items, c_it);
-            c_blk = ci.blk_begin;
-        } else {
-            ++c_blk;
+            ++consumed;
+
+            // Refill this stage with the producer's next block.
+            if (!p_done) {
+                fence_proxy_async_smem();
+                issue(stage);
+            }
+
+            if (c_blk + 1 == ci.blk_end) {
+                // ---- item done: normalised output, or the chunk's partial ----
+                l0 += __shfl_xor_sync(FULL_MASK, l0, 1);
+                l1 += __shfl_xor_sync(FULL_MASK, l1, 1);
+                l0 += __shfl_xor_sync(FULL_MASK, l0, 2);
+                l1 += __shfl_xor_sync(FULL_MASK, l1, 2);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int slot = g + 8 * h;
+                    if (slot < ns) {
+                        const int jr = slot / nh;
+                        const float m = h ? m1 : m0, l = h ? l1 : l0;
+                        if (ci.partial < 0) {
+                            const float inv = 1.f / l;
+                            T* orow = static_cast<T*>(a.out) +
+                                      ((size_t)(ci.row + jr) * a.num_q_heads + (size_t)ci.kv_head * a.group + ci.head0 +
+                                       (slot - jr * nh)) * 128;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                *reinterpret_cast<uint32_t*>(orow + 8 * j + 2 * c4) =
+                                    pack2<T>(o[j][2 * h] * inv, o[j][2 * h + 1] * inv);
+                        } else {
+                            float* po = a.part_o + ((size_t)ci.partial * a.part_stride + slot) * 128;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                *reinterpret_cast<float2*>(po + 8 * j + 2 * c4) = make_float2(o[j][2 * h], o[j][2 * h + 1]);
+                            if (c4 == 0) {
+                                float* pm = a.part_ml + ((size_t)ci.partial * a.part_stride + slot) * 2;
+                                pm[0] = m;
+                                pm[1] = l;
+                            }
+                        }
+                    }
+                }
+                // The next item is the producer's next one; none was started: the work is done.
+                if (++popped == pushed) break;
+                __syncwarp();
+                c_it = fifo[popped % kFifo];
+                ci = load_item(a.items, c_it);
+                c_blk = ci.blk_begin;
+            } else {
+                ++c_blk;
+            }
         }
     }
     return true;

@@ -81,8 +81,10 @@ constexpr uint32_t kTmemCols = 512;                  // S_A [0,128), S_B [128,25
 // more than this (log2 units); the result is exact (softmax is shift invariant) and p <= 2^8.
 constexpr float kRescaleThreshold = 8.f;
 // Of each 32 exponentials of an unmasked key tile, 2 * POLY are computed by exp2_poly2 on the FMA
-// pipe (the kernel's template parameter; default kPolyPairs, PKV_PREFILL_POLY_PAIRS overrides it).
-constexpr int kPolyPairs = 0;  // measured: with three TMEM round trips per tile, MUFU alone is fastest
+// pipe (the kernel's template parameter). Measured slower at every share tried (MUFU is not what
+// bounds the softmax: ex2 runs at 16 per clock per SM and the softmax keeps it about half busy), so
+// kernels are built with none.
+constexpr int kPolyPairs = 0;
 
 // ---- tcgen05 / TMA primitives ---------------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
@@ -213,7 +215,9 @@ __device__ __forceinline__ float2 row_sum_term(float2 p, uint32_t packed) {
 // What every role needs to know about one tile (request, KV head, 2 x 128 packed rows).
 struct TileCtx {
     int req, kvh, tok0, q0, n, ctx, prior, G, tt, nkt, nblk_ctx, rows_total;
-    int nkt_x[2];   // key tiles each MMA tile needs: keys visible to its last valid row
+    int nkt_a, nkt_b;  // key tiles each MMA tile (A, B) needs: keys visible to its last valid row
+    // Key tiles of MMA tile x (a select, so that no per-tile array lands in local memory).
+    __device__ __forceinline__ int nkt_of(int x) const { return x ? nkt_b : nkt_a; }
     bool has_b, sane;
 };
 
@@ -230,9 +234,9 @@ __device__ __forceinline__ TileCtx tile_ctx(const PrefillArgs& a, int t) {
     c.G = a.group;
     c.tt = 128 / c.G;
     c.has_b = c.tok0 + c.tt < c.n;
-    c.nkt_x[0] = (min(c.ctx, c.prior + min(c.n, c.tok0 + c.tt)) + 127) / 128;
-    c.nkt_x[1] = c.has_b ? (min(c.ctx, c.prior + min(c.n, c.tok0 + 2 * c.tt)) + 127) / 128 : 0;
-    c.nkt = max(c.nkt_x[0], c.nkt_x[1]);
+    c.nkt_a = (min(c.ctx, c.prior + min(c.n, c.tok0 + c.tt)) + 127) / 128;
+    c.nkt_b = c.has_b ? (min(c.ctx, c.prior + min(c.n, c.tok0 + 2 * c.tt)) + 127) / 128 : 0;
+    c.nkt = max(c.nkt_a, c.nkt_b);
     c.nblk_ctx = (c.ctx + kBlockSize - 1) / kBlockSize;
     c.rows_total = a.num_blocks * a.num_kv_heads * kBlockSize;
     c.sane = c.nkt >= 1 && c.n > 1 && c.tok0 < c.n;
@@ -269,7 +273,7 @@ __device__ __forceinline__ void tile_producer(const PrefillArgs& a, const CUtens
         }
     }
     int ids = -1, ids_base = -1;
-    int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
+    int last_k = -1, last_v = -1;  // the last key tile whose K (V) loads were issued
     bool ok = true;
     for (int kt = 0; kt < tile.nkt && ok; ++kt) {
         const int s = kt & 1;
@@ -304,7 +308,7 @@ __device__ __forceinline__ void tile_producer(const PrefillArgs& a, const CUtens
                 tma_load_2d(ks + kHalf + i * 2048, tm_k, 64, y[i], &bars[B_KF0 + s]);
             }
         }
-        issued_k[s] = kt;
+        last_k = kt;
         if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_VE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 101));
         if (!ok) break;
         if (lane == 0) {
@@ -316,14 +320,16 @@ __device__ __forceinline__ void tile_producer(const PrefillArgs& a, const CUtens
                 tma_load_2d(vs + kHalf + i * 2048, tm_v, 64, y[i], &bars[B_VF0 + s]);
             }
         }
-        issued_v[s] = kt;
+        last_v = kt;
         __syncwarp();
     }
     if (!ok && lane == 0) {
         // Drain: wait (bounded) for the last loads issued into each stage.
         for (int s = 0; s < 2; ++s) {
-            if (issued_k[s] >= 0) (void)mbar_wait(&bars[B_KF0 + s], (issued_k[s] >> 1) & 1);
-            if (issued_v[s] >= 0) (void)mbar_wait(&bars[B_VF0 + s], (issued_v[s] >> 1) & 1);
+            // the last loads of stage s were for key tile last - ((last - s) & 1), if any
+            const int jk = last_k - ((last_k - s) & 1), jv = last_v - ((last_v - s) & 1);
+            if (last_k >= 0 && jk >= 0) (void)mbar_wait(&bars[B_KF0 + s], (jk >> 1) & 1);
+            if (last_v >= 0 && jv >= 0) (void)mbar_wait(&bars[B_VF0 + s], (jv >> 1) & 1);
         }
         (void)mbar_wait(&bars[B_Q], 0);
     }
@@ -371,14 +377,14 @@ __device__ __forceinline__ void tile_mma(const PrefillArgs& a, unsigned char* sm
             const bool next = kt + 1 < tile.nkt;
             bool k_ready = false, v_ready = false;
             for (int x = 0; x < 2 && ok; ++x) {
-                if (kt < tile.nkt_x[x]) {
+                if (kt < tile.nkt_of(x)) {
                     ok = wait_or_abort(&bars[B_PF0 + x], kt & 1, abort_flag, a.err, 202 + x);
                     if (ok && !v_ready) ok = v_ready = wait_or_abort(&bars[B_VF0 + s], (kt >> 1) & 1, abort_flag, a.err, 204);
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(x, kt);
                 }
-                if (kt + 1 < tile.nkt_x[x]) {
+                if (kt + 1 < tile.nkt_of(x)) {
                     if (!k_ready) ok = k_ready = wait_or_abort(&bars[B_KF0 + (s ^ 1)], ((kt + 1) >> 1) & 1, abort_flag, a.err, 206);
                     if (!ok) break;
                     tc_fence_after();
@@ -398,8 +404,8 @@ __device__ __forceinline__ void tile_mma(const PrefillArgs& a, unsigned char* sm
                     ok = wait_or_abort(&bars[B_KE0 + st], (last >> 1) & 1, abort_flag, a.err, 207);
                     if (ok) ok = wait_or_abort(&bars[B_VE0 + st], (last >> 1) & 1, abort_flag, a.err, 208);
                 }
-                if (ok && tile.nkt_x[st] > 0)
-                    ok = wait_or_abort(&bars[B_OF0 + st], (tile.nkt_x[st] - 1) & 1, abort_flag, a.err, 209);
+                if (ok && tile.nkt_of(st) > 0)
+                    ok = wait_or_abort(&bars[B_OF0 + st], (tile.nkt_of(st) - 1) & 1, abort_flag, a.err, 209);
             }
         } else {
             tc_commit(&bars[B_DRAIN]);
@@ -423,7 +429,7 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
     const uint32_t ts = tl + x * 128, to = tl + 256 + x * 128;
     // Keys below this bound are visible to every row of the tile: no masking needed there.
     const int all_visible = tile.prior + tile.tok0 + x * tile.tt + 1;
-    const int my_nkt = tile.nkt_x[x];
+    const int my_nkt = tile.nkt_of(x);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int kt = 0; kt < my_nkt && ok; ++kt) {
@@ -543,7 +549,7 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
         tmem_wait_st();
         // V rows past the context (only possible in the CTA's final key tile) are zeroed by the
         // tile whose PV of that key tile is issued first: A when it reaches it, else B.
-        if (kt == tile.nkt - 1 && (kt + 1) * 128 > tile.ctx && x == (tile.nkt_x[0] == tile.nkt ? 0 : 1)) {
+        if (kt == tile.nkt - 1 && (kt + 1) * 128 > tile.ctx && x == (tile.nkt_a == tile.nkt ? 0 : 1)) {
             ok = warp_all(wait_or_abort(&bars[B_VF0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 302));
             if (!ok) break;
             unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
@@ -595,7 +601,7 @@ constexpr int kJobNone = -3;    // nothing in this step
 // other. In a round of items, warps 0-7 each run the warp-MMA loop over two stages carved from the
 // tile buffers (the third warpgroup waits). The last CTA to finish (a.work[3] counts them) resets
 // the counters for the next launch.
-template <typename T, int POLY, bool MIXED>
+template <typename T, int POLY, int DEC>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const PrefillArgs a, const DecodeArgs d, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -647,8 +653,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             first = __shfl_sync(FULL_MASK, first, 0);
             uint64_t* dbars = reinterpret_cast<uint64_t*>(smem + OFF_DBAR) + warp * kDecodeStages;
             volatile int* fifo = reinterpret_cast<volatile int*>(smem + OFF_FIFO) + warp * mma::kFifo;
-            if (!mma::decode_warp<T, kDecodeStages>(d, &tm_k, &tm_v, smem + warp * kDecodeStages * mma::kStage, dbars,
-                                                    fifo, first, 0) && lane == 0)
+            if (!mma::decode_warp<T, kDecodeStages, DEC == 2>(d, &tm_k, &tm_v, smem + warp * kDecodeStages * mma::kStage,
+                                                               dbars, fifo, first, 0) &&
+                lane == 0)
                 *abort_flag = 1;
             fence_proxy_async_smem();   // its generic writes (zeroed V rows) before later TMA writes
         };
@@ -656,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             return d.num_items > 0 && *reinterpret_cast<volatile int*>(&d.work[0]) < d.num_items && !*abort_flag;
         };
         // (a) CTAs that start on items: a round of them first.
-        if constexpr (MIXED) {
+        if constexpr (DEC != 0) {
             if (threadIdx.x == 0) *ctrl = ((int)blockIdx.x < a.decode_ctas && items_left()) ? kJobDecode : kJobNone;
             cta_sync();                                   // (1)
             if (*ctrl == kJobDecode) decode_round();
@@ -686,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (job < 0) break;
         }
         // (c) the items still left once the tiles are gone.
-        if constexpr (MIXED) {
+        if constexpr (DEC != 0) {
             if (threadIdx.x == 0) *ctrl = items_left() ? kJobDecode : kJobNone;
             cta_sync();                                   // (1)
             if (*ctrl == kJobDecode) decode_round();
@@ -710,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <typename T, int POLY, bool MIXED>
+template <typename T, int POLY, int DEC>
 cudaError_t launch_t(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cudaStream_t s) {
     const CUtensorMapDataType dt =
         std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -733,7 +740,7 @@ cudaError_t launch_t(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cud
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(prefill_tc_kernel<T, POLY, MIXED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(prefill_tc_kernel<T, POLY, DEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = 1;
@@ -741,32 +748,18 @@ cudaError_t launch_t(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cud
     // One persistent CTA per SM (fewer when the batch has fewer tiles and no split-K items).
     int grid = num_sms;
     if (d.num_items <= 0 && a.num_tiles < grid) grid = a.num_tiles;
-    return launch_k(a.pdl, prefill_tc_kernel<T, POLY, MIXED>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, a, d, mq, mk,
+    return launch_k(a.pdl, prefill_tc_kernel<T, POLY, DEC>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, a, d, mq, mk,
                     mv);
 }
 
-int poly_pairs() {
-    static const int v = [] {
-        const char* e = getenv("PKV_PREFILL_POLY_PAIRS");
-        return e ? atoi(e) : kPolyPairs;
-    }();
-    return v;
-}
-
-template <typename T, bool MIXED>
-cudaError_t launch_p(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cudaStream_t s) {
-    switch (poly_pairs()) {
-        case 2: return launch_t<T, 2, MIXED>(a, d, num_sms, s);
-        case 4: return launch_t<T, 4, MIXED>(a, d, num_sms, s);
-        default: return launch_t<T, kPolyPairs, MIXED>(a, d, num_sms, s);
-    }
-}
-
 // Batches with tcgen05 tiles only run an instantiation without the split-K rounds (fewer registers
-// live in the softmax warps).
+// live in the softmax warps); mixed batches one whose rounds take the item form of the batch's
+// items (the transposed form for items of at most 8 (row, head) slots).
 template <typename T>
 cudaError_t launch_m(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cudaStream_t s) {
-    return d.num_items > 0 ? launch_p<T, true>(a, d, num_sms, s) : launch_p<T, false>(a, d, num_sms, s);
+    if (d.num_items <= 0) return launch_t<T, kPolyPairs, 0>(a, d, num_sms, s);
+    return d.slots_per_item <= 8 ? launch_t<T, kPolyPairs, 2>(a, d, num_sms, s)
+                                 : launch_t<T, kPolyPairs, 1>(a, d, num_sms, s);
 }
 
 }  // namespace
