@@ -61,8 +61,8 @@ constexpr int OFF_V = OFF_K + 2 * kTile;    // 2 stages
 constexpr int OFF_BAR = OFF_V + 2 * kTile;
 // barrier slots (8 bytes each); per-tile barriers are indexed by tile 0 (A) / 1 (B)
 enum {
-    B_Q = 0, B_KF0 = 1, B_VF0 = 3, B_KE0 = 5, B_VE0 = 7, B_SF0 = 9, B_PF0 = 11, B_OF0 = 13, B_DRAIN = 15,
-    NUM_BARS = 16
+    B_Q = 0, B_F0 = 1, B_E0 = 3, B_SF0 = 5, B_PF0 = 7, B_OF0 = 9, B_DRAIN = 11,
+    NUM_BARS = 12
 };
 constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;     // tcgen05.alloc result
 constexpr int OFF_ABORT = OFF_TMEM + 4;
@@ -248,10 +248,8 @@ __device__ __forceinline__ TileCtx tile_ctx(const PrefillArgs& a, int t) {
 __device__ __forceinline__ void init_tile_barriers(uint64_t* bars) {
     mbar_init(&bars[B_Q], 1);
     for (int s = 0; s < 2; ++s) {
-        mbar_init(&bars[B_KF0 + s], 1);
-        mbar_init(&bars[B_VF0 + s], 1);
-        mbar_init(&bars[B_KE0 + s], 1);
-        mbar_init(&bars[B_VE0 + s], 1);
+        mbar_init(&bars[B_F0 + s], 1);
+        mbar_init(&bars[B_E0 + s], 1);
         mbar_init(&bars[B_SF0 + s], 1);
         mbar_init(&bars[B_PF0 + s], 128);
         mbar_init(&bars[B_OF0 + s], 1);
@@ -261,75 +259,82 @@ __device__ __forceinline__ void init_tile_barriers(uint64_t* bars) {
 }
 
 // ---- TMA producer (warp 8) ----
+// Loads go in groups, one barrier wait and one transaction barrier per key tile: the Q tiles with
+// K(0) on B_Q, then group kt = V(kt) and K(kt+1) on B_F(kt & 1), the two operands the MMA issuer
+// consumes in its iteration kt (PV(kt), QK^T(kt+1)). V(kt) goes to V stage kt & 1, K(kt+1) to K
+// stage (kt+1) & 1, so group kt reuses the stages of group kt-2, which the issuer frees with one
+// commit on B_E(kt & 1) at the end of its iteration kt-2; for group 1 that is the commit after
+// the prologue's QK^T(0), which frees K(0)'s stage. Lane l < 16 serves one block of a group:
+// l < 8 block l of V(kt), l >= 8 block l-8 of K(kt+1); each lane reads its own block-table entry
+// a group ahead.
 __device__ __forceinline__ void tile_producer(const PrefillArgs& a, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                               const CUtensorMap* tm_v, unsigned char* smem, uint64_t* bars,
                                               volatile int* abort_flag, const TileCtx& tile, int lane) {
+    const int j = lane & 7;
+    // Table entry of block j of key tile t: -2 past the context (never read), -3 past the table's
+    // width (device lengths larger than the planned ones: a range error below).
+    auto block_id = [&](int t) -> int {
+        const int b = t * 8 + j;
+        return b >= tile.nblk_ctx ? -2
+               : b < a.max_blocks_per_seq ? __ldg(a.block_tables + (size_t)tile.req * a.max_blocks_per_seq + b) : -3;
+    };
+    // Pool row of that block's K/V for this KV head; the row past the pool (zero fill) past the
+    // context or on a range error.
+    auto block_row = [&](int id, int t) -> int {
+        if (id == -2) return tile.rows_total;
+        if (id < 0 || id >= a.num_blocks) {
+            record_error(a.err, 6 /*PKV_ERR_DEVICE_RANGE*/, (long long)tile.req * a.max_blocks_per_seq + t * 8 + j);
+            return tile.rows_total;
+        }
+        return (id * a.num_kv_heads + tile.kvh) * kBlockSize;
+    };
+    const bool v_lane = lane < 8, k_lane = lane >= 8 && lane < 16;
+    const int id0 = k_lane ? block_id(0) : 0;
     if (lane == 0) {
-        mbar_arrive_expect_tx(&bars[B_Q], tile.has_b ? 2 * kTile : kTile);
+        mbar_arrive_expect_tx(&bars[B_Q], (tile.has_b ? 2 * kTile : kTile) + kTile);
         for (int x = 0; x < (tile.has_b ? 2 : 1); ++x) {
             const int z = tile.q0 + tile.tok0 + x * tile.tt;
             tma_load_3d(smem + OFF_Q + x * kTile, tm_q, 0, tile.kvh * tile.G, z, &bars[B_Q]);
             tma_load_3d(smem + OFF_Q + x * kTile + kHalf, tm_q, 64, tile.kvh * tile.G, z, &bars[B_Q]);
         }
     }
-    int ids = -1, ids_base = -1;
-    int last_k = -1, last_v = -1;  // the last key tile whose K (V) loads were issued
+    __syncwarp();
+    if (k_lane) {
+        const int y = block_row(id0, 0);
+        tma_load_2d(smem + OFF_K + j * 2048, tm_k, 0, y, &bars[B_Q]);
+        tma_load_2d(smem + OFF_K + kHalf + j * 2048, tm_k, 64, y, &bars[B_Q]);
+    }
+    int id_next = v_lane ? block_id(0) : k_lane && 1 < tile.nkt ? block_id(1) : -2;
+    int last = -1;  // the last group issued
     bool ok = true;
     for (int kt = 0; kt < tile.nkt && ok; ++kt) {
-        const int s = kt & 1;
-        if (ids_base < 0 || kt * 8 >= ids_base + 32) {
-            ids_base = kt * 8;
-            // Entries past the context are never read (-2: zero fill). The context comes from the
-            // device lengths, so an entry past the table's width (device lengths larger than the
-            // planned ones) is not read either: -3 is recorded as a range error below.
-            const int b = ids_base + lane;
-            ids = b >= tile.nblk_ctx ? -2
-                  : b < a.max_blocks_per_seq ? __ldg(a.block_tables + (size_t)tile.req * a.max_blocks_per_seq + b) : -3;
-        }
-        int y[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int id = __shfl_sync(FULL_MASK, ids, kt * 8 - ids_base + i);
-            if (id == -2) y[i] = tile.rows_total;                       // past the context: zero fill
-            else if (id < 0 || id >= a.num_blocks) {
-                if (lane == 0) record_error(a.err, 6 /*PKV_ERR_DEVICE_RANGE*/, (long long)tile.req * a.max_blocks_per_seq + kt * 8 + i);
-                y[i] = tile.rows_total;
-            } else y[i] = (id * a.num_kv_heads + tile.kvh) * kBlockSize;
-        }
-        // K of tile kt may land once both QK^T of tile kt-2 are done; V once both PV of tile kt-2.
-        if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_KE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 100));
+        const int g = kt & 1;
+        const bool has_k = kt + 1 < tile.nkt;
+        const int id = id_next;
+        if (has_k) id_next = v_lane ? block_id(kt + 1) : k_lane && kt + 2 < tile.nkt ? block_id(kt + 2) : -2;
+        if (kt >= 1) ok = warp_all(wait_or_abort(&bars[B_E0 + g], ((kt - 2 + g) >> 1) & 1, abort_flag, a.err, 100));
         if (!ok) break;
-        if (lane == 0) {
-            unsigned char* ks = smem + OFF_K + s * kTile;
-            mbar_arrive_expect_tx(&bars[B_KF0 + s], kTile);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                tma_load_2d(ks + i * 2048, tm_k, 0, y[i], &bars[B_KF0 + s]);
-                tma_load_2d(ks + kHalf + i * 2048, tm_k, 64, y[i], &bars[B_KF0 + s]);
-            }
+        if (lane == 0) mbar_arrive_expect_tx(&bars[B_F0 + g], has_k ? 2 * kTile : kTile);
+        __syncwarp();
+        if (v_lane) {
+            unsigned char* vs = smem + OFF_V + g * kTile;
+            const int y = block_row(id, kt);
+            tma_load_2d(vs + j * 2048, tm_v, 0, y, &bars[B_F0 + g]);
+            tma_load_2d(vs + kHalf + j * 2048, tm_v, 64, y, &bars[B_F0 + g]);
+        } else if (k_lane && has_k) {
+            unsigned char* ks = smem + OFF_K + (g ^ 1) * kTile;
+            const int y = block_row(id, kt + 1);
+            tma_load_2d(ks + j * 2048, tm_k, 0, y, &bars[B_F0 + g]);
+            tma_load_2d(ks + kHalf + j * 2048, tm_k, 64, y, &bars[B_F0 + g]);
         }
-        last_k = kt;
-        if (kt >= 2) ok = warp_all(wait_or_abort(&bars[B_VE0 + s], ((kt - 2) >> 1) & 1, abort_flag, a.err, 101));
-        if (!ok) break;
-        if (lane == 0) {
-            unsigned char* vs = smem + OFF_V + s * kTile;
-            mbar_arrive_expect_tx(&bars[B_VF0 + s], kTile);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                tma_load_2d(vs + i * 2048, tm_v, 0, y[i], &bars[B_VF0 + s]);
-                tma_load_2d(vs + kHalf + i * 2048, tm_v, 64, y[i], &bars[B_VF0 + s]);
-            }
-        }
-        last_v = kt;
+        last = kt;
         __syncwarp();
     }
     if (!ok && lane == 0) {
-        // Drain: wait (bounded) for the last loads issued into each stage.
-        for (int s = 0; s < 2; ++s) {
-            // the last loads of stage s were for key tile last - ((last - s) & 1), if any
-            const int jk = last_k - ((last_k - s) & 1), jv = last_v - ((last_v - s) & 1);
-            if (last_k >= 0 && jk >= 0) (void)mbar_wait(&bars[B_KF0 + s], (jk >> 1) & 1);
-            if (last_v >= 0 && jv >= 0) (void)mbar_wait(&bars[B_VF0 + s], (jv >> 1) & 1);
+        // Drain: wait (bounded) for the last group issued on each barrier, and for Q with K(0).
+        for (int g = 0; g < 2; ++g) {
+            const int jl = last - ((last - g) & 1);
+            if (last >= 0 && jl >= 0) (void)mbar_wait(&bars[B_F0 + g], (jl >> 1) & 1);
         }
         (void)mbar_wait(&bars[B_Q], 0);
     }
@@ -364,48 +369,42 @@ __device__ __forceinline__ void tile_mma(const PrefillArgs& a, unsigned char* sm
                           id_pv, kt > 0 || k > 0);
             tc_commit(&bars[B_OF0 + x]);
         };
-        bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, a.err, 200);
-        if (ok) ok = wait_or_abort(&bars[B_KF0], 0, abort_flag, a.err, 201);
+        // Each barrier wait of this thread leaves the tensor pipe idle for its latency, so an
+        // iteration waits three times: P_A, the group's loads (once), P_B; and commits once.
+        bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag, a.err, 200);   // Q tiles and K(0)
         if (ok) {
             tc_fence_after();
             issue_qk(0, 0);
             if (tile.has_b) issue_qk(1, 0);
-            tc_commit(&bars[B_KE0]);
+            tc_commit(&bars[B_E0 + 1]);   // K(0)'s stage, for group 1
         }
         for (int kt = 0; kt < tile.nkt && ok; ++kt) {
-            const int s = kt & 1;
-            const bool next = kt + 1 < tile.nkt;
-            bool k_ready = false, v_ready = false;
+            const int g = kt & 1;
+            bool f_ready = false;
             for (int x = 0; x < 2 && ok; ++x) {
                 if (kt < tile.nkt_of(x)) {
                     ok = wait_or_abort(&bars[B_PF0 + x], kt & 1, abort_flag, a.err, 202 + x);
-                    if (ok && !v_ready) ok = v_ready = wait_or_abort(&bars[B_VF0 + s], (kt >> 1) & 1, abort_flag, a.err, 204);
+                    if (ok && !f_ready) ok = f_ready = wait_or_abort(&bars[B_F0 + g], (kt >> 1) & 1, abort_flag, a.err, 204);
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(x, kt);
                 }
-                if (kt + 1 < tile.nkt_of(x)) {
-                    if (!k_ready) ok = k_ready = wait_or_abort(&bars[B_KF0 + (s ^ 1)], ((kt + 1) >> 1) & 1, abort_flag, a.err, 206);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_qk(x, kt + 1);
-                }
+                // QK^T(kt+1) of tile x follows its PV(kt) (kt + 1 < nkt_x implies kt < nkt_x), so
+                // group kt (which holds K(kt+1)) has been waited for.
+                if (kt + 1 < tile.nkt_of(x)) issue_qk(x, kt + 1);
             }
             if (!ok) break;
-            tc_commit(&bars[B_VE0 + s]);
-            if (next) tc_commit(&bars[B_KE0 + (s ^ 1)]);
+            tc_commit(&bars[B_E0 + g]);
         }
         if (ok) {
             // Every commit of this tile has arrived before the barriers are armed for the next one:
-            // the last phase of each K and V stage and of each tile's O.
-            for (int st = 0; st < 2 && ok; ++st) {
-                const int last = st < tile.nkt ? tile.nkt - 1 - ((tile.nkt - 1 - st) & 1) : -1;  // last key tile of stage st
-                if (last >= 0) {
-                    ok = wait_or_abort(&bars[B_KE0 + st], (last >> 1) & 1, abort_flag, a.err, 207);
-                    if (ok) ok = wait_or_abort(&bars[B_VE0 + st], (last >> 1) & 1, abort_flag, a.err, 208);
-                }
-                if (ok && tile.nkt_of(st) > 0)
-                    ok = wait_or_abort(&bars[B_OF0 + st], (tile.nkt_of(st) - 1) & 1, abort_flag, a.err, 209);
+            // the last phase of each stage-free barrier (B_E0 takes iterations 0, 2, ...; B_E1 the
+            // prologue and iterations 1, 3, ...) and of each tile's O.
+            const int n_e[2] = {(tile.nkt + 1) / 2, 1 + tile.nkt / 2};
+            for (int g = 0; g < 2 && ok; ++g) {
+                ok = wait_or_abort(&bars[B_E0 + g], (n_e[g] - 1) & 1, abort_flag, a.err, 207);
+                if (ok && tile.nkt_of(g) > 0)
+                    ok = wait_or_abort(&bars[B_OF0 + g], (tile.nkt_of(g) - 1) & 1, abort_flag, a.err, 209);
             }
         } else {
             tc_commit(&bars[B_DRAIN]);
@@ -550,7 +549,7 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
         // V rows past the context (only possible in the CTA's final key tile) are zeroed by the
         // tile whose PV of that key tile is issued first: A when it reaches it, else B.
         if (kt == tile.nkt - 1 && (kt + 1) * 128 > tile.ctx && x == (tile.nkt_a == tile.nkt ? 0 : 1)) {
-            ok = warp_all(wait_or_abort(&bars[B_VF0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 302));
+            ok = warp_all(wait_or_abort(&bars[B_F0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 302));
             if (!ok) break;
             unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
             const int r0 = tile.ctx - kt * 128;  // first V row past the context
