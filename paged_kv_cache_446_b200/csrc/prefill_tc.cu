@@ -61,8 +61,8 @@ constexpr int OFF_V = OFF_K + 2 * kTile;    // 2 stages
 constexpr int OFF_BAR = OFF_V + 2 * kTile;
 // barrier slots (8 bytes each); per-tile barriers are indexed by tile 0 (A) / 1 (B)
 enum {
-    B_Q = 0, B_F0 = 1, B_E0 = 3, B_SF0 = 5, B_PF0 = 7, B_OF0 = 9, B_DRAIN = 11,
-    NUM_BARS = 12
+    B_Q = 0, B_F0 = 1, B_E0 = 3, B_SF0 = 5, B_PF0 = 7, B_OF0 = 9, B_DRAIN = 11, B_PH0 = 12, B_OH0 = 14,
+    NUM_BARS = 16
 };
 constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;     // tcgen05.alloc result
 constexpr int OFF_ABORT = OFF_TMEM + 4;
@@ -253,6 +253,8 @@ __device__ __forceinline__ void init_tile_barriers(uint64_t* bars) {
         mbar_init(&bars[B_SF0 + s], 1);
         mbar_init(&bars[B_PF0 + s], 128);
         mbar_init(&bars[B_OF0 + s], 1);
+        mbar_init(&bars[B_PH0 + s], 128);
+        mbar_init(&bars[B_OH0 + s], 1);
     }
     mbar_init(&bars[B_DRAIN], 1);
     fence_mbar_init();
@@ -359,15 +361,15 @@ __device__ __forceinline__ void tile_mma(const PrefillArgs& a, unsigned char* sm
             }
             tc_commit(&bars[B_SF0 + x]);
         };
-        auto issue_pv = [&](int x, int kt) {
+        // PV of one half (64 keys) of key tile kt. P_X(kt) sits as packed 16-bit pairs in the first
+        // 64 columns of S_X; each K step of 16 keys is 8 columns.
+        auto issue_pv = [&](int x, int kt, int h) {
             const unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
-            // P_X(kt) sits as packed 16-bit pairs in the first 64 columns of S_X; each K step of
-            // 16 keys is 8 columns.
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
+            for (int k = 4 * h; k < 4 * h + 4; ++k)
                 tc_mma_ts(tmem + 256 + x * 128, tmem + x * 128 + k * 8, smem_desc(vs + k * 2048, kHalf, 1024),
                           id_pv, kt > 0 || k > 0);
-            tc_commit(&bars[B_OF0 + x]);
+            tc_commit(&bars[(h ? B_OF0 : B_OH0) + x]);
         };
         // Each barrier wait of this thread leaves the tensor pipe idle for its latency, so an
         // iteration waits three times: P_A, the group's loads (once), P_B; and commits once.
@@ -383,11 +385,15 @@ __device__ __forceinline__ void tile_mma(const PrefillArgs& a, unsigned char* sm
             bool f_ready = false;
             for (int x = 0; x < 2 && ok; ++x) {
                 if (kt < tile.nkt_of(x)) {
-                    ok = wait_or_abort(&bars[B_PF0 + x], kt & 1, abort_flag, a.err, 202 + x);
+                    ok = wait_or_abort(&bars[B_PH0 + x], kt & 1, abort_flag, a.err, 210 + x);
                     if (ok && !f_ready) ok = f_ready = wait_or_abort(&bars[B_F0 + g], (kt >> 1) & 1, abort_flag, a.err, 204);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(x, kt);
+                    issue_pv(x, kt, 0);
+                    ok = wait_or_abort(&bars[B_PF0 + x], kt & 1, abort_flag, a.err, 202 + x);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(x, kt, 1);
                 }
                 // QK^T(kt+1) of tile x follows its PV(kt) (kt + 1 < nkt_x implies kt < nkt_x), so
                 // group kt (which holds K(kt+1)) has been waited for.
@@ -405,6 +411,8 @@ __device__ __forceinline__ void tile_mma(const PrefillArgs& a, unsigned char* sm
                 ok = wait_or_abort(&bars[B_E0 + g], (n_e[g] - 1) & 1, abort_flag, a.err, 207);
                 if (ok && tile.nkt_of(g) > 0)
                     ok = wait_or_abort(&bars[B_OF0 + g], (tile.nkt_of(g) - 1) & 1, abort_flag, a.err, 209);
+                if (ok && tile.nkt_of(g) > 0)
+                    ok = wait_or_abort(&bars[B_OH0 + g], (tile.nkt_of(g) - 1) & 1, abort_flag, a.err, 212);
             }
         } else {
             tc_commit(&bars[B_DRAIN]);
@@ -431,6 +439,26 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
     const int my_nkt = tile.nkt_of(x);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    // O in TMEM times f, row by row (warp-collective; rows whose factor is 1 are rewritten unchanged).
+    auto scale_o = [&](float f) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(to + c * 32, o);
+            tmem_wait_ld();
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * f);
+            tmem_st32(to + c * 32, w);
+        }
+    };
+    // P of the first half of a key tile (keys 0..63, columns 0..31) is signalled on B_PH, the rest
+    // on B_PF, so that the PV of the first half runs while the second half's exponentials are taken.
+    auto signal = [&](int bar) {
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars[bar + x]);
+    };
     for (int kt = 0; kt < my_nkt && ok; ++kt) {
         ok = warp_all(wait_or_abort(&bars[B_SF0 + x], kt & 1, abort_flag, a.err, 300));
         if (!ok) break;
@@ -439,11 +467,12 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
         float alpha = 1.f;
         float2 ps2 = make_float2(0.f, 0.f);
         if (full && a.scale_log2 >= 0.f) {
-            // Two TMEM round trips, one per half of the key tile: the half's maximum is taken in
+            // One TMEM round trip per half of the key tile: the half's maximum is taken in
             // registers and P computed from the same registers against the row's reference m,
             // raised first when the half exceeds it by more than the threshold. P of keys
-            // 64*h.. goes to columns 32*h.. (over S already read). If the second half raises m,
-            // the first half's P, already stored, is scaled down by the same factor.
+            // 64*h.. goes to columns 32*h.. (over S already read). A raise rescales what O holds
+            // against the old reference: PV(kt-1) before the first half (none when kt = 0), the
+            // first half's PV before the second.
             const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
 #pragma unroll 1
             for (int h = 0; h < 2; ++h) {
@@ -457,25 +486,19 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
                 hm *= a.scale_log2;
                 const bool raise = hm > m + kRescaleThreshold;
                 const float f = raise ? fast_exp2(m - hm) : 1.f;  // 0 while m is -inf
-                // The TMEM accesses are warp-collective: the whole warp takes this branch when
-                // any of its rows raised, each lane scaling its own row by its own factor.
-                if (h == 1 && __any_sync(FULL_MASK, raise)) {
-                    tmem_wait_st();
-                    float pv[32];
-                    tmem_ld32(ts, pv);
-                    tmem_wait_ld();
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float2 q = unpack2<T>(__float_as_uint(pv[i]));
-                        pk[i] = pack2<T>(q.x * f, q.y * f);
-                    }
-                    tmem_st32(ts, pk);
-                }
                 if (raise) {
                     ps2 = make_float2(ps2.x * f, ps2.y * f);
                     alpha *= f;
                     m = hm;
+                }
+                // The TMEM accesses are warp-collective: the whole warp takes this branch when
+                // any of its rows raised, each lane scaling its own row by its own factor.
+                if ((kt >= 1 || h == 1) && __any_sync(FULL_MASK, raise)) {
+                    ok = warp_all(h == 0 ? wait_or_abort(&bars[B_OF0 + x], (kt - 1) & 1, abort_flag, a.err, 301)
+                                         : wait_or_abort(&bars[B_OH0 + x], kt & 1, abort_flag, a.err, 304));
+                    if (!ok) break;
+                    tc_fence_after();
+                    scale_o(f);
                 }
                 const float2 nm2 = make_float2(-m, -m);
                 uint32_t pk[32];
@@ -487,7 +510,9 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
                     ps2 = __fadd2_rn(ps2, row_sum_term<T>(p, pk[i]));
                 }
                 tmem_st32(ts + h * 32, pk);
+                signal(h ? B_PF0 : B_PH0);
             }
+            if (!ok) break;
         } else {
             // pass 1: row maximum of scale * s over the visible keys
             float mx = -INFINITY;
@@ -504,6 +529,27 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
             if (mx > m + kRescaleThreshold) {
                 alpha = fast_exp2(m - mx);  // 0 on the first tile
                 m = mx;
+            }
+            // O against the old reference (PV(kt-1) complete) is rescaled before any P is signalled.
+            if (kt >= 1 && __any_sync(FULL_MASK, alpha != 1.f)) {
+                ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (kt - 1) & 1, abort_flag, a.err, 301));
+                if (!ok) break;
+                tc_fence_after();
+                scale_o(alpha);
+            }
+            // V rows past the context (only possible in the CTA's final key tile) are zeroed by the
+            // tile whose PV of that key tile is issued first: A when it reaches it, else B.
+            if (kt == tile.nkt - 1 && (kt + 1) * 128 > tile.ctx && x == (tile.nkt_a == tile.nkt ? 0 : 1)) {
+                ok = warp_all(wait_or_abort(&bars[B_F0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 302));
+                if (!ok) break;
+                unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
+                const int r0 = tile.ctx - kt * 128;  // first V row past the context
+                const int chunks = (128 - r0) * 16;  // 16-byte chunks over both halves
+                for (int c = (warp & 3) * 32 + lane; c < chunks; c += 128) {
+                    const int r = r0 + (c >> 4), h = (c >> 3) & 1, k = c & 7;
+                    *reinterpret_cast<uint4*>(vs + h * kHalf + r * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
             }
             // pass 2: p = 2^(s*scale - m), rounded to T, written over S as the A operand of PV.
             // Chunk c's P goes to columns 16c.., which pass 2 has already read.
@@ -524,44 +570,11 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
                     ps2 = __fadd2_rn(ps2, row_sum_term<T>(make_float2(p0, p1), pk[i]));
                 }
                 tmem_st16(ts + c * 16, pk);
+                if (c & 1) signal(c == 1 ? B_PH0 : B_PF0);
             }
         }
         const float ps = ps2.x + ps2.y;
         l = l * alpha + ps;
-        // Rescale O in TMEM when a row of this warp raised its reference (rare after the first
-        // tiles). PV(kt-1) must be complete before O is read.
-        if (kt >= 1 && __any_sync(FULL_MASK, alpha != 1.f)) {
-            ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (kt - 1) & 1, abort_flag, a.err, 301));
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float o[32];
-                tmem_ld32(to + c * 32, o);
-                tmem_wait_ld();
-                uint32_t w[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
-                tmem_st32(to + c * 32, w);
-            }
-        }
-        tmem_wait_st();
-        // V rows past the context (only possible in the CTA's final key tile) are zeroed by the
-        // tile whose PV of that key tile is issued first: A when it reaches it, else B.
-        if (kt == tile.nkt - 1 && (kt + 1) * 128 > tile.ctx && x == (tile.nkt_a == tile.nkt ? 0 : 1)) {
-            ok = warp_all(wait_or_abort(&bars[B_F0 + (kt & 1)], (kt >> 1) & 1, abort_flag, a.err, 302));
-            if (!ok) break;
-            unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
-            const int r0 = tile.ctx - kt * 128;  // first V row past the context
-            const int chunks = (128 - r0) * 16;  // 16-byte chunks over both halves
-            for (int c = (warp & 3) * 32 + lane; c < chunks; c += 128) {
-                const int r = r0 + (c >> 4), h = (c >> 3) & 1, k = c & 7;
-                *reinterpret_cast<uint4*>(vs + h * kHalf + r * 128 + k * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        mbar_arrive(&bars[B_PF0 + x]);
     }
     if (ok) ok = warp_all(wait_or_abort(&bars[B_OF0 + x], (my_nkt - 1) & 1, abort_flag, a.err, 303));
     if (ok) {
