@@ -100,7 +100,8 @@ def recorded_traffic(kernel: str, workload: str):
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel)
+            data = json.load(f)
+        rec = data.get(f"{kernel}@{workload}") or data.get(kernel)
         if not rec or rec.get("workload") != workload:
             return None
         with open(os.path.join(ROOT, rec["source"]), "rb") as f:
