@@ -307,8 +307,8 @@ pkv_status pkv_device_error(int* code, int64_t* detail, pkv_stream_t stream);
  * Arguments: the host batch description and options of pkv_attention_plan, then the device
  * tensors and scale of pkv_paged_attention (same layouts and meaning); out receives the result.
  * The array's device address is looked up on the first call made on each device (and again when
- * that device's current CUDA context is a different one, e.g. after cudaDeviceReset), so make that
- * first call before any stream capture begins. The batch is planned once per call, on the host. Every call reuses the same array, which keeps the
+ * that device's current CUDA context is a different one, e.g. after cudaDeviceReset), with
+ * cudaGetSymbolAddress. The batch is planned once per call, on the host. Every call reuses the same array, which keeps the
  * last call's contents; calls that may overlap on the GPU (other streams or host threads) race on
  * it and must be serialised by the caller. No part of it has to start zeroed: each call writes
  * what its kernels read.

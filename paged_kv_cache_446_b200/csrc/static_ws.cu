@@ -10,9 +10,9 @@
 //
 // The array (PKV_STATIC_WS_BYTES) is part of this file's device module: every GPU that loads it
 // holds the memory until the process exits. Its device address is looked up with
-// cudaGetSymbolAddress on the first call made with a device current, so make that first call before
-// any stream capture begins; the address is kept per CUDA context and looked up again when the
-// device's current context is a different one (for example after cudaDeviceReset). All calls share
+// cudaGetSymbolAddress on the first call made with a device current; the address is kept per CUDA
+// context and looked up again when the device's current context is a different one (for example
+// after cudaDeviceReset). All calls share
 // the one array and it keeps the contents of the last call: calls that can overlap on the GPU
 // (different streams, or different host threads) race on it and must be serialised by the caller.
 // Nothing in it has to start at zero -- each call writes every byte its kernels read (the uploaded
