@@ -115,6 +115,25 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc)
         : "memory");
 }
+// The same two MMAs with each shared-memory descriptor given as its low and high 32-bit words.
+__device__ __forceinline__ void tc_mma_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                                          bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 ad, {%1, %3};\n\tmov.b64 bd, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %4, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"((uint32_t)acc)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                             uint32_t idesc, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 bd, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"((uint32_t)acc)
+        : "memory");
+}
 // 32 lanes x 32 consecutive 32-bit columns from registers (thread i writes TMEM lane base + i).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
     asm volatile(
@@ -160,6 +179,9 @@ __device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo, uint3
     return (uint64_t)((a >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
+// High word of every shared-memory descriptor here: SBO 1024 bytes (bits 32-45), descriptor
+// version 1 (bit 46), 128-byte swizzling (bits 61-63 = 2).
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
 // Instruction descriptor of kind::f16 with fp32 accumulation, M = N = 128.
 __host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_format, uint32_t b_mn_major) {
     return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (b_mn_major << 16) | ((128u >> 3) << 17) |
@@ -339,25 +361,32 @@ __device__ __forceinline__ void tile_mma(const PrefillArgs& a, unsigned char* sm
         const uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
         const uint32_t id_qk = idesc_f16(fmt, 0);
         const uint32_t id_pv = idesc_f16(fmt, 1);
+        // This thread shares its SM sub-partition with two busy softmax warps, so each of its
+        // instructions waits for an issue slot while the tensor pipe may run dry. The shared-memory
+        // descriptors are therefore a precomputed low word plus a constant per MMA (the high word,
+        // SBO 1024 with 128-byte swizzling, is the same for all).
+        const uint32_t base = smem_u32(smem) >> 4;
+        const uint32_t lo_q = base + (OFF_Q >> 4) + (1u << 16);                       // K-major, LBO 16 B
+        const uint32_t lo_k = base + (OFF_K >> 4) + (1u << 16);
+        const uint32_t lo_v = base + (OFF_V >> 4) + ((uint32_t)(kHalf >> 4) << 16);   // MN-major, LBO one half
         auto issue_qk = [&](int x, int kt) {
-            const unsigned char* ks = smem + OFF_K + (kt & 1) * kTile;
-            const unsigned char* qs = smem + OFF_Q + x * kTile;
+            const uint32_t qa = lo_q + (uint32_t)x * (kTile >> 4), kb = lo_k + (uint32_t)(kt & 1) * (kTile >> 4);
+            const uint32_t d = tmem + x * 128;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const int half = k >> 2, off = (k & 3) * 32;
-                tc_mma(tmem + x * 128, smem_desc(qs + half * kHalf + off, 16, 1024),
-                       smem_desc(ks + half * kHalf + off, 16, 1024), id_qk, k > 0);
+                const uint32_t off = (uint32_t)(((k >> 2) * kHalf + (k & 3) * 32) >> 4);
+                tc_mma_lo(d, qa + off, kb + off, kDescHi, id_qk, k > 0);
             }
             tc_commit(&bars[B_SF0 + x]);
         };
         // PV of one half (64 keys) of key tile kt. P_X(kt) sits as packed 16-bit pairs in the first
         // 64 columns of S_X; each K step of 16 keys is 8 columns.
         auto issue_pv = [&](int x, int kt, int h) {
-            const unsigned char* vs = smem + OFF_V + (kt & 1) * kTile;
+            const uint32_t vb = lo_v + (uint32_t)(kt & 1) * (kTile >> 4);
+            const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128;
 #pragma unroll
             for (int k = 4 * h; k < 4 * h + 4; ++k)
-                tc_mma_ts(tmem + 256 + x * 128, tmem + x * 128 + k * 8, smem_desc(vs + k * 2048, kHalf, 1024),
-                          id_pv, kt > 0 || k > 0);
+                tc_mma_ts_lo(d, pa + k * 8, vb + (uint32_t)(k * (2048 >> 4)), kDescHi, id_pv, kt > 0 || k > 0);
             tc_commit(&bars[(h ? B_OF0 : B_OH0) + x]);
         };
         // Each barrier wait of this thread leaves the tensor pipe idle for its latency, so an
