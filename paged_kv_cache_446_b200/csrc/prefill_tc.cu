@@ -23,10 +23,12 @@
 // mixed batch they also serve the split-K decode items (warps 0-7 run the warp-MMA loop of
 // decode_mma.cuh over buffers carved from the tile stages), so the HBM-bound decode rows and the
 // tensor-bound tiles share the GPU in one launch.
-// A softmax thread reads its row's key tile in two halves of 64 columns (one TMEM round trip each).
-// O accumulates in TMEM across key tiles. A row's exponentials use a reference maximum that is
-// raised only when a tile's maximum exceeds it by 2^8; O is then rescaled in TMEM (exact: softmax is
-// shift invariant, and p stays <= 2^8).
+// A softmax thread reads its row's key tile in two halves of 64 columns (one TMEM round trip each)
+// and signals each half's P separately. O accumulates in TMEM across key tiles. A row's
+// exponentials use a reference maximum that is raised only when a half's maximum exceeds it by
+// 2^8; O is then rescaled in TMEM (exact: softmax is shift invariant, and p stays <= 2^8). The
+// half's maximum is only taken when the weights' sum against the current reference shows that a
+// raise may be due.
 // Blocks past the context are fetched at an out-of-range coordinate (TMA fills zeros); V rows past
 // the context inside the last block are zeroed before PV (stale slots may hold anything).
 // Every wait is bounded; on expiry the CTA records PKV_ERR_DEVICE_TIMEOUT, drains its own copies
@@ -64,7 +66,8 @@ enum {
     B_Q = 0, B_F0 = 1, B_E0 = 3, B_SF0 = 5, B_PF0 = 7, B_OF0 = 9, B_DRAIN = 11, B_PH0 = 12, B_OH0 = 14,
     NUM_BARS = 16
 };
-constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;     // tcgen05.alloc result
+constexpr int OFF_TMEM = OFF_BAR + 2 * NUM_BARS * 8; // tcgen05.alloc result (after two barrier sets)
+constexpr int OFF_BSET = OFF_TMEM + 12;              // the current tile's barrier set (thread 0 writes it)
 constexpr int OFF_ABORT = OFF_TMEM + 4;
 constexpr int OFF_CTRL = OFF_ABORT + 4;              // the CTA's next step (thread 0 writes it)
 // Rounds of split-K items: warps 0-7 each use kDecodeStages stages of the tile buffers (8 x 2 x 12 KiB
@@ -80,6 +83,9 @@ constexpr uint32_t kTmemCols = 512;                  // S_A [0,128), S_B [128,25
 // A row's exponentials use a reference max that is only raised when the tile max exceeds it by
 // more than this (log2 units); the result is exact (softmax is shift invariant) and p <= 2^8.
 constexpr float kRescaleThreshold = 8.f;
+// A half key tile whose weights (against the current reference) sum to at most this has none
+// above 2^kRescaleThreshold, even counting the fp16 rounding of the summed weights.
+constexpr float kRescaleBound = 255.f;
 // Of each 32 exponentials of an unmasked key tile, 2 * POLY are computed by exp2_poly2 on the FMA
 // pipe (the kernel's template parameter). Measured slower at every share tried (MUFU is not what
 // bounds the softmax: ex2 runs at 16 per clock per SM and the softmax keeps it about half busy), so
@@ -100,22 +106,8 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc)
-        : "memory");
-}
-// Same MMA with the A operand (M x K, K-major, two 16-bit elements per 32-bit column) in TMEM.
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, bool acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc)
-        : "memory");
-}
-// The same two MMAs with each shared-memory descriptor given as its low and high 32-bit words.
+// tcgen05.mma kind::f16 with each shared-memory descriptor given as its low and high 32-bit words;
+// the _ts form reads the A operand (M x K, K-major, two 16-bit elements per 32-bit column) from TMEM.
 __device__ __forceinline__ void tc_mma_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
                                           bool acc) {
     asm volatile(
@@ -173,12 +165,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Shared-memory matrix descriptor, SWIZZLE_128B (layout type 2), descriptor version 1.
-__device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo, uint32_t sbo) {
-    const uint32_t a = smem_u32(p);
-    return (uint64_t)((a >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
 // High word of every shared-memory descriptor here: SBO 1024 bytes (bits 32-45), descriptor
 // version 1 (bit 46), 128-byte swizzling (bits 61-63 = 2).
 constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
@@ -498,35 +484,50 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
                 tmem_ld32(ts + h * 64, sv);
                 tmem_ld32(ts + h * 64 + 32, sv + 32);
                 tmem_wait_ld();
-                float hm = -INFINITY;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) hm = fmaxf(hm, sv[i]);
-                hm *= a.scale_log2;
-                const bool raise = hm > m + kRescaleThreshold;
-                const float f = raise ? fast_exp2(m - hm) : 1.f;  // 0 while m is -inf
-                if (raise) {
-                    ps2 = make_float2(ps2.x * f, ps2.y * f);
-                    alpha *= f;
-                    m = hm;
-                }
-                // The TMEM accesses are warp-collective: the whole warp takes this branch when
-                // any of its rows raised, each lane scaling its own row by its own factor.
-                if ((kt >= 1 || h == 1) && __any_sync(FULL_MASK, raise)) {
-                    ok = warp_all(h == 0 ? wait_or_abort(&bars[B_OF0 + x], (kt - 1) & 1, abort_flag, a.err, 301)
-                                         : wait_or_abort(&bars[B_OH0 + x], kt & 1, abort_flag, a.err, 304));
-                    if (!ok) break;
-                    tc_fence_after();
-                    scale_o(f);
-                }
-                const float2 nm2 = make_float2(-m, -m);
                 uint32_t pk[32];
+                float2 hs;
+                // P of the half against the row's current reference m. Its sum bounds every weight,
+                // so a sum within kRescaleBound shows that no key of the half exceeds m by more than
+                // the threshold and m stays: the half's maximum is not needed. Otherwise (rare after the
+                // first key tiles; always while m is -inf, whose sum is infinite) the half takes the
+                // maximum, raises m as before and computes P again. The weights are the same as
+                // with the maximum taken first.
+                auto weights = [&]() {
+                    const float2 nm2 = make_float2(-m, -m);
+                    hs = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
-                    const float2 p = (i & 15) < POLY ? exp2_poly2(e) : make_float2(fast_exp2(e.x), fast_exp2(e.y));
-                    pk[i] = pack2<T>(p.x, p.y);
-                    ps2 = __fadd2_rn(ps2, row_sum_term<T>(p, pk[i]));
+                    for (int i = 0; i < 32; ++i) {
+                        const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
+                        const float2 p = (i & 15) < POLY ? exp2_poly2(e) : make_float2(fast_exp2(e.x), fast_exp2(e.y));
+                        pk[i] = pack2<T>(p.x, p.y);
+                        hs = __fadd2_rn(hs, row_sum_term<T>(p, pk[i]));
+                    }
+                };
+                weights();
+                if (__any_sync(FULL_MASK, !(hs.x + hs.y <= kRescaleBound))) {
+                    float hm = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) hm = fmaxf(hm, sv[i]);
+                    hm *= a.scale_log2;
+                    const bool raise = hm > m + kRescaleThreshold;
+                    const float f = raise ? fast_exp2(m - hm) : 1.f;  // 0 while m is -inf
+                    if (raise) {
+                        ps2 = make_float2(ps2.x * f, ps2.y * f);
+                        alpha *= f;
+                        m = hm;
+                    }
+                    // The TMEM accesses are warp-collective: the whole warp takes this branch when
+                    // any of its rows raised, each lane scaling its own row by its own factor.
+                    if ((kt >= 1 || h == 1) && __any_sync(FULL_MASK, raise)) {
+                        ok = warp_all(h == 0 ? wait_or_abort(&bars[B_OF0 + x], (kt - 1) & 1, abort_flag, a.err, 301)
+                                             : wait_or_abort(&bars[B_OH0 + x], kt & 1, abort_flag, a.err, 304));
+                        if (!ok) break;
+                        tc_fence_after();
+                        scale_o(f);
+                    }
+                    weights();
                 }
+                ps2 = __fadd2_rn(ps2, hs);
                 tmem_st32(ts + h * 32, pk);
                 signal(h ? B_PF0 : B_PH0);
             }
@@ -666,9 +667,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (job == kJobExit) break;
             if (job >= 0) {
                 const TileCtx tile = tile_ctx(a, job);
+                uint64_t* tb = bars + *reinterpret_cast<volatile int*>(smem + OFF_BSET) * NUM_BARS;
                 if (tile.sane) {
-                    if (warp == 8) tile_producer(a, &tm_q, &tm_k, &tm_v, smem, bars, abort_flag, tile, lane);
-                    else if (warp == 9) tile_mma<T>(a, smem, bars, abort_flag, tmem, tile, lane);
+                    if (warp == 8) tile_producer(a, &tm_q, &tm_k, &tm_v, smem, tb, abort_flag, tile, lane);
+                    else if (warp == 9) tile_mma<T>(a, smem, tb, abort_flag, tmem, tile, lane);
                 }
             }
             tc_fence_before();
@@ -701,12 +703,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             cta_sync();                                   // (2)
         }
         // (b) tiles, longest first, while any is left.
+        int bset_seq = 1;   // thread 0: the barrier set of the last tile (tiles alternate between two)
         while (true) {
             if (threadIdx.x == 0) {
                 int t = kJobNone;
                 if (!*abort_flag && *reinterpret_cast<volatile int*>(&a.work[2]) < a.num_tiles) {
                     t = atomicAdd(&a.work[2], 1);
-                    if (t < a.num_tiles) init_tile_barriers(bars);
+                    if (t < a.num_tiles) {
+                        // Tiles alternate between two barrier sets, so a tile's barriers are armed
+                        // again only two tiles later. (With one set armed for every tile, batches
+                        // whose CTAs take several tiles met bounded-wait timeouts under some
+                        // schedules; the cause was not found.)
+                        bset_seq ^= 1;
+                        *reinterpret_cast<volatile int*>(smem + OFF_BSET) = bset_seq;
+                        init_tile_barriers(bars + bset_seq * NUM_BARS);
+                    }
                     else t = kJobNone;
                 }
                 *ctrl = t;
@@ -716,7 +727,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (job >= 0) {
                 tc_fence_after();
                 const TileCtx tile = tile_ctx(a, job);
-                if (tile.sane && (warp < 4 || tile.has_b)) tile_softmax<T, POLY>(a, smem, bars, abort_flag, tmem, tile, warp, lane);
+                uint64_t* tb = bars + *reinterpret_cast<volatile int*>(smem + OFF_BSET) * NUM_BARS;
+                if (tile.sane && (warp < 4 || tile.has_b)) tile_softmax<T, POLY>(a, smem, tb, abort_flag, tmem, tile, warp, lane);
             }
             tc_fence_before();
             cta_sync();                                   // (2)
