@@ -487,14 +487,12 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
         float alpha = 1.f;
         float2 ps2 = make_float2(0.f, 0.f);
         if (full && a.scale_log2 >= 0.f) {
-            // One TMEM round trip per half of the key tile: the half's maximum is taken in
-            // registers and P computed from the same registers against the row's reference m,
-            // raised first when the half exceeds it by more than the threshold. P of keys
-            // 64*h.. goes to columns 32*h.. (over S already read). A raise rescales what O holds
-            // against the old reference: PV(kt-1) before the first half (none when kt = 0), the
-            // first half's PV before the second.
+            // S in one TMEM round trip; then per half of 64 keys, P against the row's reference m
+            // (raised first, when needed, as below). P of keys 64*h.. goes to columns 32*h.. (over S
+            // already read) and is signalled per half. A raise rescales what O holds against the old
+            // reference: PV(kt-1) before the first half (none when kt = 0), the first half's PV
+            // before the second.
             const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-            // Both halves of S in one TMEM round trip.
             float sa[128];
             tmem_ld128_sync(ts, sa);
 #pragma unroll
@@ -549,18 +547,14 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
             }
             if (!ok) break;
         } else {
-            // pass 1: row maximum of scale * s over the visible keys
+            // S in one TMEM round trip; the row maximum of scale * s over the visible keys first.
+            float sa[128];
+            tmem_ld128_sync(ts, sa);
+            const int key0 = kt * 128;
             float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float sv[32];
-                tmem_ld32(ts + c * 32, sv);
-                tmem_wait_ld();
-                const int key0 = kt * 128 + c * 32;
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    mx = fmaxf(mx, (full || key0 + i < limit) ? sv[i] * a.scale_log2 : -INFINITY);
-            }
+            for (int i = 0; i < 128; ++i)
+                mx = fmaxf(mx, (full || key0 + i < limit) ? sa[i] * a.scale_log2 : -INFINITY);
             if (mx > m + kRescaleThreshold) {
                 alpha = fast_exp2(m - mx);  // 0 on the first tile
                 m = mx;
@@ -586,21 +580,19 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
                 }
                 fence_proxy_async_smem();
             }
-            // pass 2: p = 2^(s*scale - m), rounded to T, written over S as the A operand of PV.
-            // Chunk c's P goes to columns 16c.., which pass 2 has already read.
+            // p = 2^(s*scale - m), rounded to T, written over S (already in registers) as the A
+            // operand of PV, 32 keys at a time into columns 16c..
             const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
-#pragma unroll 1
+#pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float sv[32];
-                tmem_ld32(ts + c * 32, sv);
-                tmem_wait_ld();
+                const float* sv = sa + 32 * c;
                 uint32_t pk[16];
-                const int key0 = kt * 128 + c * 32;
+                const int kc = key0 + c * 32;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float2 e = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
-                    const float p0 = (full || key0 + 2 * i < limit) ? fast_exp2(e.x) : 0.f;
-                    const float p1 = (full || key0 + 2 * i + 1 < limit) ? fast_exp2(e.y) : 0.f;
+                    const float p0 = (full || kc + 2 * i < limit) ? fast_exp2(e.x) : 0.f;
+                    const float p1 = (full || kc + 2 * i + 1 < limit) ? fast_exp2(e.y) : 0.f;
                     pk[i] = pack2<T>(p0, p1);
                     ps2 = __fadd2_rn(ps2, row_sum_term<T>(make_float2(p0, p1), pk[i]));
                 }
