@@ -87,30 +87,31 @@ int tile_tokens(int group) { return 2 * (128 / group); }
 
 // CTAs of the tile kernel that should start on the split-K items of a mixed batch (0: run the two
 // kernels one after the other). Model, with rates measured on B200 for these kernels: a tile CTA
-// spends ~2.4 us per 128-key tile; an SM serving items streams their K/V at ~72 GB/s while the
-// others run tiles; once the tiles are done every SM serves items, ~6.6 TB/s together. For a few
-// candidate splits, the tiles (already longest first) are dealt to the other CTAs; the step ends
-// when the tiles end plus the time the items left over take on the whole GPU. The split with the
-// shortest estimate wins.
+// spends ~1.95 us per 128-key tile while items stream beside it; an SM serving items streams their
+// K/V at ~72 GB/s while the others run tiles; the items alone stream at ~6.6 TB/s on the whole GPU.
+// With nd SMs on items, the tiles end after T = max(tile work / (S - nd), longest tile); if the nd
+// SMs have not streamed every item by then, the rest runs on the whole GPU. Once they have, the
+// item CTAs turn to the tiles still unclaimed (the shortest, since tiles go longest first), so the
+// step ends near the balanced time (tile work + item work) / S. The smallest nd that reaches the
+// minimum wins -- the split where both queues end together; on the 70B-shaped mixed batch that is
+// 56 of 148 SMs, which measured best (52: +0.5 %, 60: +0.9 %, 48: +1.7 to 2.7 %).
 int mixed_split(const std::vector<PrefillTile>& tiles, int64_t item_bytes, int num_sms) {
-    constexpr double kKeyTileSec = 2.4e-6, kSmBytesPerSec = 72e9, kGpuBytesPerSec = 6.6e12;
-    static thread_local std::vector<double> load;
-    auto tiles_end = [&](int ctas) {  // longest first, dealt in a snake (a close stand-in for greedy)
-        load.assign((size_t)ctas, 0.0);
-        for (size_t i = 0; i < tiles.size(); ++i) {
-            const size_t r = i / ctas, k = i % ctas;
-            load[(r & 1) ? ctas - 1 - k : k] += tiles[i].key_tiles * kKeyTileSec;
-        }
-        return *std::max_element(load.begin(), load.end());
-    };
-    const double all_items = (double)item_bytes / kGpuBytesPerSec;
-    double best = tiles_end(num_sms) + all_items;  // one kernel after the other
-    int best_nd = 0;
-    for (int nd = 8; nd <= num_sms / 2; nd += 8) {
-        const double t = tiles_end(num_sms - nd);
-        const double left = std::max(0.0, (double)item_bytes - nd * kSmBytesPerSec * t);
-        const double est = t + left / kGpuBytesPerSec;
-        if (est < best) {
+    constexpr double kKeyTileSec = 1.95e-6, kSmBytesPerSec = 72e9, kGpuBytesPerSec = 6.6e12;
+    double tile_work = 0.0, longest = 0.0;
+    for (const PrefillTile& t : tiles) {
+        tile_work += t.key_tiles * kKeyTileSec;
+        longest = std::max(longest, t.key_tiles * kKeyTileSec);
+    }
+    const double item_work = (double)item_bytes / kSmBytesPerSec;  // SM-seconds on item-first SMs
+    const double balanced = std::max((tile_work + item_work) / num_sms, longest);
+    double best = std::max(tile_work / num_sms, longest) + (double)item_bytes / kGpuBytesPerSec;
+    int best_nd = 0;  // one kernel after the other
+    for (int nd = 1; nd < num_sms; ++nd) {
+        const double t = std::max(tile_work / (num_sms - nd), longest);
+        const double streamed = nd * kSmBytesPerSec * t;
+        const double est = streamed >= (double)item_bytes ? std::max(balanced, item_work / nd)
+                                                          : t + ((double)item_bytes - streamed) / kGpuBytesPerSec;
+        if (est < best * (1.0 - 1e-9)) {
             best = est;
             best_nd = nd;
         }
