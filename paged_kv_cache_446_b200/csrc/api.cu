@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -85,32 +86,75 @@ PlanLists& thread_lists() {
 // Query rows per tcgen05 CTA: two 128-row MMA tiles, each (128 / G) consecutive query rows x G heads.
 int tile_tokens(int group) { return 2 * (128 / group); }
 
+// When the last tile ends if the tiles (longest first, as the ticket counter hands them out) each
+// go to the CTA that frees first: `ctas` CTAs, `late` of which free only at t_late. Durations and
+// loads are whole ticks. Tiles of equal length form runs (ticks, count) and CTAs of equal load form
+// groups (load -> count), so a run is dealt to whole groups at once and the cost grows with the
+// distinct lengths and loads, not with the tiles.
+int64_t greedy_end(const std::vector<std::pair<int64_t, int>>& runs, int ctas, int late, int64_t t_late,
+                   std::map<int64_t, int>& load) {
+    load.clear();
+    if (ctas > late) load[0] += ctas - late;
+    if (late > 0) load[t_late] += late;
+    int64_t end = late > 0 ? t_late : 0;
+    for (const auto& run : runs) {
+        for (int n = run.second; n > 0;) {
+            auto g = load.begin();
+            const int64_t l = g->first;
+            const int k = std::min(g->second, n);
+            n -= k;
+            if ((g->second -= k) == 0) load.erase(g);
+            load[l + run.first] += k;
+            end = std::max(end, l + run.first);
+        }
+    }
+    return end;
+}
+
 // CTAs of the tile kernel that should start on the split-K items of a mixed batch (0: run the two
 // kernels one after the other). Model, with rates measured on B200 for these kernels: a tile CTA
 // spends ~1.95 us per 128-key tile while items stream beside it; an SM serving items streams their
-// K/V at ~72 GB/s while the others run tiles; the items alone stream at ~6.6 TB/s on the whole GPU.
-// With nd SMs on items, the tiles end after T = max(tile work / (S - nd), longest tile); if the nd
-// SMs have not streamed every item by then, the rest runs on the whole GPU. Once they have, the
-// item CTAs turn to the tiles still unclaimed (the shortest, since tiles go longest first), so the
-// step ends near the balanced time (tile work + item work) / S. The smallest nd that reaches the
-// minimum wins -- the split where both queues end together; on the 70B-shaped mixed batch that is
-// 56 of 148 SMs, which measured best (52: +0.5 %, 60: +0.9 %, 48: +1.7 to 2.7 %).
-int mixed_split(const std::vector<PrefillTile>& tiles, int64_t item_bytes, int num_sms) {
-    constexpr double kKeyTileSec = 1.95e-6, kSmBytesPerSec = 72e9, kGpuBytesPerSec = 6.6e12;
-    double tile_work = 0.0, longest = 0.0;
+// K/V at ~85 GB/s while the others run tiles; the items alone stream at ~6.6 TB/s on the whole GPU.
+// With nd SMs on items, the tiles are dealt greedily to the other S - nd CTAs (greedy_end: long
+// tiles come in few sizes, so the step's length moves in steps as nd changes, not smoothly). If the
+// nd SMs have not streamed every item when the tiles end, the rest runs on the whole GPU and the
+// step ends about half an item later than the bytes alone say (each of the S x 8 warps finishes
+// its last item at its own time). If they have, they turn to the tiles still unclaimed, which the
+// greedy schedule models as nd CTAs freeing late. Candidates near the balanced share (both queues
+// ending together) are simulated and the shortest estimate wins. On the 70B-shaped mixed batch
+// this picks 52 of 148 SMs, which measured best (128 tiles of ~500 us and 128 of ~250 us pack
+// evenly onto 96 tile CTAs; 50: +1.9 %, 53: +3.2 %).
+int mixed_split(const std::vector<PrefillTile>& tiles, int64_t item_bytes, int64_t num_items, int num_sms) {
+    constexpr double kKeyTileSec = 1.95e-6, kSmBytesPerSec = 85e9, kGpuBytesPerSec = 6.6e12;
+    if (tiles.empty() || num_items <= 0) return 0;
+    static thread_local std::vector<std::pair<int64_t, int>> runs;
+    static thread_local std::map<int64_t, int> load;
+    // Ticks of 1/96 of the longest tile: coarse enough that equal loads recur (the simulation then
+    // adds ~10 % to the planner's time on that batch), fine enough that a CTA's few tiles add up to
+    // within ~1 % (at 1/64 the choice there moved to 50).
+    int max_kt = 1;
+    for (const PrefillTile& t : tiles) max_kt = std::max(max_kt, t.key_tiles);
+    const double tick = max_kt * kKeyTileSec / 96.0;
+    runs.clear();
+    double tile_work = 0.0;
     for (const PrefillTile& t : tiles) {
-        tile_work += t.key_tiles * kKeyTileSec;
-        longest = std::max(longest, t.key_tiles * kKeyTileSec);
+        const int64_t d = std::max<int64_t>(1, std::llround(t.key_tiles * kKeyTileSec / tick));
+        tile_work += d * tick;
+        if (!runs.empty() && runs.back().first == d) ++runs.back().second;
+        else runs.push_back({d, 1});
     }
-    const double item_work = (double)item_bytes / kSmBytesPerSec;  // SM-seconds on item-first SMs
-    const double balanced = std::max((tile_work + item_work) / num_sms, longest);
-    double best = std::max(tile_work / num_sms, longest) + (double)item_bytes / kGpuBytesPerSec;
+    const double items = (double)item_bytes;
+    const double item_work = items / kSmBytesPerSec;  // SM-seconds on item-first SMs
+    const double tail = 0.5 * (items / num_items) * (num_sms * 8.0) / kGpuBytesPerSec;
+    double best = greedy_end(runs, num_sms, 0, 0, load) * tick + items / kGpuBytesPerSec;
     int best_nd = 0;  // one kernel after the other
-    for (int nd = 1; nd < num_sms; ++nd) {
-        const double t = std::max(tile_work / (num_sms - nd), longest);
+    const int bal = (int)std::lround(num_sms * item_work / std::max(tile_work + item_work, 1e-30));
+    for (int nd = std::max(1, bal - 12); nd <= std::min(num_sms - 1, bal + 4); ++nd) {
+        const double t = greedy_end(runs, num_sms - nd, 0, 0, load) * tick;
         const double streamed = nd * kSmBytesPerSec * t;
-        const double est = streamed >= (double)item_bytes ? std::max(balanced, item_work / nd)
-                                                          : t + ((double)item_bytes - streamed) / kGpuBytesPerSec;
+        const double est =
+            streamed >= items ? greedy_end(runs, num_sms, nd, std::llround(item_work / nd / tick), load) * tick
+                              : t + (items - streamed) / kGpuBytesPerSec + tail;
         if (est < best * (1.0 - 1e-9)) {
             best = est;
             best_nd = nd;
@@ -453,7 +497,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->decode_sms = 0;
     if (o.decode_sms >= 0 && kind == 2 && n_items > 0 && !L->tiles.empty() && num_sms >= 2) {
         int nd = o.decode_sms;
-        if (nd == 0) nd = mixed_split(L->tiles, plan->core_kv_bytes, num_sms);
+        if (nd == 0) nd = mixed_split(L->tiles, plan->core_kv_bytes, (int64_t)n_items, num_sms);
         if (nd > 0) plan->decode_sms = std::min(nd, num_sms - 1);
     }
     return PKV_OK;

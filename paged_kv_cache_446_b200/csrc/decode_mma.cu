@@ -15,8 +15,8 @@
 // persistent worker with its own copy ring, as in decode.cu, and needs no tensor memory or
 // CTA-wide synchronisation.
 //
-// Per warp and block: K and V of one (block, KV head) -- 16 rows of 128 elements -- arrive by two
-// tensor-map TMA copies each (64-column halves, 128-byte swizzle, so ldmatrix reads are free of
+// Per warp and block: K and V of one (block, KV head) -- 16 rows of 128 elements -- arrive by one
+// tensor-map TMA copy each (both 64-column halves, 128-byte swizzle, so ldmatrix reads are free of
 // bank conflicts) into a ring of shared-memory stages tracked by mbarriers; the item's q rows come
 // once by plain bulk copies. S = Q K^T as 16 MMAs (two 8-token n-tiles x 8 k-steps); the online
 // softmax runs on the accumulator fragments in the log2 domain (a slot's scores sit in one lane
@@ -73,11 +73,8 @@ cudaError_t launch_mma_t(const DecodeArgs& a, int num_sms, cudaStream_t s) {
     const CUtensorMapDataType dt =
         std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const long long rows = (long long)a.num_blocks * a.num_kv_heads * kBlockSize;
-    const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {128 * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)kBlockSize};
     CUtensorMap mk, mv;
-    if (!encode_tiled(&mk, dt, 2, a.k_pool, dims, strides, box) || !encode_tiled(&mv, dt, 2, a.v_pool, dims, strides, box))
+    if (!encode_block_halves(&mk, dt, a.k_pool, rows) || !encode_block_halves(&mv, dt, a.v_pool, rows))
         return cudaErrorInvalidValue;
     constexpr int smem = smem_bytes<NSTAGE>();
     static int per_sm_cache[64] = {0};

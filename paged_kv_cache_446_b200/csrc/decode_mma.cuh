@@ -17,9 +17,10 @@
 // persistent worker with its own copy ring, as in decode.cu, and needs no tensor memory or
 // CTA-wide synchronisation.
 //
-// Per warp and block: K and V of one (block, KV head) -- 16 rows of 128 elements -- arrive by two
-// tensor-map TMA copies each (64-column halves, 128-byte swizzle, so ldmatrix reads are free of
-// bank conflicts) into a ring of shared-memory stages tracked by mbarriers; the item's q rows come
+// Per warp and block: K and V of one (block, KV head) -- 16 rows of 128 elements -- arrive by one
+// tensor-map TMA copy each (both 64-column halves through a 3-D view of the pool, 128-byte
+// swizzle, so ldmatrix reads are free of bank conflicts; the copies' issue is a large share of a
+// warp's time per block, so one copy per operand rather than one per half) into a ring of shared-memory stages tracked by mbarriers; the item's q rows come
 // once by plain bulk copies. S = Q K^T as 16 MMAs (two 8-token n-tiles x 8 k-steps); the online
 // softmax runs on the accumulator fragments in the log2 domain (a slot's scores sit in one lane
 // quad); P, rounded to the input type, is reused in registers as the A operand of P V (16 MMAs
@@ -44,6 +45,16 @@ constexpr int kKV = 4 * kHalf;                 // K half 0, K half 1, V half 0, 
 constexpr int kQ = kSlots * 256;               // an item's q rows (256 bytes each)
 constexpr int kStage = kKV + kQ;               // 12 KiB, a multiple of the 1 KiB swizzle atom
 constexpr int kFifo = 8;                       // items a warp's producer may run ahead (> NSTAGE)
+
+// K or V of one KV block (16 pool rows from row y) in one copy, both 64-column halves, through a
+// map made by encode_block_halves.
+__device__ __forceinline__ void tma_load_block(void* dst, const CUtensorMap* map, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(0), "r"(smem_u32(bar))
+        : "memory");
+}
 
 // Byte offset, inside a 16-row chunk stored as two 64-column halves with the 128-byte swizzle, of
 // the 16 bytes holding columns [8 * col8, 8 * col8 + 8) of row r (col8 in 0..15).
@@ -116,7 +127,13 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
     DecodeItem pi = load_item(a.items, p_it);
     int p_blk = pi.blk_begin;
     int p_base = p_blk;
-    int p_ids = (p_blk + lane < pi.blk_end) ? __ldg(a.block_tables + (size_t)pi.req * a.max_blocks_per_seq + p_blk + lane) : 0;
+    // Block ids of the producer's item, 32 at a time: p_ids holds those from p_base on (lane l:
+    // block p_base + l), p_nxt the next 32, loaded a window ahead so that their latency hides.
+    auto ids_at = [&](int from) {
+        return (from + lane < pi.blk_end) ? __ldg(a.block_tables + (size_t)pi.req * a.max_blocks_per_seq + from + lane) : 0;
+    };
+    int p_ids = ids_at(p_blk);
+    int p_nxt = ids_at(p_blk + 32);
     int ticket = 0;                      // lane 0: the next item's ticket, fetched ahead
     if (lane == 0) {
         ticket = atomicAdd(&a.work[0], 1);
@@ -141,10 +158,8 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
             const uint32_t qbytes = first ? qrow * (uint32_t)pi.num_rows : 0u;
             mbar_arrive_expect_tx(&bars[stage], (uint32_t)kKV + qbytes);
             const int y = (id * a.num_kv_heads + pi.kv_head) * kBlockSize;  // first pool row of the chunk
-            tma_load_2d(st, tm_k, 0, y, &bars[stage]);
-            tma_load_2d(st + kHalf, tm_k, 64, y, &bars[stage]);
-            tma_load_2d(st + 2 * kHalf, tm_v, 0, y, &bars[stage]);
-            tma_load_2d(st + 3 * kHalf, tm_v, 64, y, &bars[stage]);
+            tma_load_block(st, tm_k, y, &bars[stage]);
+            tma_load_block(st + 2 * kHalf, tm_v, y, &bars[stage]);
             if (first) {
                 for (int j = 0; j < pi.num_rows; ++j) {
                     const size_t qoff =
@@ -161,8 +176,8 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
                 pi = load_item(a.items, p_it);
                 p_blk = pi.blk_begin;
                 p_base = p_blk;
-                p_ids = (p_blk + lane < pi.blk_end)
-                            ? __ldg(a.block_tables + (size_t)pi.req * a.max_blocks_per_seq + p_blk + lane) : 0;
+                p_ids = ids_at(p_blk);
+                p_nxt = ids_at(p_blk + 32);
                 if (lane == 0) {
                     fifo[pushed % kFifo] = p_it;
                     ticket = atomicAdd(&a.work[0], 1);
@@ -173,8 +188,8 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
             }
         } else if (p_blk - p_base == 32) {
             p_base = p_blk;
-            p_ids = (p_blk + lane < pi.blk_end)
-                        ? __ldg(a.block_tables + (size_t)pi.req * a.max_blocks_per_seq + p_blk + lane) : 0;
+            p_ids = p_nxt;
+            p_nxt = ids_at(p_blk + 32);
         }
     };
 
@@ -203,6 +218,7 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
         float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
         int lima = 0, limb = 0, nh = 1, ns = 0;
         const int sa = 2 * c4, sb = 2 * c4 + 1;   // this lane's slots
+        bool zeroed = false;                      // V rows of the current stage were zeroed
 
         while (true) {
             const int stage = consumed % NSTAGE;
@@ -292,6 +308,7 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
                     *reinterpret_cast<uint4*>(st + 2 * kHalf + sw_off(r, idx & 15)) = make_uint4(0u, 0u, 0u, 0u);
                 }
                 __syncwarp();
+                zeroed = true;
             }
 
             // ---- O^T += V^T P^T: eight 16-row m-tiles of head_dim ----
@@ -305,11 +322,14 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
             __syncwarp();
             ++consumed;
 
-            // Refill this stage with the producer's next block.
+            // Refill this stage with the producer's next block. The warp's reads of the stage are
+            // complete (their values are in registers); generic writes to it (zeroed V rows) are
+            // ordered before the copy's writes by a proxy fence.
             if (!p_done) {
-                fence_proxy_async_smem();
+                if (zeroed) fence_proxy_async_smem();
                 issue(stage);
             }
+            zeroed = false;
 
             if (c_blk + 1 == ci.blk_end) {
                 // ---- item done: normalised output, or the chunk's partial ----
@@ -364,6 +384,7 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
         float o[16][4];                // O accumulators, one per 8-column n-tile
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         int lim0 = 0, lim1 = 0, nh = 1, ns = 0;
+        bool zeroed = false;                      // V rows of the current stage were zeroed
 
         while (true) {
             const int stage = consumed % NSTAGE;
@@ -477,6 +498,7 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
                     *reinterpret_cast<uint4*>(st + 2 * kHalf + sw_off(r, idx & 15)) = make_uint4(0u, 0u, 0u, 0u);
                 }
                 __syncwarp();
+                zeroed = true;
             }
 
             // ---- O += P V: sixteen 8-column n-tiles ----
@@ -490,11 +512,14 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
             __syncwarp();
             ++consumed;
 
-            // Refill this stage with the producer's next block.
+            // Refill this stage with the producer's next block. The warp's reads of the stage are
+            // complete (their values are in registers); generic writes to it (zeroed V rows) are
+            // ordered before the copy's writes by a proxy fence.
             if (!p_done) {
-                fence_proxy_async_smem();
+                if (zeroed) fence_proxy_async_smem();
                 issue(stage);
             }
+            zeroed = false;
 
             if (c_blk + 1 == ci.blk_end) {
                 // ---- item done: normalised output, or the chunk's partial ----

@@ -643,7 +643,8 @@ constexpr int kJobNone = -3;    // nothing in this step
 template <typename T, int POLY, int DEC>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const PrefillArgs a, const DecodeArgs d, const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_kb, const __grid_constant__ CUtensorMap tm_vb) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -693,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             first = __shfl_sync(FULL_MASK, first, 0);
             uint64_t* dbars = reinterpret_cast<uint64_t*>(smem + OFF_DBAR) + warp * kDecodeStages;
             volatile int* fifo = reinterpret_cast<volatile int*>(smem + OFF_FIFO) + warp * mma::kFifo;
-            if (!mma::decode_warp<T, kDecodeStages, DEC == 2>(d, &tm_k, &tm_v, smem + warp * kDecodeStages * mma::kStage,
+            if (!mma::decode_warp<T, kDecodeStages, DEC == 2>(d, &tm_kb, &tm_vb, smem + warp * kDecodeStages * mma::kStage,
                                                                dbars, fifo, first, 0) &&
                 lane == 0)
                 *abort_flag = 1;
@@ -780,10 +781,12 @@ cudaError_t launch_t(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cud
     const cuuint64_t kdims[2] = {128, (cuuint64_t)rows};
     const cuuint64_t kstr[1] = {128 * 2};
     const cuuint32_t kbox[2] = {64, (cuuint32_t)kBlockSize};
-    // One map over the pool rows serves the tiles (8 blocks per key tile) and the split-K items
-    // (one block per stage): the same 64-column x 16-row box with the 128-byte swizzle.
+    // The tiles read the pool rows through a 64-column x 16-row box (8 blocks per key tile, two
+    // halves each); the split-K items through the block-halves view (one copy per block).
+    CUtensorMap mkb, mvb;
     if (!encode_tiled(&mq, dt, 3, a.q, qdims, qstr, qbox) || !encode_tiled(&mk, dt, 2, a.k_pool, kdims, kstr, kbox) ||
-        !encode_tiled(&mv, dt, 2, a.v_pool, kdims, kstr, kbox))
+        !encode_tiled(&mv, dt, 2, a.v_pool, kdims, kstr, kbox) || !encode_block_halves(&mkb, dt, a.k_pool, rows) ||
+        !encode_block_halves(&mvb, dt, a.v_pool, rows))
         return cudaErrorInvalidValue;
     static int configured[64] = {0};
     int dev = 0;
@@ -799,7 +802,7 @@ cudaError_t launch_t(const PrefillArgs& a, const DecodeArgs& d, int num_sms, cud
     int grid = num_sms;
     if (d.num_items <= 0 && a.num_tiles < grid) grid = a.num_tiles;
     return launch_k(a.pdl, prefill_tc_kernel<T, POLY, DEC>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, a, d, mq, mk,
-                    mv);
+                    mv, mkb, mvb);
 }
 
 // Batches with tcgen05 tiles only run an instantiation without the split-K rounds (fewer registers

@@ -34,4 +34,11 @@ bool encode_tiled(CUtensorMap* m, CUtensorMapDataType t, int rank, const void* b
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_block_halves(CUtensorMap* m, CUtensorMapDataType t, const void* base, long long rows) {
+    const cuuint64_t dims[3] = {64, (cuuint64_t)rows, 2};
+    const cuuint64_t strides[2] = {128 * 2, 64 * 2};
+    const cuuint32_t box[3] = {64, 16, 2};
+    return encode_tiled(m, t, 3, base, dims, strides, box);
+}
+
 }  // namespace pkv
