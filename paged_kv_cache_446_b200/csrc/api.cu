@@ -114,18 +114,26 @@ int64_t greedy_end(const std::vector<std::pair<int64_t, int>>& runs, int ctas, i
 // CTAs of the tile kernel that should start on the split-K items of a mixed batch (0: run the two
 // kernels one after the other). Model, with rates measured on B200 for these kernels: a tile CTA
 // spends ~1.95 us per 128-key tile while items stream beside it; an SM serving items streams their
-// K/V at ~85 GB/s while the others run tiles; the items alone stream at ~6.6 TB/s on the whole GPU.
+// K/V at ~115 GB/s while the others run tiles (items of at most 8 (row, head) slots, on all twelve
+// warps; ~85 GB/s for items of up to 16 slots, on eight); the items alone stream at ~6.6 TB/s on
+// the whole GPU.
 // With nd SMs on items, the tiles are dealt greedily to the other S - nd CTAs (greedy_end: long
 // tiles come in few sizes, so the step's length moves in steps as nd changes, not smoothly). If the
 // nd SMs have not streamed every item when the tiles end, the rest runs on the whole GPU and the
-// step ends about half an item later than the bytes alone say (each of the S x 8 warps finishes
-// its last item at its own time). If they have, they turn to the tiles still unclaimed, which the
+// step ends about half an item later than the bytes alone say (each of the S x 12 (or 8) item
+// warps finishes its last item at its own time). If they have, they turn to the tiles still unclaimed, which the
 // greedy schedule models as nd CTAs freeing late. Candidates near the balanced share (both queues
-// ending together) are simulated and the shortest estimate wins. On the 70B-shaped mixed batch
-// this picks 52 of 148 SMs, which measured best (128 tiles of ~500 us and 128 of ~250 us pack
-// evenly onto 96 tile CTAs; 50: +1.9 %, 53: +3.2 %).
-int mixed_split(const std::vector<PrefillTile>& tiles, int64_t item_bytes, int64_t num_items, int num_sms) {
-    constexpr double kKeyTileSec = 1.95e-6, kSmBytesPerSec = 85e9, kGpuBytesPerSec = 6.6e12;
+// ending together) are simulated. Past the share the estimate is flat (the items end first and
+// the tiles set the step) and just below it the step grows fast, so the pick is the middle of the
+// run of candidates within 0.3 % of the best, not its low end. The step length moves in steps:
+// on the 70B-shaped mixed batch with eight item warps per SM, 52 item SMs measured 1.209 ms and 53
+// measured 1.247 ms (128 tiles of ~500 us and 128 of ~250 us pack evenly onto 96 tile CTAs, not
+// onto 95); with twelve, 44-52 measured within 0.4 % of each other and 40 2 % slower.
+int mixed_split(const std::vector<PrefillTile>& tiles, int64_t item_bytes, int64_t num_items, int item_slots,
+                int num_sms) {
+    constexpr double kKeyTileSec = 1.95e-6, kGpuBytesPerSec = 6.6e12;
+    const double kSmBytesPerSec = item_slots <= 8 ? 115e9 : 85e9;
+    const double warps_per_sm = item_slots <= 8 ? 12.0 : 8.0;
     if (tiles.empty() || num_items <= 0) return 0;
     static thread_local std::vector<std::pair<int64_t, int>> runs;
     static thread_local std::map<int64_t, int> load;
@@ -145,22 +153,35 @@ int mixed_split(const std::vector<PrefillTile>& tiles, int64_t item_bytes, int64
     }
     const double items = (double)item_bytes;
     const double item_work = items / kSmBytesPerSec;  // SM-seconds on item-first SMs
-    const double tail = 0.5 * (items / num_items) * (num_sms * 8.0) / kGpuBytesPerSec;
-    double best = greedy_end(runs, num_sms, 0, 0, load) * tick + items / kGpuBytesPerSec;
-    int best_nd = 0;  // one kernel after the other
+    const double tail = 0.5 * (items / num_items) * (num_sms * warps_per_sm) / kGpuBytesPerSec;
+    const double serial = greedy_end(runs, num_sms, 0, 0, load) * tick + items / kGpuBytesPerSec;
     const int bal = (int)std::lround(num_sms * item_work / std::max(tile_work + item_work, 1e-30));
-    for (int nd = std::max(1, bal - 12); nd <= std::min(num_sms - 1, bal + 4); ++nd) {
+    const int lo = std::max(1, bal - 12), hi = std::min(num_sms - 1, bal + 12);
+    static thread_local std::vector<double> est;
+    est.assign((size_t)std::max(hi - lo + 1, 0), 0.0);
+    double best = serial;
+    for (int nd = lo; nd <= hi; ++nd) {
         const double t = greedy_end(runs, num_sms - nd, 0, 0, load) * tick;
         const double streamed = nd * kSmBytesPerSec * t;
-        const double est =
-            streamed >= items ? greedy_end(runs, num_sms, nd, std::llround(item_work / nd / tick), load) * tick
-                              : t + (items - streamed) / kGpuBytesPerSec + tail;
-        if (est < best * (1.0 - 1e-9)) {
-            best = est;
-            best_nd = nd;
+        est[nd - lo] = streamed >= items ? greedy_end(runs, num_sms, nd, std::llround(item_work / nd / tick), load) * tick
+                                         : t + (items - streamed) / kGpuBytesPerSec + tail;
+        best = std::min(best, est[nd - lo]);
+    }
+    if (best >= serial) return 0;  // one kernel after the other
+    // The middle of the longest run of candidates within 0.3 % of the best.
+    int run_lo = -1, best_lo = lo, best_len = 0;
+    for (int nd = lo; nd <= hi + 1; ++nd) {
+        const bool near = nd <= hi && est[nd - lo] <= best * 1.003;
+        if (near && run_lo < 0) run_lo = nd;
+        if (!near && run_lo >= 0) {
+            if (nd - run_lo > best_len) {
+                best_len = nd - run_lo;
+                best_lo = run_lo;
+            }
+            run_lo = -1;
         }
     }
-    return best_nd;
+    return best_lo + (best_len - 1) / 2;
 }
 
 // out_meta / out_cap: when given and large enough, the work lists are written straight into that
@@ -497,7 +518,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->decode_sms = 0;
     if (o.decode_sms >= 0 && kind == 2 && n_items > 0 && !L->tiles.empty() && num_sms >= 2) {
         int nd = o.decode_sms;
-        if (nd == 0) nd = mixed_split(L->tiles, plan->core_kv_bytes, (int64_t)n_items, num_sms);
+        if (nd == 0) nd = mixed_split(L->tiles, plan->core_kv_bytes, (int64_t)n_items, max_slots, num_sms);
         if (nd > 0) plan->decode_sms = std::min(nd, num_sms - 1);
     }
     return PKV_OK;

@@ -109,10 +109,15 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 // here (they must be idle); fifo: kFifo ints of shared memory (the items the producer has started,
 // in order, for the consumer). On return every copy the warp issued has landed. Returns false when
 // a bounded wait expired (recorded in the device error word; the warp's copies then drained).
-template <typename T, int NSTAGE, bool T8>
+// QREG (transposed form only): the stages hold K/V alone (kKV bytes each) and the item's q rows go
+// from global memory straight into the B fragments -- for the next item as soon as the producer
+// starts it, so the load's latency hides behind the blocks still ahead of the consumer.
+template <typename T, int NSTAGE, bool T8, bool QREG = false>
 __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                             unsigned char* wbase, uint64_t* bars, volatile int* fifo, int first,
                                             int base) {
+    static_assert(!QREG || T8, "q rows in registers: the transposed form only");
+    constexpr int kSt = QREG ? kKV : kStage;   // bytes per stage
     const int lane = threadIdx.x & 31;
     if (lane == 0) {
         for (int s = 0; s < NSTAGE; ++s) mbar_init(&bars[s], 1);
@@ -121,6 +126,24 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
     __syncwarp();
     if (first >= a.num_items) return true;
     const unsigned char* qp = static_cast<const unsigned char*>(a.q);
+    const int g = lane >> 2;       // fragment row
+    const int c4 = lane & 3;       // fragment column pair
+    // QREG: item it's q rows as this lane's B fragments (slot g, words kk * 8 + c4 and + 4; zero
+    // past the item's slots).
+    auto load_q = [&](const DecodeItem& it, uint32_t (&qf)[8][2]) {
+        const int nh = min(a.heads_per_item, a.group - it.head0);
+        const bool vq = g < nh * it.num_rows;
+        const int jr = vq ? g / nh : 0;
+        const uint32_t* qg = reinterpret_cast<const uint32_t*>(
+            qp + ((size_t)(it.row + jr) * a.num_q_heads + (size_t)it.kv_head * a.group + it.head0 + (vq ? g - jr * nh : 0)) * 256);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            qf[kk][0] = vq ? __ldg(qg + kk * 8 + c4) : 0u;
+            qf[kk][1] = vq ? __ldg(qg + kk * 8 + 4 + c4) : 0u;
+        }
+    };
+    [[maybe_unused]] uint32_t qn[8][2];   // QREG: the q fragments of item qn_item, loaded ahead
+    [[maybe_unused]] int qn_item = -1;
 
     // ---------------- producer (lane 0 issues; runs up to NSTAGE blocks ahead) ----------------
     int p_it = first;
@@ -151,8 +174,8 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
                 record_error(a.err, 6 /*PKV_ERR_DEVICE_RANGE*/, (long long)pi.req * a.max_blocks_per_seq + p_blk);
                 id = 0;
             }
-            unsigned char* st = wbase + stage * kStage;
-            const bool first = (p_blk == pi.blk_begin);
+            unsigned char* st = wbase + stage * kSt;
+            const bool first = !QREG && (p_blk == pi.blk_begin);
             const int nh = min(a.heads_per_item, a.group - pi.head0);
             const uint32_t qrow = (uint32_t)(nh * 256);
             const uint32_t qbytes = first ? qrow * (uint32_t)pi.num_rows : 0u;
@@ -178,6 +201,10 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
                 p_base = p_blk;
                 p_ids = ids_at(p_blk);
                 p_nxt = ids_at(p_blk + 32);
+                if constexpr (QREG) {
+                    load_q(pi, qn);
+                    qn_item = p_it;
+                }
                 if (lane == 0) {
                     fifo[pushed % kFifo] = p_it;
                     ticket = atomicAdd(&a.work[0], 1);
@@ -202,8 +229,6 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
     int c_blk = ci.blk_begin;
     uint32_t consumed = 0;
 
-    const int g = lane >> 2;       // fragment row
-    const int c4 = lane & 3;       // fragment column pair
     const int mi = lane >> 3;      // ldmatrix: which 8x8 matrix this lane addresses
     const int mr = lane & 7;       //           and which of its rows
 
@@ -228,19 +253,31 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
                 for (uint32_t k = consumed; k < issued; ++k) (void)mbar_wait(&bars[k % NSTAGE], (k / NSTAGE) & 1u);
                 return false;
             }
-            unsigned char* st = wbase + stage * kStage;
+            unsigned char* st = wbase + stage * kSt;
             const uint32_t kb = smem_u32(st);
             const uint32_t vb = kb + 2 * kHalf;
 
             if (c_blk == ci.blk_begin) {
                 nh = min(a.heads_per_item, a.group - ci.head0);
                 ns = nh * ci.num_rows;
-                const uint32_t* qs = reinterpret_cast<const uint32_t*>(st + kKV);
-                const bool vq = g < ns;
+                if constexpr (QREG) {
+                    if (qn_item == c_it) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    qb[kk][0] = vq ? qs[g * 64 + kk * 8 + c4] : 0u;
-                    qb[kk][1] = vq ? qs[g * 64 + kk * 8 + 4 + c4] : 0u;
+                        for (int kk = 0; kk < 8; ++kk) {
+                            qb[kk][0] = qn[kk][0];
+                            qb[kk][1] = qn[kk][1];
+                        }
+                    } else {
+                        load_q(ci, qb);
+                    }
+                } else {
+                    const uint32_t* qs = reinterpret_cast<const uint32_t*>(st + kKV);
+                    const bool vq = g < ns;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        qb[kk][0] = vq ? qs[g * 64 + kk * 8 + c4] : 0u;
+                        qb[kk][1] = vq ? qs[g * 64 + kk * 8 + 4 + c4] : 0u;
+                    }
                 }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) ot[j][0] = ot[j][1] = ot[j][2] = ot[j][3] = 0.f;
@@ -394,7 +431,7 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
                 for (uint32_t k = consumed; k < issued; ++k) (void)mbar_wait(&bars[k % NSTAGE], (k / NSTAGE) & 1u);
                 return false;
             }
-            unsigned char* st = wbase + stage * kStage;
+            unsigned char* st = wbase + stage * kSt;
             const uint32_t kb = smem_u32(st);
             const uint32_t vb = kb + 2 * kHalf;
 

@@ -55,6 +55,10 @@ constexpr int kThreads = 384;
 // the shrinking one releases. ptxas fits both regions without spilling at these counts.
 constexpr int kSoftmaxRegs = 216;
 constexpr int kOtherRegs = 72;
+// Rounds of split-K items of at most 8 (row, head) slots run on all twelve warps, each at 168.
+constexpr int kItemRegs = 168;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs == kThreads * 168 && kItemRegs == 168,
+              "register split: every split must add up to the launch's registers");
 constexpr int kHalf = 128 * 128;        // 128 rows x 64 elements x 2 bytes
 constexpr int kTile = 2 * kHalf;        // 128 x 128 x 2 bytes
 constexpr int OFF_Q = 0;                // Q_A, Q_B
@@ -70,14 +74,24 @@ constexpr int OFF_TMEM = OFF_BAR + 2 * NUM_BARS * 8; // tcgen05.alloc result (af
 constexpr int OFF_BSET = OFF_TMEM + 12;              // the current tile's barrier set (thread 0 writes it)
 constexpr int OFF_ABORT = OFF_TMEM + 4;
 constexpr int OFF_CTRL = OFF_ABORT + 4;              // the CTA's next step (thread 0 writes it)
-// Rounds of split-K items: warps 0-7 each use kDecodeStages stages of the tile buffers (8 x 2 x 12 KiB
-// = 192 KiB, below OFF_BAR), with their own mbarriers and item rings after the tile barriers.
+// Rounds of split-K items take kDecodeStages stages per warp from the tile buffers, with their own
+// mbarriers and item rings after the tile barriers. An SM serving items is bound by its warps'
+// instruction issue, not by bytes in flight (4 warps stream half what 8 do; a third stage per warp
+// adds nothing), so items of at most 8 (row, head) slots -- the transposed form -- run on all 12
+// warps with K/V-only stages (12 x 2 x 8 KiB = 192 KiB) and q rows in registers; items of up to 16
+// slots on warps 0-7 with q staged beside K/V (8 x 2 x 12 KiB).
 constexpr int kDecodeStages = 2;
+template <int DEC> struct ItemRound {
+    static constexpr bool kQreg = DEC == 2;
+    static constexpr int kWarps = DEC == 2 ? 12 : 8;
+    static constexpr int kStageBytes = DEC == 2 ? mma::kKV : mma::kStage;
+    static_assert(kWarps * kDecodeStages * kStageBytes <= OFF_BAR, "split-K stages overlap the tile barriers");
+};
+constexpr int kMaxItemWarps = 12;
 constexpr int OFF_DBAR = OFF_TMEM + 16;
-constexpr int OFF_FIFO = OFF_DBAR + 8 * kDecodeStages * 8;
-constexpr int SMEM_USED = OFF_FIFO + 8 * mma::kFifo * 4;
+constexpr int OFF_FIFO = OFF_DBAR + kMaxItemWarps * kDecodeStages * 8;
+constexpr int SMEM_USED = OFF_FIFO + kMaxItemWarps * mma::kFifo * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;         // slack to align the base to 1024 bytes
-static_assert(8 * kDecodeStages * mma::kStage <= OFF_BAR, "split-K stages overlap the tile barriers");
 static_assert(OFF_DBAR % 8 == 0, "mbarrier alignment");
 constexpr uint32_t kTmemCols = 512;                  // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 // A row's exponentials use a reference max that is only raised when the tile max exceeds it by
@@ -629,17 +643,36 @@ __device__ __forceinline__ void tile_softmax(const PrefillArgs& a, unsigned char
 
 // Control word written by thread 0 before each step of the CTA: a tile index, or one of these.
 constexpr int kJobExit = -1;    // the CTA is done
-constexpr int kJobDecode = -2;  // a round of split-K items (warps 0-7)
+constexpr int kJobDecode = -2;  // a round of split-K items
 constexpr int kJobNone = -3;    // nothing in this step
+constexpr int kJobTilesDone = -4;  // no tile is left
+
+// A round of split-K items: this warp takes tickets until none is left.
+template <typename T, int DEC>
+__device__ __forceinline__ void item_round(const DecodeArgs& d, const CUtensorMap* tm_kb, const CUtensorMap* tm_vb,
+                                           unsigned char* smem, volatile int* abort_flag, int warp, int lane) {
+    using R = ItemRound<DEC>;
+    int first = 0;
+    if (lane == 0) first = atomicAdd(&d.work[0], 1);
+    first = __shfl_sync(FULL_MASK, first, 0);
+    uint64_t* dbars = reinterpret_cast<uint64_t*>(smem + OFF_DBAR) + warp * kDecodeStages;
+    volatile int* fifo = reinterpret_cast<volatile int*>(smem + OFF_FIFO) + warp * mma::kFifo;
+    if (!mma::decode_warp<T, kDecodeStages, DEC == 2, R::kQreg>(d, tm_kb, tm_vb, smem + warp * kDecodeStages * R::kStageBytes,
+                                                                 dbars, fifo, first, 0) &&
+        lane == 0)
+        *abort_flag = 1;
+    fence_proxy_async_smem();   // its generic writes (zeroed V rows) before later TMA writes
+}
 
 // Persistent CTAs (one per SM) over the batch's tcgen05 tiles and, in a mixed batch, its split-K
 // work items: tiles come from a ticket counter (a.work[2], longest first), items from the split-K
 // counter (d.work[0]). A CTA b < a.decode_ctas first serves items until none is left; every CTA
 // then serves tiles until none is left, then items again if any remain. So the HBM-bound items and
 // the tensor-bound tiles run side by side, and whichever queue empties first hands its CTAs to the
-// other. In a round of items, warps 0-7 each run the warp-MMA loop over two stages carved from the
-// tile buffers (the third warpgroup waits). The last CTA to finish (a.work[3] counts them) resets
-// the counters for the next launch.
+// other. In a round of items, warps run the warp-MMA loop over two stages each, carved from the
+// tile buffers: all twelve for items of at most 8 (row, head) slots (every warp at kItemRegs
+// registers for the round), warps 0-7 otherwise (the third warpgroup waits). The last CTA to finish
+// (a.work[3] counts them) resets the counters for the next launch.
 template <typename T, int POLY, int DEC>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const PrefillArgs a, const DecodeArgs d, const __grid_constant__ CUtensorMap tm_q,
@@ -664,6 +697,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
+    // Items of at most 8 slots run on all twelve warps at the launch's register count, so their
+    // rounds come before and after the register split; items of up to 16 slots need more registers
+    // and run on the softmax warps inside it.
+    constexpr bool kAllWarps = ItemRound<DEC>::kWarps > 8;
+    [[maybe_unused]] auto items_left = [&]() {
+        return d.num_items > 0 && *reinterpret_cast<volatile int*>(&d.work[0]) < d.num_items && !*abort_flag;
+    };
+    // One step of items, between the two CTA barriers of a step (below): thread 0 decides whether
+    // there are items to serve (in the first round only on the CTAs that start on items), then the
+    // item warps serve them until none is left.
+    [[maybe_unused]] auto item_step = [&](bool first_round) {
+        if (threadIdx.x == 0)
+            *ctrl = ((!first_round || (int)blockIdx.x < a.decode_ctas) && items_left()) ? kJobDecode : kJobNone;
+        cta_sync();                                   // (1)
+        if (*ctrl == kJobDecode && warp < ItemRound<DEC>::kWarps)
+            item_round<T, DEC>(d, &tm_kb, &tm_vb, smem, abort_flag, warp, lane);
+        tc_fence_before();
+        cta_sync();                                   // (2)
+    };
+    // The end of the CTA: TMEM back, and the last CTA resets the counters for the next launch.
+    auto finish = [&]() {
+        if (warp == 0) {
+            tc_fence_after();
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        }
+        if (threadIdx.x == 0) {
+            __threadfence();
+            if (atomicAdd(&a.work[3], 1) == (int)gridDim.x - 1) {
+                atomicExch(&a.work[2], 0);
+                atomicExch(&a.work[3], 0);
+                if (d.num_items > 0) atomicExch(&d.work[0], 0);
+            }
+        }
+    };
+    // (a) CTAs that start on items: a round of them first.
+    if constexpr (kAllWarps) item_step(true);
     // Register split: the third warpgroup (producer, MMA issuer, two idle warps) shrinks to
     // kOtherRegs, the softmax warpgroups grow to kSoftmaxRegs. Each warpgroup runs in its own branch;
     // every step is bracketed by two CTA barriers: (1) thread 0 has written the step into *ctrl,
@@ -684,38 +753,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             cta_sync();                                   // (2)
+            if (kAllWarps && job == kJobTilesDone) break;
         }
+        if constexpr (kAllWarps) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kItemRegs));
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        // A round of split-K items: this warp takes tickets until none is left.
-        [[maybe_unused]] auto decode_round = [&]() {
-            int first = 0;
-            if (lane == 0) first = atomicAdd(&d.work[0], 1);
-            first = __shfl_sync(FULL_MASK, first, 0);
-            uint64_t* dbars = reinterpret_cast<uint64_t*>(smem + OFF_DBAR) + warp * kDecodeStages;
-            volatile int* fifo = reinterpret_cast<volatile int*>(smem + OFF_FIFO) + warp * mma::kFifo;
-            if (!mma::decode_warp<T, kDecodeStages, DEC == 2>(d, &tm_kb, &tm_vb, smem + warp * kDecodeStages * mma::kStage,
-                                                               dbars, fifo, first, 0) &&
-                lane == 0)
-                *abort_flag = 1;
-            fence_proxy_async_smem();   // its generic writes (zeroed V rows) before later TMA writes
-        };
-        [[maybe_unused]] auto items_left = [&]() {
-            return d.num_items > 0 && *reinterpret_cast<volatile int*>(&d.work[0]) < d.num_items && !*abort_flag;
-        };
-        // (a) CTAs that start on items: a round of them first.
-        if constexpr (DEC != 0) {
-            if (threadIdx.x == 0) *ctrl = ((int)blockIdx.x < a.decode_ctas && items_left()) ? kJobDecode : kJobNone;
-            cta_sync();                                   // (1)
-            if (*ctrl == kJobDecode) decode_round();
-            tc_fence_before();
-            cta_sync();                                   // (2)
-        }
+        if constexpr (DEC != 0 && !kAllWarps) item_step(true);
         // (b) tiles, longest first, while any is left.
         int bset_seq = 1;   // thread 0: the barrier set of the last tile (tiles alternate between two)
         while (true) {
             if (threadIdx.x == 0) {
-                int t = kJobNone;
+                int t = kJobTilesDone;
                 if (!*abort_flag && *reinterpret_cast<volatile int*>(&a.work[2]) < a.num_tiles) {
                     t = atomicAdd(&a.work[2], 1);
                     if (t < a.num_tiles) {
@@ -727,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<volatile int*>(smem + OFF_BSET) = bset_seq;
                         init_tile_barriers(bars + bset_seq * NUM_BARS);
                     }
-                    else t = kJobNone;
+                    else t = kJobTilesDone;
                 }
                 *ctrl = t;
             }
@@ -743,28 +791,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             cta_sync();                                   // (2)
             if (job < 0) break;
         }
-        // (c) the items still left once the tiles are gone.
-        if constexpr (DEC != 0) {
-            if (threadIdx.x == 0) *ctrl = items_left() ? kJobDecode : kJobNone;
+        if constexpr (kAllWarps) {
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kItemRegs));
+        } else {
+            // (c) the items still left once the tiles are gone; then the third warpgroup leaves.
+            if constexpr (DEC != 0) item_step(false);
+            if (threadIdx.x == 0) *ctrl = kJobExit;
             cta_sync();                                   // (1)
-            if (*ctrl == kJobDecode) decode_round();
-            tc_fence_before();
-            cta_sync();                                   // (2)
+            finish();
         }
-        if (threadIdx.x == 0) *ctrl = kJobExit;
-        cta_sync();                                       // (1)
-        if (warp == 0) {
-            tc_fence_after();
-            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
-        }
-        if (threadIdx.x == 0) {
-            __threadfence();
-            if (atomicAdd(&a.work[3], 1) == (int)gridDim.x - 1) {
-                atomicExch(&a.work[2], 0);
-                atomicExch(&a.work[3], 0);
-                if (d.num_items > 0) atomicExch(&d.work[0], 0);
-            }
-        }
+    }
+    if constexpr (kAllWarps) {
+        // (c) the items still left once the tiles are gone, on all twelve warps again.
+        item_step(false);
+        finish();
     }
 }
 
