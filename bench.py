@@ -104,9 +104,13 @@ def recorded_traffic(kernel: str, workload: str):
         rec = data.get(f"{kernel}@{workload}") or data.get(kernel)
         if not rec or rec.get("workload") != workload:
             return None
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-                return None
+        # the kernel's source files (one "source", or "sources" hashed in order as one byte string)
+        h = hashlib.sha256()
+        for src in rec.get("sources") or [rec["source"]]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
         return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
     except (OSError, ValueError, KeyError):
         return None
