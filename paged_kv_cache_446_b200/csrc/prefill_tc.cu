@@ -20,11 +20,13 @@
 //   warps 10-11 idle; they complete the third warpgroup, whose registers move to the softmax
 //              warpgroups (setmaxnreg).
 // The CTAs are persistent (one per SM): they take tiles, longest first, from a ticket counter. In a
-// mixed batch they also serve the split-K decode items (warps 0-7 run the warp-MMA loop of
-// decode_mma.cuh over buffers carved from the tile stages), so the HBM-bound decode rows and the
-// tensor-bound tiles share the GPU in one launch.
-// A softmax thread reads its row's key tile in two halves of 64 columns (one TMEM round trip each)
-// and signals each half's P separately. O accumulates in TMEM across key tiles. A row's
+// mixed batch they also serve the split-K decode items (the warp-MMA loop of decode_mma.cuh over
+// buffers carved from the tile stages: all twelve warps for items of at most 8 (row, head) slots,
+// warps 0-7 for larger items), so the HBM-bound decode rows and the tensor-bound tiles share the
+// GPU in one launch.
+// A softmax thread reads its row's whole key tile from TMEM in one round trip, then works on it
+// in two halves of 64 columns and signals each half's P separately. O accumulates in TMEM across
+// key tiles. A row's
 // exponentials use a reference maximum that is raised only when a half's maximum exceeds it by
 // 2^8; O is then rescaled in TMEM (exact: softmax is shift invariant, and p stays <= 2^8). The
 // half's maximum is only taken when the weights' sum against the current reference shows that a

@@ -432,6 +432,29 @@ def test_overlapped_mixed_batch(dev, decode_sms):
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("dtype,Hq,Hkv,specs,rows_per_item,slots", [
+    # 16 query heads per KV head: 16-slot items, served by warps 0-7 inside the register split
+    ("bf16", 32, 2, [(300, 70), (0, 130)] + [(400 + 97 * i, 1) for i in range(6)], 0, 16),
+    # verify rows of 2 tokens at G = 4: 8-slot items of two rows, served by all twelve warps
+    ("f16", 16, 4, [(250, 64), (33, 48)] + [(300 + 211 * i, 2) for i in range(5)], 2, 8),
+])
+@pytest.mark.parametrize("decode_sms", [3, 37])
+def test_overlapped_mixed_batch_item_forms(dev, dtype, Hq, Hkv, specs, rows_per_item, slots, decode_sms):
+    """One persistent launch over tiles and split-K items in both item forms the launch can take,
+    with short split chunks so every CTA sees many items: within tolerance of the oracle and bit
+    for bit the two kernels run one after the other."""
+    wl = custom(dev, dtype, Hq, Hkv, 128, specs, seed=41 + decode_sms)
+    opts = dict(decode_sms=decode_sms, split_blocks=3, rows_per_item=rows_per_item)
+    _, step = run_and_compare(wl, dev, **opts)
+    p = step.plan.plan
+    assert p.num_tiles > 0 and p.num_items > 0 and p.decode_sms == decode_sms and p.decode_kernel == 2
+    assert max(1, p.rows_per_item) * min(p.heads_per_item, Hq // Hkv) == slots
+    a = step.run(wl.q, wl.k_pool, wl.v_pool, wl.scale).clone()
+    b = make_step(wl, dev, **dict(opts, decode_sms=-1)).run(wl.q, wl.k_pool, wl.v_pool, wl.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
 @pytest.mark.parametrize("config", ["c2", "c4", "c5"])
 def test_plan_reused_across_launches(dev, config):
     """One plan run many times in a row (as every layer of a model step does): the split-K kernel's
