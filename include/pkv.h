@@ -145,8 +145,9 @@ typedef struct pkv_plan_options {
      * persistent CTAs (one per SM) serve both queues in one launch -- decode_sms of them start on
      * the split-K items and the others on the tiles, and each turns to the other queue once its own
      * is empty -- so the tensor-bound tiles and the HBM-bound items share the GPU. 0 = sized by the
-     * planner from the two parts' estimated times; -1 = no overlap (the split-K kernel runs after
-     * the tiles). */
+     * planner, which simulates the greedy tile schedule beside the items' streaming for splits
+     * near the balanced share and takes the middle of the near-best run; -1 = no overlap (the
+     * split-K kernel runs after the tiles). */
     int32_t decode_sms;
 } pkv_plan_options;
 

@@ -388,3 +388,37 @@ def test_mma_items_longest_first_for_greedy_warps(pkv, config, num_sms):
     finish = max(t for t, _ in heap)
     mean = (lens + 1).sum() / W_
     assert finish <= max(1.1 * mean, mean + lens.max() + 1)
+
+
+def test_mixed_split_choice(pkv):
+    """The split of a mixed batch's SMs between split-K items and tcgen05 tiles: a batch with both
+    gets 1 .. S-1 item CTAs from the planner (none when one part is missing), the same batch with
+    twice the decode context does not get fewer, and an explicit split is honoured (clamped to
+    S - 1; -1 runs the two kernels one after the other)."""
+    from paged_kv_cache_446_b200 import workloads as W
+    wl = W.make("c5", with_tensors=False)
+    prior = np.asarray(wl.prior_lens)
+    is_dec = np.array([n == 1 for n in wl.batch.values()])
+
+    def split(prior_lens, num_sms=148, **opts):
+        qsl, ctx = pkv.flatten_batch(wl.batch, prior_lens)
+        p, _ = pkv.plan_host(qsl, ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, with_meta=False,
+                             num_sms=num_sms, **opts)
+        assert p.num_tiles > 0 and p.num_items > 0
+        return p.decode_sms
+
+    base = split(prior)
+    assert 1 <= base <= 147
+    doubled = prior.copy()
+    doubled[is_dec] *= 2
+    assert split(doubled) >= base
+    assert 1 <= split(prior, num_sms=132) <= 131
+    assert split(prior, decode_sms=10) == 10
+    assert split(prior, decode_sms=500) == 147
+    assert split(prior, decode_sms=-1) == 0
+    for part, cfg in (("prefill", "c5"), ("all", "c2")):
+        w = W.make(cfg, with_tensors=False, part=part) if part != "all" else W.make(cfg, with_tensors=False)
+        qsl, ctx = pkv.flatten_batch(w.batch, w.prior_lens)
+        p, _ = pkv.plan_host(qsl, ctx, w.num_q_heads, w.num_kv_heads, w.head_dim, w.dtype, with_meta=False,
+                             num_sms=148)
+        assert p.decode_sms == 0
