@@ -4,7 +4,6 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
-#include <map>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -89,22 +88,29 @@ int tile_tokens(int group) { return 2 * (128 / group); }
 // When the last tile ends if the tiles (longest first, as the ticket counter hands them out) each
 // go to the CTA that frees first: `ctas` CTAs, `late` of which free only at t_late. Durations and
 // loads are whole ticks. Tiles of equal length form runs (ticks, count) and CTAs of equal load form
-// groups (load -> count), so a run is dealt to whole groups at once and the cost grows with the
-// distinct lengths and loads, not with the tiles.
+// groups (load, count), kept in `load` sorted by decreasing load (the least loaded group last), so
+// a run is dealt to whole groups at once and the cost grows with the distinct lengths and loads,
+// not with the tiles.
 int64_t greedy_end(const std::vector<std::pair<int64_t, int>>& runs, int ctas, int late, int64_t t_late,
-                   std::map<int64_t, int>& load) {
+                   std::vector<std::pair<int64_t, int>>& load) {
     load.clear();
-    if (ctas > late) load[0] += ctas - late;
-    if (late > 0) load[t_late] += late;
+    if (late > 0) load.push_back({t_late, late});
+    if (ctas > late) load.push_back({0, ctas - late});
     int64_t end = late > 0 ? t_late : 0;
+    const auto add = [&](int64_t l, int k) {  // k CTAs at load l, merged into an equal group if any
+        auto it = std::lower_bound(load.begin(), load.end(), l,
+                                   [](const std::pair<int64_t, int>& g, int64_t v) { return g.first > v; });
+        if (it != load.end() && it->first == l) it->second += k;
+        else load.insert(it, {l, k});
+    };
     for (const auto& run : runs) {
         for (int n = run.second; n > 0;) {
-            auto g = load.begin();
-            const int64_t l = g->first;
-            const int k = std::min(g->second, n);
+            std::pair<int64_t, int>& g = load.back();
+            const int64_t l = g.first;
+            const int k = std::min(g.second, n);
             n -= k;
-            if ((g->second -= k) == 0) load.erase(g);
-            load[l + run.first] += k;
+            if ((g.second -= k) == 0) load.pop_back();
+            add(l + run.first, k);
             end = std::max(end, l + run.first);
         }
     }
@@ -136,10 +142,10 @@ int mixed_split(const std::vector<PrefillTile>& tiles, int64_t item_bytes, int64
     const double warps_per_sm = item_slots <= 8 ? 12.0 : 8.0;
     if (tiles.empty() || num_items <= 0) return 0;
     static thread_local std::vector<std::pair<int64_t, int>> runs;
-    static thread_local std::map<int64_t, int> load;
+    static thread_local std::vector<std::pair<int64_t, int>> load;
     // Ticks of 1/96 of the longest tile: coarse enough that equal loads recur (the simulation then
-    // adds ~10 % to the planner's time on that batch), fine enough that a CTA's few tiles add up to
-    // within ~1 % (at 1/64 the choice there moved to 50).
+    // takes ~85 us of host time on that batch), fine enough that a CTA's few tiles add up to within
+    // ~1 % (at 1/64 the choice there moved to 50).
     int max_kt = 1;
     for (const PrefillTile& t : tiles) max_kt = std::max(max_kt, t.key_tiles);
     const double tick = max_kt * kKeyTileSec / 96.0;
