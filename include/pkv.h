@@ -185,8 +185,13 @@ typedef struct pkv_plan {
     int32_t decode_sms;          /* > 0: one launch of the tile kernel also serves the split-K items,
                                     with this many CTAs starting on them; 0: the split-K kernel runs
                                     after the tiles */
-    int32_t pad0;
+    uint32_t flags;              /* PKV_PLAN_* bits below */
 } pkv_plan;
+
+/* pkv_plan.flags: every K/V block the split-K items read is read by exactly one item (no shared-
+ * prefix group, one item per KV head's query group and per request's rows), so the split-K kernel
+ * may mark those reads to leave L2 first. */
+#define PKV_PLAN_SINGLE_READ 1u
 
 /*
  * pkv_attention_workspace_size -- bytes of device workspace pkv_attention_plan will need for this

@@ -241,6 +241,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     core_rows.reserve(R > 0 ? (size_t)qsl[R] : 0);
     int64_t kv_bytes = 0, flops = 0, tile_kv = 0, tile_flops = 0;
     int decode_rows = 0, prefill_rows = 0, max_blocks = 0;
+    bool rows_split = false;  // some request's rows span several items (each reads the same blocks)
     for (int r = 0; r < R; ++r) {
         const int n = qsl[r + 1] - qsl[r];
         if (n == 0) continue;
@@ -264,6 +265,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
                 }
         } else {
             if (n == 1) ++decode_rows;
+            if (n > rpi) rows_split = true;
             for (int j = 0; j < n; j += rpi) {
                 const int nr = std::min(rpi, n - j);
                 core_rows.push_back(CoreRow{qsl[r] + j, r, P + j + 1, nr, 0, (int)ceil_div(P + j + nr, kBlockSize), 0, -1, 0});
@@ -518,6 +520,7 @@ pkv_status plan_lists(const int32_t* qsl, const int32_t* ctx, int R, int Hq, int
     plan->core_kv_bytes = kv_bytes - tile_kv - shared_saved_tokens * Hkv * 2 * D * eb;
     plan->tile_kv_bytes = tile_kv;
     plan->tile_flops = tile_flops;
+    if (grps.empty() && ceil_div(G, hpi) == 1 && !rows_split) plan->flags |= PKV_PLAN_SINGLE_READ;
     // Mixed batch: the tcgen05 kernel's persistent CTAs (one per SM) also serve the warp-MMA items;
     // decode_sms of them start on items, the rest on tiles, and each turns to the other queue when
     // its own empties.
@@ -840,6 +843,10 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_pool, con
     d.part_stride = plan->part_stride;
     d.scale_log2 = scale_log2;
     d.pdl = true;
+    // Streamed once, the split-K kernel's K/V may leave L2 first (measured: c2, c3 and c6 steps 3-4 %
+    // faster; the small kernels around it keep their data in L2). Not in the mixed launch, where
+    // it measured 0.8 % slower.
+    d.evict_first = !mixed && (plan->flags & PKV_PLAN_SINGLE_READ) != 0;
     pkv_status st = PKV_OK;
     if (plan->num_tiles > 0) {
         PrefillArgs a{};

@@ -47,13 +47,21 @@ constexpr int kStage = kKV + kQ;               // 12 KiB, a multiple of the 1 Ki
 constexpr int kFifo = 8;                       // items a warp's producer may run ahead (> NSTAGE)
 
 // K or V of one KV block (16 pool rows from row y) in one copy, both 64-column halves, through a
-// map made by encode_block_halves.
-__device__ __forceinline__ void tma_load_block(void* dst, const CUtensorMap* map, int y, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
-            smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(0), "r"(smem_u32(bar))
-        : "memory");
+// map made by encode_block_halves; with `hint`, under the L2 cache policy `policy`.
+__device__ __forceinline__ void tma_load_block(void* dst, const CUtensorMap* map, int y, uint64_t* bar, bool hint,
+                                               uint64_t policy) {
+    if (hint)
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(
+                smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(0), "r"(smem_u32(bar)), "l"(policy)
+            : "memory");
+    else
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+                smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(0), "r"(smem_u32(bar))
+            : "memory");
 }
 
 // Byte offset, inside a 16-row chunk stored as two 64-column halves with the 128-byte swizzle, of
@@ -126,6 +134,8 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
     __syncwarp();
     if (first >= a.num_items) return true;
     const unsigned char* qp = static_cast<const unsigned char*>(a.q);
+    uint64_t l2_policy = 0;   // evict first: every K/V block is read by one item
+    if (a.evict_first) asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(l2_policy));
     const int g = lane >> 2;       // fragment row
     const int c4 = lane & 3;       // fragment column pair
     // QREG: item it's q rows as this lane's B fragments (slot g, words kk * 8 + c4 and + 4; zero
@@ -181,8 +191,8 @@ __device__ __forceinline__ bool decode_warp(const DecodeArgs& a, const CUtensorM
             const uint32_t qbytes = first ? qrow * (uint32_t)pi.num_rows : 0u;
             mbar_arrive_expect_tx(&bars[stage], (uint32_t)kKV + qbytes);
             const int y = (id * a.num_kv_heads + pi.kv_head) * kBlockSize;  // first pool row of the chunk
-            tma_load_block(st, tm_k, y, &bars[stage]);
-            tma_load_block(st + 2 * kHalf, tm_v, y, &bars[stage]);
+            tma_load_block(st, tm_k, y, &bars[stage], a.evict_first, l2_policy);
+            tma_load_block(st + 2 * kHalf, tm_v, y, &bars[stage], a.evict_first, l2_policy);
             if (first) {
                 for (int j = 0; j < pi.num_rows; ++j) {
                     const size_t qoff =

@@ -84,6 +84,8 @@ struct DecodeArgs {
     int part_stride;     // slots per partial-result entry (8 for the FMA kernel, 16 for the MMA kernel)
     float scale_log2;    // scale * log2(e)
     bool pdl;            // launch with programmatic dependent launch (false after an event wait)
+    bool evict_first;    // the warp-MMA kernel's K/V copies carry an L2 evict-first hint (every
+                         // block is read by one item: nothing is lost by letting it leave L2 first)
 };
 
 struct MergeArgs {

@@ -50,7 +50,7 @@ class Plan(ctypes.Structure):
         "max_blocks", "heads_per_item", "rows_per_item", "decode_kernel", "part_stride", "merge_slots")] + [(n, ctypes.c_int64) for n in (
         "off_items", "off_tiles", "off_merge", "off_part_o", "off_part_ml", "meta_bytes", "ws_bytes", "kv_bytes",
         "attn_flops", "core_kv_bytes", "tile_kv_bytes", "tile_flops")] + [
-        ("decode_sms", ctypes.c_int32), ("pad0", ctypes.c_int32)]
+        ("decode_sms", ctypes.c_int32), ("flags", ctypes.c_uint32)]
 
 
 def _sig(name, restype, argtypes):

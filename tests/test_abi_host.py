@@ -422,3 +422,22 @@ def test_mixed_split_choice(pkv):
         p, _ = pkv.plan_host(qsl, ctx, w.num_q_heads, w.num_kv_heads, w.head_dim, w.dtype, with_meta=False,
                              num_sms=148)
         assert p.decode_sms == 0
+
+
+def test_single_read_flag(pkv):
+    """PKV_PLAN_SINGLE_READ (the split-K kernel may let its K/V leave L2 first) is set only when
+    every K/V block the items read is read by one item: not with shared-prefix groups, not when a
+    KV head's query group spans several items, not when a request's rows do."""
+    from paged_kv_cache_446_b200 import workloads as W
+
+    def flags(cfg, **opts):
+        wl = W.make(cfg, with_tensors=False)
+        qsl, ctx = pkv.flatten_batch(wl.batch, wl.prior_lens)
+        p, _ = pkv.plan_host(qsl, ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.dtype, with_meta=False,
+                             num_sms=148, shared_tables=wl.block_tables, **opts)
+        return p.flags & 1
+
+    assert flags("c2") == 1 and flags("c3") == 1 and flags("c6") == 1
+    assert flags("c4") == 0                          # shared-prefix groups
+    assert flags("c3", heads_per_item=2) == 0        # G = 4 over two items per KV head
+    assert flags("c6", rows_per_item=2) == 0         # 5 verify rows over three items
