@@ -19,9 +19,10 @@
 //
 // Per warp and block: K and V of one (block, KV head) -- 16 rows of 128 elements -- arrive by one
 // tensor-map TMA copy each (both 64-column halves through a 3-D view of the pool, 128-byte
-// swizzle, so ldmatrix reads are free of bank conflicts; the copies' issue is a large share of a
-// warp's time per block, so one copy per operand rather than one per half) into a ring of shared-memory stages tracked by mbarriers; the item's q rows come
-// once by plain bulk copies. S = Q K^T as 16 MMAs (two 8-token n-tiles x 8 k-steps); the online
+// swizzle, so ldmatrix reads are free of bank conflicts; issuing the copies is a large share of a
+// warp's time per block, so one copy per operand rather than one per half) into a ring of
+// shared-memory stages tracked by mbarriers; the item's q rows come once per item, by plain bulk
+// copies into the stage (or, with QREG, straight into registers). S = Q K^T as 16 MMAs (two 8-token n-tiles x 8 k-steps); the online
 // softmax runs on the accumulator fragments in the log2 domain (a slot's scores sit in one lane
 // quad); P, rounded to the input type, is reused in registers as the A operand of P V (16 MMAs
 // over 8-column n-tiles, V fragments by transposing ldmatrix). Masking follows each slot's own
