@@ -42,13 +42,31 @@ __global__ void __launch_bounds__(128) slot_mapping_kernel(const int32_t* __rest
     }
 }
 
-// One thread per 16-byte chunk of one (token, KV head) row, for K and for V.
+// 16 bytes from src (read under L2 policy `rd`) to dst (written under `wr`).
+__device__ __forceinline__ void copy16(uint4* dst, const uint4* src, uint64_t rd, uint64_t wr) {
+    uint4 x;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
+                 : "l"(src), "l"(rd));
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "r"(x.x), "r"(x.y), "r"(x.z),
+                 "r"(x.w), "l"(wr)
+                 : "memory");
+}
+
+// One thread per 16-byte chunk of one (token, KV head) row, for K and for V. The new K/V is read
+// once (an L2 evict-first policy lets it go first); the pool rows written stay in L2 longer (evict
+// last), where the attention kernels that follow read them (measured: the 32 k-token append of
+// the parallel-sampling batch 45.9 -> 43.9 us and its decode 53.6 -> 51.2 us; the 64-row decode
+// step unchanged; evict-first loads alone were slower).
 __global__ void __launch_bounds__(256) kv_write_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                                                        uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
                                                        const int64_t* __restrict__ slots, long long num_chunks,
                                                        int num_kv_heads, int cpr, long long num_slots,
                                                        DeviceError* err) {
     griddep_wait();
+    uint64_t read_once, keep;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(read_once));
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
     const long long per_token = (long long)num_kv_heads * cpr;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < num_chunks;
          i += (long long)gridDim.x * blockDim.x) {
@@ -64,8 +82,8 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const uint4* __restrict__
         }
         const long long blk = slot / kBlockSize, off = slot % kBlockSize;
         const long long dst = ((blk * num_kv_heads + h) * kBlockSize + off) * cpr + c;
-        k_pool[dst] = __ldg(k_new + i);
-        v_pool[dst] = __ldg(v_new + i);
+        copy16(k_pool + dst, k_new + i, read_once, keep);
+        copy16(v_pool + dst, v_new + i, read_once, keep);
     }
 }
 
