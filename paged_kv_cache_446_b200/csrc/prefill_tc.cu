@@ -720,9 +720,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // The end of the CTA: TMEM back, and the last CTA resets the counters for the next launch.
     auto finish = [&]() {
-        if (warp == 0) {
+        if (threadIdx.x < 32) {   // warp 0; the TMEM address is read again rather than kept live
             tc_fence_after();
-            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+            const uint32_t t = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(t), "r"(kTmemCols) : "memory");
         }
         if (threadIdx.x == 0) {
             __threadfence();
